@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA hot path on B200 (one process per GPU).
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  prefill of a 131072-token sequence (indexer + top-2048 + sparse GQA
+  attention: dsa_index_topk, dsa_sparse_attn_prefill), then
+  one decode step of 64 sequences with cached lengths ~ U[32768, 262144]
+  (dsa_sparse_attn_decode).
+`value` is prefill query-tokens/s over the device time of the prefill part of
+the step; the decode part is reported as decode tokens/s.  Inputs are resident
+in HBM when the timed region starts; L2 is flushed (256 MiB write) between
+timed steps, outside the per-step events.  With torchrun every rank runs its
+own independent workload (weak scaling, no collective on the data path).
+
+`--impl reference` times the CPU oracle (the reference arm of this build) on a
+bounded sample of the same workload and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gen  # noqa: E402
+
+METRIC = ("prefill query-tokens/s & decode tokens/s at 128K ctx, k=2048; "
+          "% FP8/HBM roofline")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefill-config", type=int, default=3)
+    ap.add_argument("--decode-config", type=int, default=4)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return dict(hbm=float(m["hbm_gbs"]), bf16=float(m["bf16_tflops"]),
+                    bf16_sus=float(m["bf16_tflops_sustained"]), src="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------------ work model
+
+def prefill_flops(cfg) -> float:
+    """Indexer: 2 * H_I * d_I FLOP per causal (t, s) pair."""
+    return 2.0 * cfg.H_I * cfg.d_I * cfg.L * (cfg.L + 1) / 2.0
+
+
+def prefill_attn_bytes(cfg) -> float:
+    """Gather: 2 * Hkv * d * 2 bytes per selected row, plus Q, O and the index row."""
+    L, k = cfg.L, cfg.k
+    sel = k * L - k * (k - 1) / 2.0 if L >= k else L * (L + 1) / 2.0  # sum_t min(k, t+1)
+    row = 2 * cfg.Hkv * cfg.d * 2
+    per_tok = 2 * cfg.Hq * cfg.d * 2 + 4 * k
+    return sel * row + L * per_tok
+
+
+def decode_bytes(cfg, lens) -> float:
+    """k_I scan (d_I bytes per cached key) + gathered K/V rows + queries/outputs."""
+    sel = float(np.minimum(lens, cfg.k).sum())
+    return (float(lens.sum()) * cfg.d_I + sel * 2 * cfg.Hkv * cfg.d * 2
+            + cfg.B * (cfg.H_I * cfg.d_I + cfg.H_I * 4 + 2 * 2 * cfg.Hq * cfg.d))
+
+
+# ------------------------------------------------------------------ clocks
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in open(self.path):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return dict(sm_mhz=statistics.median(sm) if sm else None,
+                    sm_max_mhz=max(smax) if smax else None, reasons=sorted(reasons),
+                    samples=len(sm))
+
+
+# ------------------------------------------------------------------ our arm
+
+def upload(torch, a: np.ndarray, dtype=None, pin=False):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.view(dtype)
+    if pin:
+        t = t.pin_memory()
+    return t.cuda(non_blocking=False), t
+
+
+def build_prefill(torch, cfg, keep_host: bool):
+    import sparse_long_context_02_b200 as dsa  # noqa: F401
+    host = gen.prefill_inputs(cfg)
+    dev, pinned = {}, {}
+    for name, dt in (("q_I", None), ("k_I", None), ("w", None), ("Q", torch.bfloat16),
+                     ("K", torch.bfloat16), ("V", torch.bfloat16)):
+        dev[name], h = upload(torch, host[name], dt, pin=keep_host)
+        if keep_host:
+            pinned[name] = h
+    dev["idx"] = torch.empty((cfg.L, cfg.k), dtype=torch.int32, device="cuda")
+    dev["O"] = torch.empty((cfg.L, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda")
+    return dev, pinned, host
+
+
+def build_decode(torch, cfg, keep_host: bool):
+    import sparse_long_context_02_b200 as dsa
+    off = gen.decode_offsets(cfg)
+    N = int(off[-1])
+    q = gen.decode_queries(cfg)
+    dev, pinned = {}, {}
+    for name, dt in (("q_I", None), ("w", None), ("Q", torch.bfloat16)):
+        dev[name], h = upload(torch, q[name], dt, pin=keep_host)
+        if keep_host:
+            pinned[name] = h
+    dev["cache_off"], h = upload(torch, off, None, pin=keep_host)
+    if keep_host:
+        pinned["cache_off"] = h
+    # caches: generated in row blocks straight into device memory
+    dev["kI_cache"] = torch.empty((N, cfg.d_I), dtype=torch.uint8, device="cuda")
+    dev["K_cache"] = torch.empty((N, cfg.Hkv, cfg.d), dtype=torch.bfloat16, device="cuda")
+    dev["V_cache"] = torch.empty((N, cfg.Hkv, cfg.d), dtype=torch.bfloat16, device="cuda")
+    step = 1 << 19
+    for r0 in range(0, N, step):
+        r1 = min(N, r0 + step)
+        dev["kI_cache"][r0:r1].copy_(torch.from_numpy(gen.decode_kI_rows(cfg, r0, r1)))
+        dev["K_cache"][r0:r1].copy_(torch.from_numpy(
+            gen.decode_K_rows(cfg, r0, r1).view(np.int16)).view(torch.bfloat16))
+        dev["V_cache"][r0:r1].copy_(torch.from_numpy(
+            gen.decode_V_rows(cfg, r0, r1).view(np.int16)).view(torch.bfloat16))
+    dev["O"] = torch.empty((cfg.B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda")
+    dev["idx"] = torch.empty((cfg.B, cfg.k), dtype=torch.int32, device="cuda")
+    need = dsa.decode_workspace_size(cfg.B, N, cfg.H_I, cfg.d_I, cfg.k, cfg.Hq, cfg.Hkv, cfg.d)
+    dev["ws"] = torch.empty(need, dtype=torch.uint8, device="cuda")
+    return dev, pinned, off
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as tdist
+    import sparse_long_context_02_b200 as dsa
+
+    torch.cuda.set_device(local_rank)
+    pcfg = gen.CONFIGS[args.prefill_config]
+    dcfg = gen.CONFIGS[args.decode_config]
+    if world > 1:  # independent problem per rank
+        pcfg = pcfg.with_(seed=pcfg.seed_ + 1000 * rank)
+        dcfg = dcfg.with_(seed=dcfg.seed_ + 1000 * rank)
+    keep_host = not args.no_e2e
+    P, Ph, p_host = build_prefill(torch, pcfg, keep_host)
+    D, Dh, off = build_decode(torch, dcfg, keep_host)
+    lens = np.diff(off)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def prefill():
+        dsa.index_topk(P["q_I"], P["k_I"], P["w"], pcfg.k, idx=P["idx"], stream=stream)
+
+    def attn():
+        dsa.sparse_attn_prefill(P["Q"], P["K"], P["V"], P["idx"], pcfg.scale, O=P["O"],
+                                stream=stream)
+
+    def decode():
+        dsa.sparse_attn_decode(D["q_I"], D["w"], D["Q"], D["kI_cache"], D["K_cache"],
+                               D["V_cache"], D["cache_off"], dcfg.k, dcfg.scale, O=D["O"],
+                               idx_out=D["idx"], workspace=D["ws"], stream=stream)
+
+    launches_per_step = 1 + 1 + 5
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        prefill()
+        if ev is not None:
+            ev[1].record(stream)
+        attn()
+        if ev is not None:
+            ev[2].record(stream)
+        decode()
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if dsa.device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = Clocks(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                    else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    if world > 1:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        tdist.barrier()
+    clk = clocks.stop()
+    t_idx = [e[0].elapsed_time(e[1]) for e in evs]
+    t_att = [e[1].elapsed_time(e[2]) for e in evs]
+    t_dec = [e[2].elapsed_time(e[3]) for e in evs]
+    err = dsa.device_error()
+    if err != 0:
+        raise RuntimeError(f"device error {err} in the timed region")
+
+    tot = np.array([sum(t_idx) + sum(t_att), sum(t_dec)], dtype=np.float64)  # ms over K steps
+    if world > 1:
+        tt = torch.tensor(tot, device="cuda")
+        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
+        tot = tt.cpu().numpy()
+    K = args.steps
+    prefill_ms = tot[0] / K
+    decode_ms = tot[1] / K
+    value = world * pcfg.L / (prefill_ms / 1e3)
+    decode_tps = world * dcfg.B / (decode_ms / 1e3)
+
+    # ---- roofline of each kernel, reported for the dominant one
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_sus"]
+    ms_idx, ms_att, ms_dec = (statistics.mean(t_idx), statistics.mean(t_att),
+                              statistics.mean(t_dec))
+    kernels = {
+        "dsa_index_topk": dict(bound="tensor", ms=ms_idx, work=prefill_flops(pcfg),
+                               achieved=prefill_flops(pcfg) / (ms_idx / 1e3) / 1e12,
+                               peak=fp8_peak, unit="TFLOP/s"),
+        "dsa_sparse_attn_prefill": dict(bound="hbm", ms=ms_att, work=prefill_attn_bytes(pcfg),
+                                        achieved=prefill_attn_bytes(pcfg) / (ms_att / 1e3) / 1e9,
+                                        peak=pk["hbm"], unit="GB/s"),
+        "dsa_sparse_attn_decode": dict(bound="hbm", ms=ms_dec, work=decode_bytes(dcfg, lens),
+                                       achieved=decode_bytes(dcfg, lens) / (ms_dec / 1e3) / 1e9,
+                                       peak=pk["hbm"], unit="GB/s"),
+    }
+    for v in kernels.values():
+        v["frac"] = v["achieved"] / v["peak"]
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    dk = kernels[dom]
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get(dom)
+        except ValueError:
+            traffic = None
+    roofline = dict(bound=dk["bound"], achieved=dk["achieved"], peak=dk["peak"], unit=dk["unit"],
+                    frac=dk["frac"], traffic=traffic, kernel=dom,
+                    peak_source=f"{pk['src']} ({'2 x sustained bf16' if dk['bound'] == 'tensor' else 'hbm copy'})")
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if keep_host:
+        O_host = torch.empty(P["O"].shape, dtype=torch.bfloat16).pin_memory()
+        Od_host = torch.empty(D["O"].shape, dtype=torch.bfloat16).pin_memory()
+        h2d_p = sum(v.numel() * v.element_size() for v in Ph.values())
+        h2d_d = sum(v.numel() * v.element_size() for v in Dh.values())
+        d2h_p = O_host.numel() * 2
+        d2h_d = Od_host.numel() * 2
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        if world > 1:
+            tdist.barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.zero_()
+            ev2[i][0].record(stream)
+            for n, h in Ph.items():
+                P[n].copy_(h, non_blocking=True)
+            prefill()
+            attn()
+            O_host.copy_(P["O"], non_blocking=True)
+            ev2[i][1].record(stream)
+            for n, h in Dh.items():
+                D[n].copy_(h, non_blocking=True)
+            decode()
+            Od_host.copy_(D["O"], non_blocking=True)
+            ev2[i][2].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            tdist.barrier()
+        e_p = sum(e[0].elapsed_time(e[1]) for e in ev2)
+        e_d = sum(e[1].elapsed_time(e[2]) for e in ev2)
+        et = np.array([e_p, e_d])
+        if world > 1:
+            tt = torch.tensor(et, device="cuda")
+            tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
+            et = tt.cpu().numpy()
+        e2e = dict(value=world * pcfg.L / (et[0] / K / 1e3), unit="query-tokens/s",
+                   h2d_bytes_per_step=int(h2d_p + h2d_d), d2h_bytes_per_step=int(d2h_p + d2h_d),
+                   decode_value=world * dcfg.B / (et[1] / K / 1e3), decode_unit="tokens/s",
+                   ms_per_step=float((et[0] + et[1]) / K))
+        # result read back: a sanity check that the copy carried real output
+        if not torch.isfinite(O_host.float()).all():
+            raise RuntimeError("non-finite output")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(pcfg, p_host, args.cpu_seconds)
+
+    return dict(value=value, prefill_ms=prefill_ms, decode_ms=decode_ms, decode_tps=decode_tps,
+                clocks=clk, kernels=kernels, roofline=roofline, e2e=e2e, cpu=cpu,
+                launches=launches_per_step * K, pcfg=pcfg, dcfg=dcfg)
+
+
+# ------------------------------------------------------------------ oracle timing
+
+def sample_rows(L, n, seed=0):
+    """n query rows stratified over [0, L): the sample's mean causal length
+    matches the whole sequence's."""
+    rng = np.random.default_rng(seed)
+    return np.array(sorted(int((i + rng.random()) * L / n) for i in range(n)), np.int64)
+
+
+def oracle_prefill_rows(pcfg, host, rows, nthreads=0):
+    import oracle
+    idx = oracle.index_topk(host["q_I"], host["k_I"], host["w"], pcfg.k, rows=rows,
+                            nthreads=nthreads)
+    oracle.sparse_attn(host["Q"], host["K"], host["V"], idx, pcfg.scale, rows=rows,
+                       nthreads=nthreads, idx_by_row=True)
+
+
+def cpu_baseline(pcfg, host, seconds):
+    cores = os.cpu_count() or 1
+    # calibrate on a small stratified sample, then size the timed sample
+    probe = sample_rows(pcfg.L, max(cores, 8), seed=1)
+    t0 = time.perf_counter()
+    oracle_prefill_rows(pcfg, host, probe)
+    dt = time.perf_counter() - t0
+    n = int(max(cores, min(16 * cores, len(probe) * seconds / max(dt, 1e-3))))
+    rows = sample_rows(pcfg.L, n, seed=2)
+    t0 = time.perf_counter()
+    oracle_prefill_rows(pcfg, host, rows)
+    dt = time.perf_counter() - t0
+    return dict(value=n / dt, unit="query-tokens/s", cores=cores, kind="oracle",
+                sample=f"{n} query rows stratified over t in [0, {pcfg.L}) of the "
+                       f"{pcfg.name} workload (indexer + top-k + attention per row), "
+                       f"{dt:.1f} s")
+
+
+def run_reference(args):
+    pcfg = gen.CONFIGS[args.prefill_config]
+    host = gen.prefill_inputs(pcfg)
+    cores = os.cpu_count() or 1
+    probe = sample_rows(pcfg.L, max(cores, 8), seed=1)
+    t0 = time.perf_counter()
+    oracle_prefill_rows(pcfg, host, probe)
+    dt = time.perf_counter() - t0
+    n = int(max(cores, min(16 * cores, len(probe) * 8.0 / max(dt, 1e-3))))
+    for w in range(args.warmup):
+        oracle_prefill_rows(pcfg, host, sample_rows(pcfg.L, max(1, n // 4), seed=100 + w))
+    times = []
+    for i in range(args.steps):
+        rows = sample_rows(pcfg.L, n, seed=10 + i)
+        t0 = time.perf_counter()
+        oracle_prefill_rows(pcfg, host, rows)
+        times.append(time.perf_counter() - t0)
+    value = n * args.steps / sum(times)
+    sample = (f"{n} query rows per step, stratified over t in [0, {pcfg.L}) of the {pcfg.name} "
+              f"workload (indexer + top-k + attention per row)")
+    return dict(impl="reference", metric=METRIC, value=value, unit="query-tokens/s",
+                n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
+                ms_per_step=1e3 * sum(times) / args.steps, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                config=dict(workload=pcfg.name, L=pcfg.L, k=pcfg.k, H_I=pcfg.H_I, d_I=pcfg.d_I,
+                            Hq=pcfg.Hq, Hkv=pcfg.Hkv, d=pcfg.d, seed=pcfg.seed_),
+                cpu_baseline=dict(value=value, unit="query-tokens/s", cores=cores, kind="oracle",
+                                  sample=sample),
+                e2e=dict(value=value, unit="query-tokens/s", h2d_bytes_per_step=0,
+                         d2h_bytes_per_step=0))
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import datetime
+    import torch
+    import torch.distributed as tdist
+    if world > 1:
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        r = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            tdist.destroy_process_group()
+    if rank != 0:
+        return
+    pcfg, dcfg = r["pcfg"], r["dcfg"]
+    out = dict(
+        metric=METRIC, value=r["value"], unit="query-tokens/s", n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=r["prefill_ms"] + r["decode_ms"],
+        higher_is_better=True, scaling="weak", vs_baseline=None, dtype="fp8-e4m3/bf16",
+        data="synthetic",
+        config=dict(workload=f"{pcfg.name} + {dcfg.name}", prefill_L=pcfg.L, k=pcfg.k,
+                    H_I=pcfg.H_I, d_I=pcfg.d_I, Hq=pcfg.Hq, Hkv=pcfg.Hkv, d=pcfg.d,
+                    decode_B=dcfg.B, decode_n=f"U[{dcfg.n_lo},{dcfg.n_hi}]",
+                    parallelism=f"independent problem per rank x{world}",
+                    l2="flushed between timed steps (256 MiB write, outside the events)"),
+        decode=dict(value=r["decode_tps"], unit="tokens/s", ms_per_step=r["decode_ms"]),
+        prefill_ms=r["prefill_ms"],
+        kernels=r["kernels"], roofline=r["roofline"], clocks=r["clocks"],
+        gpu_launches=r["launches"],
+    )
+    if r["e2e"] is not None:
+        out["e2e"] = r["e2e"]
+    if r["cpu"] is not None:
+        out["cpu_baseline"] = r["cpu"]
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,176 @@
+/*
+ * dsa.h - C ABI of the B200 (sm_100a) DeepSeek-Sparse-Attention hot path:
+ * Lightning-Indexer scores -> per-query top-k -> sparse GQA attention, for
+ * prefill and for single-token decode.
+ *
+ * Source of the operations: Kwai Keye-VL-2.0 technical-report summary,
+ * section 1 (a light MQA-style indexer scans the whole context, each query
+ * keeps its 2048 best positions, attention runs over those only, cost falls
+ * from O(L^2) to O(Lk); the base model is GQA) and section 8 (decode-time
+ * sparse attention; a deterministic top-k so that training and inference
+ * select the same keys).  The pages give no formula for the indexer; it is
+ * read as DeepSeek's published one:
+ *
+ *     I[t,s] = sum_j w[t,j] * max(0, sum_c qI[t,j,c] * kI[s,c]),   s <= t.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer is a DEVICE pointer unless stated, 16-byte aligned, to a
+ *   dense row-major array with the layout given.  The caller owns all
+ *   memory; the library never allocates device memory.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream) and do not synchronize, except dsa_device_error.
+ * - Arguments are validated on the host before anything is launched; a
+ *   failing call returns a status, launches nothing and leaves a message in
+ *   dsa_last_error().  No C++ exception crosses this boundary.
+ * - FP8 tensors are OCP e4m3 bytes; bf16 tensors are raw bf16 bits.
+ * - Top-k order: higher score first, then lower key index (a total order,
+ *   so exactly one set is correct).  Scores are accumulated in fp32; they
+ *   are exact (and the selected sets bit-identical to an exact reference)
+ *   whenever the inputs are integer-valued with |score| < 2^24, e.g.
+ *   indexer values in [-8, 8] with d_I <= 128 and weights in {0..3}.
+ * - Index rows list the selected keys in ascending order, then -1 padding.
+ *   The result is deterministic: the same inputs give the same bits.
+ * - A kernel that detects an error (a bounded wait that timed out, an index
+ *   out of range) records a code in a per-device error word instead of
+ *   faulting; read it with dsa_device_error.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative or inconsistent size */
+    DSA_ERR_UNSUPPORTED = 2,   /* a shape outside the compiled variants (see each call) */
+    DSA_ERR_WORKSPACE = 3,     /* workspace smaller than the matching *_workspace_size */
+    DSA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+    DSA_ERR_DEVICE = 5         /* a kernel recorded an error in the device error word */
+} dsa_status_t;
+
+/* Device error word codes (dsa_device_error). */
+#define DSA_DEVERR_NONE 0
+#define DSA_DEVERR_TIMEOUT 1     /* a bounded wait inside a kernel gave up */
+#define DSA_DEVERR_INDEX 2       /* an index row held a key outside the cache */
+
+typedef void* dsa_stream_t;   /* cudaStream_t */
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+DSA_API int dsa_version(void);
+
+/* Human-readable name of a status code; never NULL. */
+DSA_API const char* dsa_status_string(int status);
+
+/* Message of the last failing call on this host thread ("" if none). */
+DSA_API const char* dsa_last_error(void);
+
+/*
+ * dsa_index_topk - prefill indexer + top-k (hot-path steps A1 and A2).
+ * Computes I[t,s] for every causal pair with FP8 tcgen05 tensor-core MMAs,
+ * applies the per-head ReLU and weighted head sum in the epilogue, and keeps
+ * a streaming top-k per query in shared memory; the L x L score matrix is
+ * never written.
+ *
+ *   q_I  [L][H_I][d_I]  e4m3   indexer queries
+ *   k_I  [L][d_I]       e4m3   indexer keys (one per token, shared by heads)
+ *   w    [L][H_I]       fp32   per-query head weights
+ *   idx  [L][k]         int32  OUT: row t = the min(k, t+1) selected keys
+ *                              s <= t, ascending, then -1
+ * Supported: H_I in {4, 64}, d_I in {64, 128}, 1 <= k <= 2048,
+ * 1 <= L <= 2^30.  Others return DSA_ERR_UNSUPPORTED.
+ */
+DSA_API dsa_status_t dsa_index_topk(const void* q_I, const void* k_I, const float* w, int64_t L,
+                            int H_I, int d_I, int k, int32_t* idx, dsa_stream_t stream);
+
+/*
+ * dsa_index_scores - the same indexer, writing the dense causal score
+ * matrix instead of selecting (for small L: checks and training losses that
+ * need the whole score distribution).
+ *
+ *   scores [L][L] fp32  OUT: I[t,s] for s <= t, -inf for s > t
+ * Same shape support as dsa_index_topk; L * L must fit in 2^31 elements.
+ */
+DSA_API dsa_status_t dsa_index_scores(const void* q_I, const void* k_I, const float* w, int64_t L,
+                              int H_I, int d_I, float* scores, dsa_stream_t stream);
+
+/*
+ * dsa_sparse_attn_prefill - sparse GQA attention over selected rows (A3).
+ * For every query token t and query head h, with group g = h / (Hq / Hkv):
+ *   O[t,h] = sum_{s in idx[t]} softmax_s(scale * Q[t,h] . K[s,g]) V[s,g]
+ * Each selected K/V row is gathered once per token and shared by all query
+ * heads of its group; softmax is online in fp32; O is rounded to bf16 (RNE).
+ *
+ *   Q    [L][Hq][d]   bf16
+ *   K, V [L][Hkv][d]  bf16
+ *   idx  [L][k]       int32  keys to attend; entries < 0 are skipped, so
+ *                            rows may be padded with -1 in any position;
+ *                            an entry >= L is skipped and flagged
+ *                            DSA_DEVERR_INDEX
+ *   O    [L][Hq][d]   bf16   OUT (a row with no valid entry is all zeros)
+ * Supported: d in {64, 128}; (Hkv, Hq/Hkv) in {(2, 4), (4, 8)}; k <= 65536.
+ */
+DSA_API dsa_status_t dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
+                                     const int32_t* idx, int64_t L, int Hq, int Hkv, int d,
+                                     int k, float scale, void* O, dsa_stream_t stream);
+
+/*
+ * dsa_decode_workspace_size - bytes of device workspace that
+ * dsa_sparse_attn_decode needs for these sizes (256-byte aligned pointer).
+ */
+DSA_API size_t dsa_decode_workspace_size(int B, int64_t total_n, int H_I, int d_I, int k, int Hq,
+                                 int Hkv, int d);
+
+/*
+ * dsa_sparse_attn_decode - one new token per sequence over a long cache (A4):
+ * indexer over each sequence's whole cache, top-k, sparse GQA attention.
+ * The caches are packed: sequence b owns rows [cache_off[b], cache_off[b+1])
+ * and its newest row (the token being decoded, appended by the caller
+ * before the call) is the last one, so the result equals prefill row
+ * t = n_b - 1 of that sequence.
+ *
+ *   q_I       [B][H_I][d_I]      e4m3
+ *   w         [B][H_I]           fp32
+ *   Q         [B][Hq][d]         bf16
+ *   kI_cache  [total_n][d_I]     e4m3
+ *   K_cache, V_cache [total_n][Hkv][d] bf16
+ *   cache_off [B+1]              int64, device: prefix sums, cache_off[0] = 0,
+ *                                cache_off[B] = total_n, every n_b >= 1
+ *   O         [B][Hq][d]         bf16  OUT
+ *   idx_out   [B][k]             int32 OUT or NULL: sequence-local keys,
+ *                                ascending, -1 padded
+ *   workspace / workspace_bytes  >= dsa_decode_workspace_size(...)
+ * Supported: H_I = 64, d_I = 128, d = 128, Hkv = 4, Hq = 32, k <= 2048,
+ * 1 <= B <= 4096, total_n < 2^31.
+ */
+DSA_API dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void* Q,
+                                    const void* kI_cache, const void* K_cache,
+                                    const void* V_cache, const int64_t* cache_off, int B,
+                                    int64_t total_n, int H_I, int d_I, int Hq, int Hkv, int d,
+                                    int k, float scale, void* O, int32_t* idx_out,
+                                    void* workspace, size_t workspace_bytes,
+                                    dsa_stream_t stream);
+
+/*
+ * dsa_device_error - synchronizes `stream`, then reads and clears the
+ * current device's error word into *code (DSA_DEVERR_*).  Returns DSA_OK if
+ * the word could be read (whatever its value), DSA_ERR_CUDA otherwise.
+ */
+DSA_API dsa_status_t dsa_device_error(int* code, dsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -47,8 +47,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_index_topk.restype = i32
         L.oracle_index_scores.argtypes = [vp, vp, vp, i64, i32, i32, vp, i64, vp, i32]
         L.oracle_index_scores.restype = i32
-        L.oracle_sparse_attn.argtypes = [vp, vp, vp, i64, vp, i32, i32, i32, i32, dbl, vp, i64,
-                                         vp, i32]
+        L.oracle_sparse_attn.argtypes = [vp, vp, vp, i64, vp, i32, i32, i32, i32, i32, dbl, vp,
+                                         i64, vp, i32]
         L.oracle_sparse_attn.restype = i32
         L.oracle_attn_weights.argtypes = [vp, vp, i64, vp, i32, i32, i32, i32, dbl, i64, i32, vp]
         L.oracle_attn_weights.restype = i64
@@ -113,9 +113,10 @@ def index_scores(q_I, k_I, w, rows=None, nthreads: int = 0) -> np.ndarray:
     return out
 
 
-def sparse_attn(Q, K, V, idx, scale: float, rows=None, nthreads: int = 0) -> np.ndarray:
+def sparse_attn(Q, K, V, idx, scale: float, rows=None, nthreads: int = 0,
+                idx_by_row: bool = False) -> np.ndarray:
     """fp64 [len(rows)][Hq][d].  Q [*][Hq][d], K/V [n][Hkv][d] as bf16 bits
-    (uint16); idx int32 [rows of Q][k]."""
+    (uint16); idx int32 [rows of Q][k], or [len(rows)][k] with idx_by_row."""
     Q, K, V = _c(Q, np.uint16), _c(K, np.uint16), _c(V, np.uint16)
     idx = _c(idx, np.int32)
     Lq, Hq, d = Q.shape
@@ -123,9 +124,11 @@ def sparse_attn(Q, K, V, idx, scale: float, rows=None, nthreads: int = 0) -> np.
     k = idx.shape[1]
     r = _rows(rows, Lq)
     out = np.empty((r.size, Hq, d), np.float64)
+    if idx_by_row:
+        assert idx.shape[0] == r.size
     _check(lib().oracle_sparse_attn(Q.ctypes.data, K.ctypes.data, V.ctypes.data, n,
-                                    idx.ctypes.data, k, Hq, Hkv, d, float(scale), r.ctypes.data,
-                                    r.size, out.ctypes.data, nthreads))
+                                    idx.ctypes.data, int(idx_by_row), k, Hq, Hkv, d, float(scale),
+                                    r.ctypes.data, r.size, out.ctypes.data, nthreads))
     return out
 
 

@@ -248,7 +248,8 @@ static int64_t softmax_weights(const uint16_t* q, const uint16_t* K, int64_t n, 
 typedef struct {
     const uint16_t *Q, *K, *V;
     int64_t n;              /* rows of K/V */
-    const int32_t* idx;     /* [rows of Q][k] */
+    const int32_t* idx;     /* [rows of Q][k], or [nrows][k] when idx_by_r */
+    int idx_by_r;
     int k, Hq, Hkv, d;
     double scale;
     const int64_t* rows;
@@ -261,7 +262,7 @@ static void attn_row(void* c_, int64_t r, void* scratch) {
     double* x = (double*)scratch;
     double* p = x + c->k;
     int G = c->Hq / c->Hkv;
-    const int32_t* idx = c->idx + t * (int64_t)c->k;
+    const int32_t* idx = c->idx + (c->idx_by_r ? r : t) * (int64_t)c->k;
     for (int h = 0; h < c->Hq; ++h) {
         int g = h / G;
         const uint16_t* q = c->Q + (t * c->Hq + h) * (int64_t)c->d;
@@ -277,12 +278,14 @@ static void attn_row(void* c_, int64_t r, void* scratch) {
 }
 
 /* Sparse GQA attention for query rows rows[0..nrows) of Q [*][Hq][d] over
- * K, V [n][Hkv][d] (bf16 bits) at the positions idx[t][0..k); entries
- * outside [0, n) are skipped.  out [nrows][Hq][d] fp64. */
+ * K, V [n][Hkv][d] (bf16 bits) at the positions idx[t][0..k) (or idx[r][..]
+ * for the r-th listed row when idx_by_r is set); entries outside [0, n) are
+ * skipped.  out [nrows][Hq][d] fp64. */
 int oracle_sparse_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t n,
-                       const int32_t* idx, int k, int Hq, int Hkv, int d, double scale,
-                       const int64_t* rows, int64_t nrows, double* out, int nthreads) {
-    attn_ctx c = {Q, K, V, n, idx, k, Hq, Hkv, d, scale, rows, out};
+                       const int32_t* idx, int idx_by_r, int k, int Hq, int Hkv, int d,
+                       double scale, const int64_t* rows, int64_t nrows, double* out,
+                       int nthreads) {
+    attn_ctx c = {Q, K, V, n, idx, idx_by_r, k, Hq, Hkv, d, scale, rows, out};
     return run_rows(attn_row, &c, nrows, 2 * (size_t)k * sizeof(double), nthreads);
 }
 

@@ -1,0 +1,168 @@
+"""B200-native DeepSeek-Sparse-Attention hot path (indexer -> top-k -> sparse
+GQA attention, prefill and decode).
+
+This module is the Python binding of ``libdsa_b200.so`` (C ABI in
+``include/dsa.h``): it checks and marshals arguments and calls the library;
+every step of the computation runs in the library's CUDA kernels.  PyTorch
+only provides device memory and streams.  There is no fallback: if the
+library is missing, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa_b200.so")
+
+DSA_OK = 0
+DEVERR_NONE, DEVERR_TIMEOUT, DEVERR_INDEX = 0, 1, 2
+
+_lib = None
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing; build it with "
+                "`python -m sparse_long_context_02_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, f32, sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float,
+                                 ctypes.c_size_t)
+        L.dsa_version.restype = i32
+        L.dsa_version.argtypes = []
+        L.dsa_status_string.restype = ctypes.c_char_p
+        L.dsa_status_string.argtypes = [i32]
+        L.dsa_last_error.restype = ctypes.c_char_p
+        L.dsa_last_error.argtypes = []
+        L.dsa_index_topk.restype = i32
+        L.dsa_index_topk.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp]
+        L.dsa_index_scores.restype = i32
+        L.dsa_index_scores.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
+        L.dsa_sparse_attn_prefill.restype = i32
+        L.dsa_sparse_attn_prefill.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, f32, vp,
+                                              vp]
+        L.dsa_decode_workspace_size.restype = sz
+        L.dsa_decode_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32, i32]
+        L.dsa_sparse_attn_decode.restype = i32
+        L.dsa_sparse_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                             i32, i32, i32, f32, vp, vp, vp, sz, vp]
+        L.dsa_device_error.restype = i32
+        L.dsa_device_error.argtypes = [ctypes.POINTER(i32), vp]
+        _lib = L
+    return _lib
+
+
+def _check(status: int, name: str) -> None:
+    if status != DSA_OK:
+        L = lib()
+        raise DSAError(status, f"{name}: {L.dsa_status_string(status).decode()}: "
+                               f"{L.dsa_last_error().decode()}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, nbytes_per_elem: Optional[int] = None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if nbytes_per_elem is not None and t.element_size() != nbytes_per_elem:
+        raise ValueError(f"{name} must have {nbytes_per_elem}-byte elements, got {t.dtype}")
+    return t.data_ptr()
+
+
+def version() -> int:
+    return lib().dsa_version()
+
+
+def index_topk(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, k: int,
+               idx: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Indexer + top-k.  q_I [L][H_I][d_I] and k_I [L][d_I] e4m3 (uint8 or
+    float8_e4m3fn), w [L][H_I] float32 -> idx [L][k] int32 (ascending, -1 pad)."""
+    L, H, d = q_I.shape
+    if idx is None:
+        idx = torch.empty((L, k), dtype=torch.int32, device=q_I.device)
+    _check(lib().dsa_index_topk(_dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), L, H, d,
+                                k, _dev(idx, "idx", 4), _stream(stream)), "dsa_index_topk")
+    return idx
+
+
+def index_scores(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor,
+                 scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Dense causal indexer scores [L][L] float32 (-inf above the diagonal)."""
+    L, H, d = q_I.shape
+    if scores is None:
+        scores = torch.empty((L, L), dtype=torch.float32, device=q_I.device)
+    _check(lib().dsa_index_scores(_dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), L, H,
+                                  d, _dev(scores, "scores", 4), _stream(stream)),
+           "dsa_index_scores")
+    return scores
+
+
+def sparse_attn_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, idx: torch.Tensor,
+                        scale: float, O: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """Sparse GQA attention.  Q [L][Hq][d], K/V [L][Hkv][d] bf16, idx [L][k]
+    int32 -> O [L][Hq][d] bf16."""
+    L, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    k = idx.shape[1]
+    if O is None:
+        O = torch.empty_like(Q)
+    _check(lib().dsa_sparse_attn_prefill(_dev(Q, "Q", 2), _dev(K, "K", 2), _dev(V, "V", 2),
+                                         _dev(idx, "idx", 4), L, Hq, Hkv, d, k, float(scale),
+                                         _dev(O, "O", 2), _stream(stream)),
+           "dsa_sparse_attn_prefill")
+    return O
+
+
+def decode_workspace_size(B: int, total_n: int, H_I: int, d_I: int, k: int, Hq: int, Hkv: int,
+                          d: int) -> int:
+    return lib().dsa_decode_workspace_size(B, total_n, H_I, d_I, k, Hq, Hkv, d)
+
+
+def sparse_attn_decode(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, k: int, scale: float,
+                       O=None, idx_out=None, workspace=None, stream=None):
+    """One new token per sequence.  Returns (O [B][Hq][d] bf16, idx_out or None)."""
+    B, H, dI = q_I.shape
+    _, Hq, d = Q.shape
+    total_n = kI_cache.shape[0]
+    Hkv = K_cache.shape[1]
+    if O is None:
+        O = torch.empty_like(Q)
+    need = decode_workspace_size(B, total_n, H, dI, k, Hq, Hkv, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    _check(lib().dsa_sparse_attn_decode(
+        _dev(q_I, "q_I", 1), _dev(w, "w", 4), _dev(Q, "Q", 2), _dev(kI_cache, "kI_cache", 1),
+        _dev(K_cache, "K_cache", 2), _dev(V_cache, "V_cache", 2), _dev(cache_off, "cache_off", 8),
+        B, total_n, H, dI, Hq, Hkv, d, k, float(scale), _dev(O, "O", 2),
+        _dev(idx_out, "idx_out", 4) if idx_out is not None else None,
+        _dev(workspace, "workspace", 1), workspace.numel(), _stream(stream)),
+        "dsa_sparse_attn_decode")
+    return O, idx_out
+
+
+def device_error(stream=None) -> int:
+    """Synchronizes the stream; returns and clears the device error word."""
+    code = ctypes.c_int(0)
+    _check(lib().dsa_device_error(ctypes.byref(code), _stream(stream)), "dsa_device_error")
+    return code.value

@@ -1,0 +1,384 @@
+// C ABI of the DSA hot path (declarations and contracts in include/dsa.h).
+// Host side only: argument validation, TMA descriptor encoding, launches.
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "dsa.h"
+#include "decode.cuh"
+#include "index_topk.cuh"
+#include "sparse_attn.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+dsa_status_t fail(dsa_status_t st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+dsa_status_t ok() {
+    g_last_error[0] = '\0';
+    return DSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define CHECK_PTR(p)                                                                  \
+    do {                                                                              \
+        if ((p) == nullptr) return fail(DSA_ERR_INVALID_ARG, "%s: " #p " is NULL", fn); \
+        if (!aligned16(p))                                                            \
+            return fail(DSA_ERR_INVALID_ARG, "%s: " #p " is not 16-byte aligned", fn); \
+    } while (0)
+
+#define CUDA_TRY(call)                                                                     \
+    do {                                                                                   \
+        cudaError_t e_ = (call);                                                           \
+        if (e_ != cudaSuccess)                                                             \
+            return fail(DSA_ERR_CUDA, "%s: %s failed: %s", fn, #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes] with box [box_rows][row_bytes], swizzled
+// to match the UMMA K-major layout for 64- or 128-byte rows.
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+              uint32_t box_rows) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {row_bytes, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)row_bytes, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw =
+        row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int max_optin_smem() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return 0;
+    return v;
+}
+
+int num_sms() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return v;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ------------------------------------------------------------ indexer
+
+template <int HI, int DI, bool TOPK>
+dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
+                          int64_t L, int k, int32_t* idx, float* scores, cudaStream_t st) {
+    CUtensorMap mq, mk;
+    if (!make_map(&mq, q_I, DI, (uint64_t)L * HI, dsa::idx::kTokens * HI) ||
+        !make_map(&mk, k_I, DI, (uint64_t)L, dsa::idx::kKeyTile))
+        return fail(DSA_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed", fn);
+    const dsa::idx::Layout lay(HI, DI, k, TOPK);
+    const int smem = lay.total + 1024;
+    if (smem > max_optin_smem())
+        return fail(DSA_ERR_UNSUPPORTED, "%s: needs %d bytes of shared memory", fn, smem);
+    auto kern = dsa::idx::index_kernel<HI, DI, TOPK>;
+    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    dsa::idx::Params p;
+    p.w = w;
+    p.L = L;
+    p.k = k;
+    p.idx = idx;
+    p.scores = scores;
+    p.nblocks = (int)((L + dsa::idx::kTokens - 1) / dsa::idx::kTokens);
+    kern<<<p.nblocks, dsa::idx::kThreads, smem, st>>>(mq, mk, p);
+    CUDA_TRY(cudaGetLastError());
+    return ok();
+}
+
+template <bool TOPK>
+dsa_status_t dispatch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
+                            int64_t L, int H_I, int d_I, int k, int32_t* idx, float* scores,
+                            cudaStream_t st) {
+    if (H_I == 64 && d_I == 128)
+        return launch_index<64, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, st);
+    if (H_I == 64 && d_I == 64)
+        return launch_index<64, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, st);
+    if (H_I == 4 && d_I == 128)
+        return launch_index<4, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, st);
+    if (H_I == 4 && d_I == 64)
+        return launch_index<4, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, st);
+    return fail(DSA_ERR_UNSUPPORTED, "%s: (H_I, d_I) = (%d, %d) not in {4, 64} x {64, 128}", fn,
+                H_I, d_I);
+}
+
+// ------------------------------------------------------------ attention
+
+template <int D, int HKV, int G, bool SPLIT>
+dsa_status_t launch_attn(const char* fn, const dsa::attn::Params& p, int64_t grid,
+                         cudaStream_t st) {
+    using C = dsa::attn::Cfg<D, HKV>;
+    auto kern = dsa::attn::attn_kernel<D, HKV, G, SPLIT>;
+    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(p);
+    CUDA_TRY(cudaGetLastError());
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_version(void) { return 100; }
+
+const char* dsa_status_string(int status) {
+    switch (status) {
+        case DSA_OK: return "DSA_OK";
+        case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+        case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+        case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+        case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+        case DSA_ERR_DEVICE: return "DSA_ERR_DEVICE";
+        default: return "DSA_ERR_UNKNOWN";
+    }
+}
+
+const char* dsa_last_error(void) { return g_last_error; }
+
+dsa_status_t dsa_index_topk(const void* q_I, const void* k_I, const float* w, int64_t L,
+                            int H_I, int d_I, int k, int32_t* idx, dsa_stream_t stream) {
+    static const char fn[] = "dsa_index_topk";
+    CHECK_PTR(q_I);
+    CHECK_PTR(k_I);
+    CHECK_PTR(w);
+    CHECK_PTR(idx);
+    if (L < 1 || L > (int64_t(1) << 30)) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (k > 2048) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > 2048", fn, k);
+    if (L * H_I >= (int64_t(1) << 31))
+        return fail(DSA_ERR_UNSUPPORTED, "%s: L * H_I too large", fn);
+    return dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr,
+                                static_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_index_scores(const void* q_I, const void* k_I, const float* w, int64_t L,
+                              int H_I, int d_I, float* scores, dsa_stream_t stream) {
+    static const char fn[] = "dsa_index_scores";
+    CHECK_PTR(q_I);
+    CHECK_PTR(k_I);
+    CHECK_PTR(w);
+    CHECK_PTR(scores);
+    if (L < 1 || L * L >= (int64_t(1) << 31))
+        return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld (L * L must be < 2^31)", fn, (long long)L);
+    return dispatch_index<false>(fn, q_I, k_I, w, L, H_I, d_I, 1, nullptr, scores,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
+                                     const int32_t* idx, int64_t L, int Hq, int Hkv, int d,
+                                     int k, float scale, void* O, dsa_stream_t stream) {
+    static const char fn[] = "dsa_sparse_attn_prefill";
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(idx);
+    CHECK_PTR(O);
+    if (L < 1 || L > (int64_t(1) << 30)) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
+    if (k < 1 || k > 65536) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (Hkv < 1 || Hq < 1 || Hq % Hkv) return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d", fn, Hq, Hkv);
+    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
+    const int G = Hq / Hkv;
+    dsa::attn::Params p{};
+    p.Q = static_cast<const __nv_bfloat16*>(Q);
+    p.K = static_cast<const __nv_bfloat16*>(K);
+    p.V = static_cast<const __nv_bfloat16*>(V);
+    p.idx = idx;
+    p.nkeys = L;
+    p.k = k;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.O = static_cast<__nv_bfloat16*>(O);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    dsa_status_t r;
+    if (d == 128 && Hkv == 4 && G == 8) r = launch_attn<128, 4, 8, false>(fn, p, L, st);
+    else if (d == 64 && Hkv == 2 && G == 4) r = launch_attn<64, 2, 4, false>(fn, p, L, st);
+    else if (d == 128 && Hkv == 2 && G == 4) r = launch_attn<128, 2, 4, false>(fn, p, L, st);
+    else if (d == 64 && Hkv == 4 && G == 8) r = launch_attn<64, 4, 8, false>(fn, p, L, st);
+    else
+        return fail(DSA_ERR_UNSUPPORTED, "%s: (d, Hkv, Hq/Hkv) = (%d, %d, %d)", fn, d, Hkv, G);
+    return r == DSA_OK ? ok() : r;
+}
+
+// ------------------------------------------------------------ decode
+
+namespace {
+constexpr int kMinChunk = 4096;
+
+struct DecodePlan {
+    int ck, max_chunks, nsplit;
+    size_t off_cs, off_sc, off_ix, off_cnt, off_idx, off_po, off_pml, total;
+};
+
+DecodePlan plan_decode(int B, int64_t total_n, int k, int Hq, int d, int sms) {
+    DecodePlan pl;
+    // about two chunk CTAs per SM, each quarter a whole number of 128-key tiles
+    int64_t ck = (total_n + 2 * sms - 1) / (2 * sms);
+    ck = (ck + 511) / 512 * 512;
+    if (ck < kMinChunk) ck = kMinChunk;
+    if (ck > 131072) ck = 131072;
+    pl.ck = (int)ck;
+    pl.max_chunks = (int)((total_n + kMinChunk - 1) / kMinChunk) + B;
+    int ns = (2 * sms + B - 1) / B;
+    if (ns < 1) ns = 1;
+    if (ns > 16) ns = 16;
+    pl.nsplit = ns;
+    size_t o = 0;
+    pl.off_cs = o;  o = align256(o + (size_t)(B + 1) * 4);
+    pl.off_sc = o;  o = align256(o + (size_t)pl.max_chunks * k * 4);
+    pl.off_ix = o;  o = align256(o + (size_t)pl.max_chunks * k * 4);
+    pl.off_cnt = o; o = align256(o + (size_t)pl.max_chunks * 4);
+    pl.off_idx = o; o = align256(o + (size_t)B * k * 4);
+    pl.off_po = o;  o = align256(o + (size_t)B * ns * Hq * d * 4);
+    pl.off_pml = o; o = align256(o + (size_t)B * ns * Hq * 2 * 4);
+    pl.total = o;
+    return pl;
+}
+}  // namespace
+
+size_t dsa_decode_workspace_size(int B, int64_t total_n, int H_I, int d_I, int k, int Hq,
+                                 int Hkv, int d) {
+    (void)H_I;
+    (void)d_I;
+    (void)Hkv;
+    if (B < 1 || total_n < 1 || k < 1) return 0;
+    return plan_decode(B, total_n, k, Hq, d, num_sms()).total;
+}
+
+dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void* Q,
+                                    const void* kI_cache, const void* K_cache,
+                                    const void* V_cache, const int64_t* cache_off, int B,
+                                    int64_t total_n, int H_I, int d_I, int Hq, int Hkv, int d,
+                                    int k, float scale, void* O, int32_t* idx_out,
+                                    void* workspace, size_t workspace_bytes,
+                                    dsa_stream_t stream) {
+    static const char fn[] = "dsa_sparse_attn_decode";
+    CHECK_PTR(q_I);
+    CHECK_PTR(w);
+    CHECK_PTR(Q);
+    CHECK_PTR(kI_cache);
+    CHECK_PTR(K_cache);
+    CHECK_PTR(V_cache);
+    CHECK_PTR(cache_off);
+    CHECK_PTR(O);
+    CHECK_PTR(workspace);
+    if (idx_out && !aligned16(idx_out))
+        return fail(DSA_ERR_INVALID_ARG, "%s: idx_out is not 16-byte aligned", fn);
+    if (B < 1 || B > 4096) return fail(DSA_ERR_INVALID_ARG, "%s: B = %d", fn, B);
+    if (total_n < B || total_n >= (int64_t(1) << 31))
+        return fail(DSA_ERR_INVALID_ARG, "%s: total_n = %lld", fn, (long long)total_n);
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
+    if (H_I != 64 || d_I != 128 || d != 128 || Hkv != 4 || Hq != 32 || k > 2048)
+        return fail(DSA_ERR_UNSUPPORTED,
+                    "%s: supported H_I=64, d_I=128, d=128, Hkv=4, Hq=32, k<=2048", fn);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: workspace is not 256-byte aligned", fn);
+    const DecodePlan pl = plan_decode(B, total_n, k, Hq, d, num_sms());
+    if (workspace_bytes < pl.total)
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, workspace_bytes,
+                    pl.total);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+    dsa::dec::Params dp;
+    dp.w = w;
+    dp.cache_off = cache_off;
+    dp.B = B;
+    dp.total_n = total_n;
+    dp.k = k;
+    dp.ck = pl.ck;
+    dp.chunk_start = reinterpret_cast<int*>(ws + pl.off_cs);
+    dp.cand_sc = reinterpret_cast<float*>(ws + pl.off_sc);
+    dp.cand_ix = reinterpret_cast<int32_t*>(ws + pl.off_ix);
+    dp.cand_cnt = reinterpret_cast<int*>(ws + pl.off_cnt);
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + pl.off_idx);
+
+    CUtensorMap mq, mk;
+    if (!make_map(&mq, q_I, 128, (uint64_t)B * 64, 64) ||
+        !make_map(&mk, kI_cache, 128, (uint64_t)total_n, dsa::idx::kKeyTile))
+        return fail(DSA_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed", fn);
+    const int smem_idx = dsa::dec::Layout(k).total + 1024;
+    if (smem_idx > max_optin_smem())
+        return fail(DSA_ERR_UNSUPPORTED, "%s: needs %d bytes of shared memory", fn, smem_idx);
+
+    dsa::dec::prep_kernel<<<1, 1024, 0, st>>>(dp);
+    CUDA_TRY(cudaGetLastError());
+    CUDA_TRY(cudaFuncSetAttribute(dsa::dec::index_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem_idx));
+    const int grid_idx = (int)((total_n + pl.ck - 1) / pl.ck) + B;
+    dsa::dec::index_kernel<<<grid_idx, dsa::dec::kThreads, smem_idx, st>>>(mq, mk, dp);
+    CUDA_TRY(cudaGetLastError());
+
+    const int merge_smem_cap = 24576;  // entries staged in shared memory (192 KB)
+    const int smem_merge = merge_smem_cap * 8;
+    CUDA_TRY(cudaFuncSetAttribute(dsa::dec::merge_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem_merge));
+    dsa::dec::merge_kernel<<<B, 1024, smem_merge, st>>>(dp, idx, merge_smem_cap);
+    CUDA_TRY(cudaGetLastError());
+
+    dsa::attn::Params ap{};
+    ap.Q = static_cast<const __nv_bfloat16*>(Q);
+    ap.K = static_cast<const __nv_bfloat16*>(K_cache);
+    ap.V = static_cast<const __nv_bfloat16*>(V_cache);
+    ap.idx = idx;
+    ap.k = k;
+    ap.scale_log2 = scale * 1.4426950408889634f;
+    ap.cache_off = cache_off;
+    ap.nsplit = pl.nsplit;
+    ap.part_o = reinterpret_cast<float*>(ws + pl.off_po);
+    ap.part_ml = reinterpret_cast<float*>(ws + pl.off_pml);
+    dsa_status_t r = launch_attn<128, 4, 8, true>(fn, ap, (int64_t)B * pl.nsplit, st);
+    if (r != DSA_OK) return r;
+    dsa::attn::combine_kernel<128, 32><<<B, 256, 0, st>>>(ap.part_o, ap.part_ml, pl.nsplit,
+                                                          static_cast<__nv_bfloat16*>(O));
+    CUDA_TRY(cudaGetLastError());
+    return ok();
+}
+
+dsa_status_t dsa_device_error(int* code, dsa_stream_t stream) {
+    static const char fn[] = "dsa_device_error";
+    if (!code) return fail(DSA_ERR_INVALID_ARG, "%s: code is NULL", fn);
+    CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int v = 0, zero = 0;
+    CUDA_TRY(cudaMemcpyFromSymbol(&v, dsa::g_dsa_device_error, sizeof(int)));
+    CUDA_TRY(cudaMemcpyToSymbol(dsa::g_dsa_device_error, &zero, sizeof(int)));
+    *code = v;
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,328 @@
+// Sparse GQA attention over selected K/V rows (prefill; split form for decode).
+//
+// Kwai Keye-VL-2.0 technical-report summary, section 1: attention runs only
+// over the positions the indexer kept, O(Lk) instead of O(L^2); the base
+// model is GQA, and one index set per query token serves every KV group and
+// query head.  For query row t and head h in group g = h / G:
+//     O[t,h] = sum_{s in idx[t]} softmax_s(scale * Q[t,h] . K[s,g]) V[s,g].
+//
+// The step is bound by the gather: every selected token contributes its K and
+// V rows for all Hkv groups, 2 * Hkv * d * 2 bytes, read once per query token.
+// One CTA serves one query token (or one slice of its index row, for decode).
+// A producer warp turns index entries into untiled bulk copies (one per K row
+// and one per V row, each a contiguous Hkv * d * 2 byte run) into a ring of
+// shared-memory stages; rows are padded by 16 bytes so that the consumers'
+// ldmatrix reads hit distinct banks.  Consumer warp g owns KV group g: its G
+// query heads are the rows of an m16n8k16 tile (rows G..15 are zero), keys the
+// columns.  S = Q K^T and O += P V run on the tensor cores in bf16 with fp32
+// accumulation; the softmax is online in the exp2 domain; P is rounded to
+// bf16 for the second product, O stays fp32 until the final store.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace dsa {
+namespace attn {
+
+constexpr int kNK = 16;      // keys per stage
+constexpr int kStages = 3;
+
+template <int D, int HKV>
+struct Cfg {
+    static constexpr int ROW = HKV * D * 2;       // bytes of one token's K (or V) row
+    static constexpr int STRIDE = ROW + 16;       // padded shared-memory row
+    static constexpr int STAGE = 2 * kNK * STRIDE;
+    static constexpr int THREADS = (HKV + 1) * 32;
+    static constexpr int SMEM = kStages * STAGE + 128;
+};
+
+struct Params {
+    const __nv_bfloat16* Q;   // [rows][Hq][d]
+    const __nv_bfloat16* K;   // [keys][Hkv][d]
+    const __nv_bfloat16* V;
+    const int32_t* idx;       // [rows][k]
+    int64_t nkeys;            // prefill: valid keys are [0, nkeys)
+    int k;
+    float scale_log2;         // softmax scale * log2(e)
+    __nv_bfloat16* O;         // [rows][Hq][d]           (prefill)
+    const int64_t* cache_off; // [B + 1]                 (decode)
+    int nsplit;               // index-row slices per sequence (decode)
+    float* part_o;            // [B][nsplit][Hq][d]      unnormalised partial O
+    float* part_ml;           // [B][nsplit][Hq][2]      running max (log2 units), sum
+};
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                         uint32_t b1) {
+    // A rows 8..15 are zero (a1 = a3 = 0): only d[0], d[1] carry results.
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+template <int D, int HKV, int G, bool SPLIT>
+__global__ void __launch_bounds__(Cfg<D, HKV>::THREADS)
+attn_kernel(const Params p) {
+    using C = Cfg<D, HKV>;
+    constexpr int HQ = HKV * G;
+    static_assert(G <= 8, "at most 8 query heads per KV group");
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::STAGE);
+    uint64_t* empty = full + kStages;
+    uint32_t* mask = reinterpret_cast<uint32_t*>(empty + kStages);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- the unit this CTA serves
+    const __nv_bfloat16 *Kb = p.K, *Vb = p.V, *qrow;
+    const int32_t* irow;
+    int nent;
+    int64_t nkeys, orow = 0;
+    int split = 0;
+    if constexpr (SPLIT) {
+        const int64_t b = blockIdx.x / p.nsplit;
+        split = blockIdx.x % p.nsplit;
+        const int per = ((p.k + p.nsplit - 1) / p.nsplit + kNK - 1) / kNK * kNK;
+        const int e0 = split * per;
+        nent = p.k - e0 < per ? p.k - e0 : per;
+        if (nent < 0) nent = 0;
+        const int64_t base = p.cache_off[b];
+        nkeys = p.cache_off[b + 1] - base;
+        Kb = p.K + base * HKV * D;
+        Vb = p.V + base * HKV * D;
+        irow = p.idx + b * p.k + e0;
+        qrow = p.Q + b * HQ * D;
+        orow = b;
+    } else {
+        const int64_t t = blockIdx.x;
+        nent = p.k;
+        nkeys = p.nkeys;
+        irow = p.idx + t * p.k;
+        qrow = p.Q + t * HQ * D;
+        orow = t;
+    }
+    const int nchunks = (nent + kNK - 1) / kNK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), HKV);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == HKV) {
+        // ------------------------------------------------ gather producer
+        int issued = 0;
+        bool ok = true;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kStages;
+            if (c >= kStages) {
+                bool got = false;
+                if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ((c / kStages) - 1) & 1);
+                if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
+            }
+            const int e = c * kNK + lane;
+            int32_t si = -1;
+            if (lane < kNK && e < nent) si = irow[e];
+            if (si >= nkeys) record_device_error(2);
+            const bool valid = si >= 0 && si < nkeys;
+            const uint32_t bal = __ballot_sync(0xffffffffu, valid);
+            const uint32_t fb = smem_u32(&full[s]);
+            if (lane == 0) {
+                mask[s] = bal;
+                if (bal) mbar_arrive_expect_tx(fb, 2u * kNK * C::ROW);
+                else mbar_arrive(fb);
+            }
+            __syncwarp();
+            if (bal && lane < kNK) {
+                const int64_t row = valid ? si : 0;
+                const uint32_t dstK = smem_u32(smem + s * C::STAGE + lane * C::STRIDE);
+                const uint32_t dstV = dstK + kNK * C::STRIDE;
+                bulk_load(dstK, Kb + row * HKV * D, C::ROW, fb);
+                bulk_load(dstV, Vb + row * HKV * D, C::ROW, fb);
+            }
+            issued = c + 1;
+        }
+        (void)ok;
+        if (lane == 0) {
+            for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
+                mbar_wait(smem_u32(&full[c % kStages]), (c / kStages) & 1);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------- consumer: group g
+    const int g = warp;
+    const int r = lane >> 2;          // query-head row of this thread (0..7)
+    const int cq = (lane & 3) * 2;    // first of the two columns this thread holds
+    const bool hrow = r < G;
+
+    uint32_t qa[D / 16][2];
+    {
+        const __nv_bfloat16* qh = qrow + (g * G + (hrow ? r : 0)) * D;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            uint32_t lo = *reinterpret_cast<const uint32_t*>(qh + ks * 16 + cq);
+            uint32_t hi = *reinterpret_cast<const uint32_t*>(qh + ks * 16 + 8 + cq);
+            qa[ks][0] = hrow ? lo : 0u;
+            qa[ks][1] = hrow ? hi : 0u;
+        }
+    }
+
+    float o[D / 8][2];
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = 0.f;
+    float m_run = -INFINITY, l_part = 0.f;
+
+    const int mi = lane >> 3, ri = lane & 7;  // ldmatrix: matrix id, row in matrix
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % kStages;
+        bool got = mbar_wait(smem_u32(&full[s]), (c / kStages) & 1);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        const uint32_t msk = mask[s];
+        if (msk) {
+            const uint32_t kbase = smem_u32(smem + s * C::STAGE) + g * D * 2;
+            const uint32_t vbase = kbase + kNK * C::STRIDE;
+            float sacc[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+                for (int kp = 0; kp < D / 32; ++kp) {
+                    uint32_t b[4];
+                    ldsm_x4(kbase + (nt * 8 + ri) * C::STRIDE + (kp * 32 + mi * 8) * 2, b);
+                    mma_bf16(sacc[nt], qa[2 * kp][0], qa[2 * kp][1], b[0], b[1]);
+                    mma_bf16(sacc[nt], qa[2 * kp + 1][0], qa[2 * kp + 1][1], b[2], b[3]);
+                }
+            }
+            float x[2][2];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int col = nt * 8 + cq + e;
+                    const float v = (msk >> col) & 1u ? sacc[nt][e] * p.scale_log2 : -INFINITY;
+                    x[nt][e] = v;
+                    mx = fmaxf(mx, v);
+                }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            const float m_use = m_new == -INFINITY ? 0.f : m_new;
+            const float corr = ex2(m_run - m_use);
+            float pr[2][2];
+            float psum = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    pr[nt][e] = ex2(x[nt][e] - m_use);
+                    psum += pr[nt][e];
+                }
+            l_part = l_part * corr + psum;
+            m_run = m_new;
+#pragma unroll
+            for (int n = 0; n < D / 8; ++n) {
+                o[n][0] *= corr;
+                o[n][1] *= corr;
+            }
+            const uint32_t pa0 = pack_bf16(pr[0][0], pr[0][1]);
+            const uint32_t pa2 = pack_bf16(pr[1][0], pr[1][1]);
+#pragma unroll
+            for (int np = 0; np < D / 16; ++np) {
+                uint32_t b[4];
+                ldsm_x4_trans(vbase + ((mi & 1) * 8 + ri) * C::STRIDE + (np * 16 + (mi >> 1) * 8) * 2,
+                              b);
+                float d0[4] = {o[2 * np][0], o[2 * np][1], 0.f, 0.f};
+                float d1[4] = {o[2 * np + 1][0], o[2 * np + 1][1], 0.f, 0.f};
+                mma_bf16(d0, pa0, pa2, b[0], b[1]);
+                mma_bf16(d1, pa0, pa2, b[2], b[3]);
+                o[2 * np][0] = d0[0];
+                o[2 * np][1] = d0[1];
+                o[2 * np + 1][0] = d1[0];
+                o[2 * np + 1][1] = d1[1];
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+    }
+    if (!ok) return;
+
+    float l = l_part;
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    if (!hrow) return;
+    const int h = g * G + r;
+    if constexpr (SPLIT) {
+        float* po = p.part_o + (((int64_t)orow * p.nsplit + split) * HQ + h) * D;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n)
+            *reinterpret_cast<float2*>(po + n * 8 + cq) = make_float2(o[n][0], o[n][1]);
+        if ((lane & 3) == 0) {
+            float* pm = p.part_ml + (((int64_t)orow * p.nsplit + split) * HQ + h) * 2;
+            pm[0] = m_run;
+            pm[1] = l;
+        }
+    } else {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16* out = p.O + ((int64_t)orow * HQ + h) * D;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n)
+            *reinterpret_cast<uint32_t*>(out + n * 8 + cq) = pack_bf16(o[n][0] * inv, o[n][1] * inv);
+    }
+}
+
+// Merges the nsplit partial results of each (sequence, head):
+//   M = max_j m_j,  l = sum_j l_j 2^(m_j - M),  O = sum_j O_j 2^(m_j - M) / l.
+template <int D, int HQ>
+__global__ void __launch_bounds__(256) combine_kernel(const float* part_o, const float* part_ml,
+                                                      int nsplit, __nv_bfloat16* O) {
+    const int64_t b = blockIdx.x;
+    for (int e = threadIdx.x; e < HQ * D; e += blockDim.x) {
+        const int h = e / D, c = e % D;
+        float M = -INFINITY;
+        for (int j = 0; j < nsplit; ++j) M = fmaxf(M, part_ml[((b * nsplit + j) * HQ + h) * 2]);
+        const float Mu = M == -INFINITY ? 0.f : M;
+        float l = 0.f, acc = 0.f;
+        for (int j = 0; j < nsplit; ++j) {
+            const float* ml = part_ml + ((b * nsplit + j) * HQ + h) * 2;
+            const float f = ex2(ml[0] - Mu);
+            l += ml[1] * f;
+            acc += part_o[((b * nsplit + j) * HQ + h) * D + c] * f;
+        }
+        O[(b * HQ + h) * D + c] = __float2bfloat16_rn(l > 0.f ? acc / l : 0.f);
+    }
+}
+
+}  // namespace attn
+}  // namespace dsa

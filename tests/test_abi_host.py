@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and
+loads, exports every entry point include/dsa.h declares, and rejects bad
+arguments with a status before it touches the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sparse_long_context_02_b200 as dsa
+from sparse_long_context_02_b200 import build as dsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def L():
+    dsa_build.build()
+    return dsa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"DSA_API\s+[\w\s\*]+?\b(dsa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("dsa_index_topk", "dsa_sparse_attn_prefill", "dsa_sparse_attn_decode",
+                 "dsa_index_scores", "dsa_decode_workspace_size", "dsa_device_error",
+                 "dsa_last_error", "dsa_status_string", "dsa_version"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_status_strings_and_version(L):
+    assert L.dsa_version() >= 100
+    assert L.dsa_status_string(0) == b"DSA_OK"
+    assert L.dsa_status_string(3) == b"DSA_ERR_WORKSPACE"
+    assert L.dsa_status_string(99) == b"DSA_ERR_UNKNOWN"
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation
+
+
+def test_index_topk_rejects_bad_arguments(L):
+    f = L.dsa_index_topk
+    assert f(None, FAKE, FAKE, 64, 4, 64, 8, FAKE, None) == INVALID
+    assert b"q_I is NULL" in L.dsa_last_error()
+    assert f(FAKE + 4, FAKE, FAKE, 64, 4, 64, 8, FAKE, None) == INVALID
+    assert b"aligned" in L.dsa_last_error()
+    assert f(FAKE, FAKE, FAKE, 0, 4, 64, 8, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 64, 4, 64, 0, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 64, 4, 64, 4096, FAKE, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 64, 8, 64, 8, FAKE, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 64, 64, 96, 8, FAKE, None) == UNSUPPORTED
+
+
+def test_index_scores_rejects_bad_arguments(L):
+    f = L.dsa_index_scores
+    assert f(FAKE, FAKE, None, 64, 4, 64, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 1 << 16, 4, 64, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 64, 16, 64, FAKE, None) == UNSUPPORTED
+
+
+def test_prefill_attention_rejects_bad_arguments(L):
+    f = L.dsa_sparse_attn_prefill
+    sc = ctypes.c_float(0.125)
+    assert f(FAKE, FAKE, FAKE, None, 64, 8, 2, 64, 16, sc, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 3, 64, 16, sc, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 64, 16, ctypes.c_float(-1.0), FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 96, 16, sc, FAKE, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 16, 1, 64, 16, sc, FAKE, None) == UNSUPPORTED
+
+
+def test_decode_rejects_bad_arguments_and_small_workspace(L):
+    f = L.dsa_sparse_attn_decode
+    sc = ctypes.c_float(0.088)
+    args = [FAKE] * 7 + [4, 40000, 64, 128, 32, 4, 128, 2048, sc, FAKE, None, FAKE]
+    need = L.dsa_decode_workspace_size(4, 40000, 64, 128, 2048, 32, 4, 128)
+    assert need > 0
+    assert f(*args, need - 1, None) == WORKSPACE
+    assert b"workspace" in L.dsa_last_error()
+    bad = list(args)
+    bad[0] = None
+    assert f(*bad, need, None) == INVALID
+    bad = list(args)
+    bad[7] = 0
+    assert f(*bad, need, None) == INVALID
+    bad = list(args)
+    bad[11] = 16  # Hq
+    assert f(*bad, need, None) == UNSUPPORTED
+    bad = list(args)
+    bad[18] = FAKE + 16  # workspace not 256-byte aligned
+    assert f(*bad, need, None) == INVALID
+
+
+def test_device_error_rejects_null(L):
+    assert L.dsa_device_error(None, None) == INVALID
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(dsa, "_lib", None)
+    monkeypatch.setattr(dsa, "LIB_PATH", "/nonexistent/libdsa_b200.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        dsa.lib()
