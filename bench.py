@@ -43,8 +43,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--prefill-config", type=int, default=3)
-    ap.add_argument("--decode-config", type=int, default=4)
+    ap.add_argument("--prefill-config", type=int, default=3,
+                    help="workload id of the prefill part (0: no prefill part)")
+    ap.add_argument("--decode-config", type=int, default=4,
+                    help="workload id of the decode part (0: no decode part)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="use only the first B sequences of the decode workload (profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -200,31 +204,39 @@ def run_ours(args, rank, world, local_rank):
     import sparse_long_context_02_b200 as dsa
 
     torch.cuda.set_device(local_rank)
-    pcfg = gen.CONFIGS[args.prefill_config]
-    dcfg = gen.CONFIGS[args.decode_config]
+    pcfg = gen.CONFIGS[args.prefill_config] if args.prefill_config else None
+    dcfg = gen.CONFIGS[args.decode_config] if args.decode_config else None
+    if dcfg is not None and args.decode_batch:
+        dcfg = dcfg.with_(B=args.decode_batch)
     if world > 1:  # independent problem per rank
-        pcfg = pcfg.with_(seed=pcfg.seed_ + 1000 * rank)
-        dcfg = dcfg.with_(seed=dcfg.seed_ + 1000 * rank)
+        pcfg = pcfg and pcfg.with_(seed=pcfg.seed_ + 1000 * rank)
+        dcfg = dcfg and dcfg.with_(seed=dcfg.seed_ + 1000 * rank)
     keep_host = not args.no_e2e
-    P, Ph, p_host = build_prefill(torch, pcfg, keep_host)
-    D, Dh, off = build_decode(torch, dcfg, keep_host)
+    P, Ph, p_host = build_prefill(torch, pcfg, keep_host) if pcfg else ({}, {}, None)
+    D, Dh, off = build_decode(torch, dcfg, keep_host) if dcfg else ({}, {}, np.zeros(1))
     lens = np.diff(off)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     def prefill():
+        if pcfg is None:
+            return
         dsa.index_topk(P["q_I"], P["k_I"], P["w"], pcfg.k, idx=P["idx"], stream=stream)
 
     def attn():
+        if pcfg is None:
+            return
         dsa.sparse_attn_prefill(P["Q"], P["K"], P["V"], P["idx"], pcfg.scale, O=P["O"],
                                 stream=stream)
 
     def decode():
+        if dcfg is None:
+            return
         dsa.sparse_attn_decode(D["q_I"], D["w"], D["Q"], D["kI_cache"], D["K_cache"],
                                D["V_cache"], D["cache_off"], dcfg.k, dcfg.scale, O=D["O"],
                                idx_out=D["idx"], workspace=D["ws"], stream=stream)
 
-    launches_per_step = 1 + 1 + 5
+    launches_per_step = (2 if pcfg else 0) + (5 if dcfg else 0)
 
     def step(ev=None):
         if ev is not None:
@@ -275,25 +287,28 @@ def run_ours(args, rank, world, local_rank):
     K = args.steps
     prefill_ms = tot[0] / K
     decode_ms = tot[1] / K
-    value = world * pcfg.L / (prefill_ms / 1e3)
-    decode_tps = world * dcfg.B / (decode_ms / 1e3)
+    value = world * pcfg.L / (prefill_ms / 1e3) if pcfg else 0.0
+    decode_tps = world * dcfg.B / (decode_ms / 1e3) if dcfg else 0.0
 
     # ---- roofline of each kernel, reported for the dominant one
     pk = peaks()
     fp8_peak = 2.0 * pk["bf16_sus"]
     ms_idx, ms_att, ms_dec = (statistics.mean(t_idx), statistics.mean(t_att),
                               statistics.mean(t_dec))
-    kernels = {
-        "dsa_index_topk": dict(bound="tensor", ms=ms_idx, work=prefill_flops(pcfg),
-                               achieved=prefill_flops(pcfg) / (ms_idx / 1e3) / 1e12,
-                               peak=fp8_peak, unit="TFLOP/s"),
-        "dsa_sparse_attn_prefill": dict(bound="hbm", ms=ms_att, work=prefill_attn_bytes(pcfg),
-                                        achieved=prefill_attn_bytes(pcfg) / (ms_att / 1e3) / 1e9,
-                                        peak=pk["hbm"], unit="GB/s"),
-        "dsa_sparse_attn_decode": dict(bound="hbm", ms=ms_dec, work=decode_bytes(dcfg, lens),
-                                       achieved=decode_bytes(dcfg, lens) / (ms_dec / 1e3) / 1e9,
-                                       peak=pk["hbm"], unit="GB/s"),
-    }
+    kernels = {}
+    if pcfg:
+        kernels["dsa_index_topk"] = dict(
+            bound="tensor", ms=ms_idx, work=prefill_flops(pcfg),
+            achieved=prefill_flops(pcfg) / (ms_idx / 1e3) / 1e12, peak=fp8_peak, unit="TFLOP/s")
+        kernels["dsa_sparse_attn_prefill"] = dict(
+            bound="hbm", ms=ms_att, work=prefill_attn_bytes(pcfg),
+            achieved=prefill_attn_bytes(pcfg) / (ms_att / 1e3) / 1e9, peak=pk["hbm"],
+            unit="GB/s")
+    if dcfg:
+        kernels["dsa_sparse_attn_decode"] = dict(
+            bound="hbm", ms=ms_dec, work=decode_bytes(dcfg, lens),
+            achieved=decode_bytes(dcfg, lens) / (ms_dec / 1e3) / 1e9, peak=pk["hbm"],
+            unit="GB/s")
     for v in kernels.values():
         v["frac"] = v["achieved"] / v["peak"]
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
@@ -312,12 +327,12 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the public API with host buffers
     e2e = None
     if keep_host:
-        O_host = torch.empty(P["O"].shape, dtype=torch.bfloat16).pin_memory()
-        Od_host = torch.empty(D["O"].shape, dtype=torch.bfloat16).pin_memory()
+        O_host = torch.empty(P["O"].shape if pcfg else (1,), dtype=torch.bfloat16).pin_memory()
+        Od_host = torch.empty(D["O"].shape if dcfg else (1,), dtype=torch.bfloat16).pin_memory()
         h2d_p = sum(v.numel() * v.element_size() for v in Ph.values())
         h2d_d = sum(v.numel() * v.element_size() for v in Dh.values())
-        d2h_p = O_host.numel() * 2
-        d2h_d = Od_host.numel() * 2
+        d2h_p = O_host.numel() * 2 if pcfg else 0
+        d2h_d = Od_host.numel() * 2 if dcfg else 0
         ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
         if world > 1:
             tdist.barrier()
@@ -329,12 +344,14 @@ def run_ours(args, rank, world, local_rank):
                 P[n].copy_(h, non_blocking=True)
             prefill()
             attn()
-            O_host.copy_(P["O"], non_blocking=True)
+            if pcfg:
+                O_host.copy_(P["O"], non_blocking=True)
             ev2[i][1].record(stream)
             for n, h in Dh.items():
                 D[n].copy_(h, non_blocking=True)
             decode()
-            Od_host.copy_(D["O"], non_blocking=True)
+            if dcfg:
+                Od_host.copy_(D["O"], non_blocking=True)
             ev2[i][2].record(stream)
         torch.cuda.synchronize()
         if world > 1:
@@ -346,16 +363,17 @@ def run_ours(args, rank, world, local_rank):
             tt = torch.tensor(et, device="cuda")
             tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
             et = tt.cpu().numpy()
-        e2e = dict(value=world * pcfg.L / (et[0] / K / 1e3), unit="query-tokens/s",
+        e2e = dict(value=world * pcfg.L / (et[0] / K / 1e3) if pcfg else 0.0,
+                   unit="query-tokens/s",
                    h2d_bytes_per_step=int(h2d_p + h2d_d), d2h_bytes_per_step=int(d2h_p + d2h_d),
-                   decode_value=world * dcfg.B / (et[1] / K / 1e3), decode_unit="tokens/s",
-                   ms_per_step=float((et[0] + et[1]) / K))
+                   decode_value=world * dcfg.B / (et[1] / K / 1e3) if dcfg else 0.0,
+                   decode_unit="tokens/s", ms_per_step=float((et[0] + et[1]) / K))
         # result read back: a sanity check that the copy carried real output
         if not torch.isfinite(O_host.float()).all():
             raise RuntimeError("non-finite output")
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and pcfg:
         cpu = cpu_baseline(pcfg, p_host, args.cpu_seconds)
 
     return dict(value=value, prefill_ms=prefill_ms, decode_ms=decode_ms, decode_tps=decode_tps,
@@ -398,8 +416,20 @@ def cpu_baseline(pcfg, host, seconds):
                        f"{dt:.1f} s")
 
 
+def workload_config(pcfg, dcfg, world=1):
+    names = [c.name for c in (pcfg, dcfg) if c is not None]
+    c = dict(workload=" + ".join(names), parallelism=f"independent problem per rank x{world}",
+             l2="flushed between timed steps (256 MiB write, outside the events)")
+    if pcfg is not None:
+        c.update(prefill_L=pcfg.L, k=pcfg.k, H_I=pcfg.H_I, d_I=pcfg.d_I, Hq=pcfg.Hq,
+                 Hkv=pcfg.Hkv, d=pcfg.d)
+    if dcfg is not None:
+        c.update(decode_B=dcfg.B, decode_n=f"U[{dcfg.n_lo},{dcfg.n_hi}]", k=dcfg.k)
+    return c
+
+
 def run_reference(args):
-    pcfg = gen.CONFIGS[args.prefill_config]
+    pcfg = gen.CONFIGS[args.prefill_config or 3]
     host = gen.prefill_inputs(pcfg)
     cores = os.cpu_count() or 1
     probe = sample_rows(pcfg.L, max(cores, 8), seed=1)
@@ -417,13 +447,14 @@ def run_reference(args):
         times.append(time.perf_counter() - t0)
     value = n * args.steps / sum(times)
     sample = (f"{n} query rows per step, stratified over t in [0, {pcfg.L}) of the {pcfg.name} "
-              f"workload (indexer + top-k + attention per row)")
+              f"workload (indexer + top-k + attention per row); the oracle's throughput on the "
+              f"prefill part, in the unit of `value`")
     return dict(impl="reference", metric=METRIC, value=value, unit="query-tokens/s",
                 n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
                 ms_per_step=1e3 * sum(times) / args.steps, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
-                config=dict(workload=pcfg.name, L=pcfg.L, k=pcfg.k, H_I=pcfg.H_I, d_I=pcfg.d_I,
-                            Hq=pcfg.Hq, Hkv=pcfg.Hkv, d=pcfg.d, seed=pcfg.seed_),
+                config=workload_config(pcfg, gen.CONFIGS[args.decode_config]
+                                       if args.decode_config else None),
                 cpu_baseline=dict(value=value, unit="query-tokens/s", cores=cores, kind="oracle",
                                   sample=sample),
                 e2e=dict(value=value, unit="query-tokens/s", h2d_bytes_per_step=0,
@@ -460,11 +491,7 @@ def main():
         warmup=args.warmup, ms_per_step=r["prefill_ms"] + r["decode_ms"],
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="fp8-e4m3/bf16",
         data="synthetic",
-        config=dict(workload=f"{pcfg.name} + {dcfg.name}", prefill_L=pcfg.L, k=pcfg.k,
-                    H_I=pcfg.H_I, d_I=pcfg.d_I, Hq=pcfg.Hq, Hkv=pcfg.Hkv, d=pcfg.d,
-                    decode_B=dcfg.B, decode_n=f"U[{dcfg.n_lo},{dcfg.n_hi}]",
-                    parallelism=f"independent problem per rank x{world}",
-                    l2="flushed between timed steps (256 MiB write, outside the events)"),
+        config=workload_config(pcfg, dcfg, world),
         decode=dict(value=r["decode_tps"], unit="tokens/s", ms_per_step=r["decode_ms"]),
         prefill_ms=r["prefill_ms"],
         kernels=r["kernels"], roofline=r["roofline"], clocks=r["clocks"],
