@@ -163,6 +163,30 @@ DSA_API dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, con
                                     dsa_stream_t stream);
 
 /*
+ * dsa_sparse_attn_decode_noalloc - dsa_sparse_attn_decode for callers that
+ * cannot pass a workspace (the pages have no counterpart: this is a
+ * deployment convenience).  Callers that run inside a host framework owning
+ * all device memory, or a decode loop that must not call cudaMalloc, use it:
+ * the scratch lives in a fixed 64 MiB array inside the library's device
+ * image, held by every GPU that loads the library until the process exits.
+ * Arguments, layouts and results are those of dsa_sparse_attn_decode.
+ *
+ * - Sizes whose dsa_decode_workspace_size exceeds 64 MiB are rejected with
+ *   DSA_ERR_WORKSPACE before any launch.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - All calls share the array and it keeps the last call's contents (no
+ *   part of it needs to start at zero).  Calls that overlap on the GPU race
+ *   on it: serialize them.
+ * - It allocates nothing and frees nothing.
+ */
+DSA_API dsa_status_t dsa_sparse_attn_decode_noalloc(
+    const void* q_I, const float* w, const void* Q, const void* kI_cache, const void* K_cache,
+    const void* V_cache, const int64_t* cache_off, int B, int64_t total_n, int H_I, int d_I,
+    int Hq, int Hkv, int d, int k, float scale, void* O, int32_t* idx_out, dsa_stream_t stream);
+
+/*
  * dsa_device_error - synchronizes `stream`, then reads and clears the
  * current device's error word into *code (DSA_DEVERR_*).  Returns DSA_OK if
  * the word could be read (whatever its value), DSA_ERR_CUDA otherwise.

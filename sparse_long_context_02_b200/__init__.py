@@ -58,6 +58,9 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_attn_decode.restype = i32
         L.dsa_sparse_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
                                              i32, i32, i32, f32, vp, vp, vp, sz, vp]
+        L.dsa_sparse_attn_decode_noalloc.restype = i32
+        L.dsa_sparse_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
+                                                     i32, i32, i32, i32, i32, f32, vp, vp, vp]
         L.dsa_device_error.restype = i32
         L.dsa_device_error.argtypes = [ctypes.POINTER(i32), vp]
         _lib = L
@@ -158,6 +161,27 @@ def sparse_attn_decode(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, k: int,
         _dev(idx_out, "idx_out", 4) if idx_out is not None else None,
         _dev(workspace, "workspace", 1), workspace.numel(), _stream(stream)),
         "dsa_sparse_attn_decode")
+    return O, idx_out
+
+
+def sparse_attn_decode_noalloc(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, k: int,
+                               scale: float, O=None, idx_out=None, stream=None):
+    """sparse_attn_decode without a workspace argument, for callers that
+    cannot allocate device memory at call time: the scratch is a fixed
+    64 MiB array inside the library (see include/dsa.h).  Calls that overlap
+    on the GPU share that array and must be serialized by the caller."""
+    B, H, dI = q_I.shape
+    _, Hq, d = Q.shape
+    total_n = kI_cache.shape[0]
+    Hkv = K_cache.shape[1]
+    if O is None:
+        O = torch.empty_like(Q)
+    _check(lib().dsa_sparse_attn_decode_noalloc(
+        _dev(q_I, "q_I", 1), _dev(w, "w", 4), _dev(Q, "Q", 2), _dev(kI_cache, "kI_cache", 1),
+        _dev(K_cache, "K_cache", 2), _dev(V_cache, "V_cache", 2), _dev(cache_off, "cache_off", 8),
+        B, total_n, H, dI, Hq, Hkv, d, k, float(scale), _dev(O, "O", 2),
+        _dev(idx_out, "idx_out", 4) if idx_out is not None else None, _stream(stream)),
+        "dsa_sparse_attn_decode_noalloc")
     return O, idx_out
 
 

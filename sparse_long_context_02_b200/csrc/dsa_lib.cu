@@ -382,3 +382,70 @@ dsa_status_t dsa_device_error(int* code, dsa_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ decode without allocation
+//
+// Some callers cannot hand the library a workspace: code that runs inside a
+// host framework which owns every byte of device memory and forbids
+// allocations after start-up, or a latency-critical decode loop where a
+// cudaMalloc (which can synchronize the device) is not acceptable.  For them,
+// dsa_sparse_attn_decode_noalloc runs the same decode with its scratch in a
+// fixed array that is part of this library's device image.
+//
+// * Every GPU that loads this library holds the array (kNoAllocScratchBytes)
+//   until the process exits.
+// * Host code cannot use the array's name as a device address; the address
+//   is looked up with cudaGetSymbolAddress once per device, on the first call
+//   made with that device current.  Make that first call before any stream
+//   capture.
+// * All calls share the one array and it keeps the last call's contents.
+//   Nothing in it has to start at zero: every scratch byte a decode reads was
+//   written earlier by the same call.  Calls whose work overlaps on the GPU
+//   (two streams, or two host threads) race on the array and must be
+//   serialized by the caller.
+// * A request whose scratch need exceeds the array is rejected with
+//   DSA_ERR_WORKSPACE before anything is launched.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" dsa_status_t dsa_sparse_attn_decode_noalloc(
+    const void* q_I, const float* w, const void* Q, const void* kI_cache, const void* K_cache,
+    const void* V_cache, const int64_t* cache_off, int B, int64_t total_n, int H_I, int d_I,
+    int Hq, int Hkv, int d, int k, float scale, void* O, int32_t* idx_out, dsa_stream_t stream) {
+    static const char fn[] = "dsa_sparse_attn_decode_noalloc";
+    if (B < 1 || total_n < 1 || k < 1)
+        return fail(DSA_ERR_INVALID_ARG, "%s: B = %d, total_n = %lld, k = %d", fn, B,
+                    (long long)total_n, k);
+    const size_t need = dsa_decode_workspace_size(B, total_n, H_I, d_I, k, Hq, Hkv, d);
+    if (need > kNoAllocScratchBytes)
+        return fail(DSA_ERR_WORKSPACE,
+                    "%s: these sizes need %zu bytes of scratch but the built-in array holds %zu; "
+                    "use dsa_sparse_attn_decode with a caller workspace",
+                    fn, need, kNoAllocScratchBytes);
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: device ordinal %d", fn, dev);
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void* p = nullptr;
+            CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    return dsa_sparse_attn_decode(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, B, total_n,
+                                  H_I, d_I, Hq, Hkv, d, k, scale, O, idx_out, scratch,
+                                  kNoAllocScratchBytes, stream);
+}
