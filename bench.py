@@ -90,6 +90,34 @@ def decode_bytes(cfg, lens) -> float:
             + cfg.B * (cfg.H_I * cfg.d_I + cfg.H_I * 4 + 2 * 2 * cfg.Hq * cfg.d))
 
 
+# ------------------------------------------------------------------ ranks
+
+def rank_workloads(pcfg, dcfg, rank: int, world: int):
+    """Weak scaling: every rank solves its own problem of the same shape (the
+    seeds differ by rank, so no two ranks hold the same data)."""
+    if world <= 1:
+        return pcfg, dcfg
+    return (pcfg and pcfg.with_(seed=pcfg.seed_ + 1000 * rank),
+            dcfg and dcfg.with_(seed=dcfg.seed_ + 1000 * rank))
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Elementwise max of per-rank timings (the slowest rank sets the pace)."""
+    arr = np.asarray(values, dtype=np.float64)
+    if world <= 1:
+        return arr
+    import torch
+    import torch.distributed as tdist
+    t = torch.tensor(arr, device=device if device is not None else "cpu")
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return t.cpu().numpy()
+
+
+def job_throughput(units_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the max time."""
+    return world * units_per_rank / seconds
+
+
 # ------------------------------------------------------------------ clocks
 
 class Clocks:
@@ -208,9 +236,7 @@ def run_ours(args, rank, world, local_rank):
     dcfg = gen.CONFIGS[args.decode_config] if args.decode_config else None
     if dcfg is not None and args.decode_batch:
         dcfg = dcfg.with_(B=args.decode_batch)
-    if world > 1:  # independent problem per rank
-        pcfg = pcfg and pcfg.with_(seed=pcfg.seed_ + 1000 * rank)
-        dcfg = dcfg and dcfg.with_(seed=dcfg.seed_ + 1000 * rank)
+    pcfg, dcfg = rank_workloads(pcfg, dcfg, rank, world)
     keep_host = not args.no_e2e
     P, Ph, p_host = build_prefill(torch, pcfg, keep_host) if pcfg else ({}, {}, None)
     D, Dh, off = build_decode(torch, dcfg, keep_host) if dcfg else ({}, {}, np.zeros(1))
@@ -279,16 +305,13 @@ def run_ours(args, rank, world, local_rank):
     if err != 0:
         raise RuntimeError(f"device error {err} in the timed region")
 
-    tot = np.array([sum(t_idx) + sum(t_att), sum(t_dec)], dtype=np.float64)  # ms over K steps
-    if world > 1:
-        tt = torch.tensor(tot, device="cuda")
-        tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
-        tot = tt.cpu().numpy()
+    # ms over the K steps, max over ranks
+    tot = max_over_ranks([sum(t_idx) + sum(t_att), sum(t_dec)], world, device="cuda")
     K = args.steps
     prefill_ms = tot[0] / K
     decode_ms = tot[1] / K
-    value = world * pcfg.L / (prefill_ms / 1e3) if pcfg else 0.0
-    decode_tps = world * dcfg.B / (decode_ms / 1e3) if dcfg else 0.0
+    value = job_throughput(pcfg.L, world, prefill_ms / 1e3) if pcfg else 0.0
+    decode_tps = job_throughput(dcfg.B, world, decode_ms / 1e3) if dcfg else 0.0
 
     # ---- roofline of each kernel, reported for the dominant one
     pk = peaks()
@@ -358,15 +381,11 @@ def run_ours(args, rank, world, local_rank):
             tdist.barrier()
         e_p = sum(e[0].elapsed_time(e[1]) for e in ev2)
         e_d = sum(e[1].elapsed_time(e[2]) for e in ev2)
-        et = np.array([e_p, e_d])
-        if world > 1:
-            tt = torch.tensor(et, device="cuda")
-            tdist.all_reduce(tt, op=tdist.ReduceOp.MAX)
-            et = tt.cpu().numpy()
-        e2e = dict(value=world * pcfg.L / (et[0] / K / 1e3) if pcfg else 0.0,
+        et = max_over_ranks([e_p, e_d], world, device="cuda")
+        e2e = dict(value=job_throughput(pcfg.L, world, et[0] / K / 1e3) if pcfg else 0.0,
                    unit="query-tokens/s",
                    h2d_bytes_per_step=int(h2d_p + h2d_d), d2h_bytes_per_step=int(d2h_p + d2h_d),
-                   decode_value=world * dcfg.B / (et[1] / K / 1e3) if dcfg else 0.0,
+                   decode_value=job_throughput(dcfg.B, world, et[1] / K / 1e3) if dcfg else 0.0,
                    decode_unit="tokens/s", ms_per_step=float((et[0] + et[1]) / K))
         # result read back: a sanity check that the copy carried real output
         if not torch.isfinite(O_host.float()).all():

@@ -24,6 +24,7 @@ real model's data and stay unpinned.
 from __future__ import annotations
 
 import ctypes
+import os
 from typing import Optional, Sequence
 
 import numpy as np
@@ -34,10 +35,16 @@ _lib = None
 
 
 def lib() -> ctypes.CDLL:
+    """The compiled oracle.  ORACLE_LIB_PATH, if set, names another build of
+    dsa_oracle.c to load instead (the mutation test uses it to run the pins
+    against a copy with a planted mistake)."""
     global _lib
     if _lib is None:
-        _build()
-        L = ctypes.CDLL(LIB_PATH)
+        path = os.environ.get("ORACLE_LIB_PATH")
+        if not path:
+            _build()
+            path = LIB_PATH
+        L = ctypes.CDLL(path)
         vp, i64, i32, dbl = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
         L.oracle_e4m3.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3.restype = dbl
