@@ -4,39 +4,46 @@
 // the same indexer -> top-k -> sparse attention for the single new query of
 // each sequence, whose row is the last row of its cache.
 //
-// Phase 1 (prep): chunk_start[b] = sum over earlier sequences of
-//          ceil(n_b / CK), so every cache chunk of CK keys gets one CTA.
-// Phase 2 (index): a CTA scans one chunk.  Its four epilogue warpgroups each
-//          own a contiguous quarter; the MMA issuer interleaves their tiles
-//          (M = 128 keys, N = 64 indexer heads of the one query) into eight
-//          TMEM accumulators, so the dominant HBM stream (128 bytes of k_I per
-//          cached key) is read exactly once.  Each warpgroup keeps the top-k
-//          of its quarter; the CTA then merges the four lists (which are in
-//          ascending key order) into the chunk's top-k.
-// Phase 3 (merge): one CTA per sequence selects the top-k of its chunks'
-//          lists, again in ascending key order.  Every chunk but the last of a
-//          sequence holds exactly k entries (CK >= k), so a sequence's lists
-//          are one contiguous run of the candidate arrays.
+// The dominant cost is the scan of the indexer-key cache (128 bytes per cached
+// key), so the scan is split into equal row ranges, one per CTA, in a single
+// wave: CTA c covers packed-cache rows [c R, (c+1) R).  A range may hold the
+// tail of one sequence, whole short sequences and the head of another; each
+// such piece is a "segment".
+// Phase 1 (prep): seg_base[b] = number of segments of the sequences before b
+//          (sequence b's segments are the CTAs its rows touch, in order).
+// Phase 2 (index): per segment the CTA loads that sequence's query block,
+//          its four epilogue warpgroups each scan a contiguous quarter of the
+//          segment (the MMA thread interleaves their tiles into eight TMEM
+//          accumulators, N = 64 indexer heads of the one query) keeping the
+//          top-k of the quarter, and the CTA merges the four ordered lists
+//          into the segment's top-k, written to slot seg_base[b] + (c - first
+//          CTA of b).
+// Phase 3 (merge): one CTA per sequence selects the top-k of its slots'
+//          lists (in key order) into the index row.
 // Attention (split over index-row slices) and the split merge live in
 // sparse_attn.cuh.
 #pragma once
 
 #include "index_topk.cuh"
+#include "topk_select.cuh"
 
 namespace dsa {
 namespace dec {
 
 using idx::kKeyTile;
-using idx::kStages;
 using idx::cand_capacity;
-using idx::WgTopk;
-using idx::FlatAccess;
-using idx::SegAccess;
+using sel::FlatAccess;
+using sel::Scratch;
+using sel::SegAccess;
+using sel::WgTopk;
 
 constexpr int HI = 64;
 constexpr int DI = 128;
-constexpr int kThreads = 640;
-constexpr int kEpiWarps = 16;
+constexpr int kStages = 5;        // HBM-bound: keep more key tiles in flight
+constexpr int kEpiWarps = 16;     // warps 0-15: four warpgroups, one per chunk quarter
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 18 * 32;
 
 struct Params {
     const float* w;            // [B][HI]
@@ -44,15 +51,20 @@ struct Params {
     int B;
     int64_t total_n;           // rows of the packed caches
     int k;
-    int ck;                    // keys per chunk (multiple of 4 * 128, >= k)
-    int* chunk_start;          // [B + 1]
-    float* cand_sc;            // [max_chunks][k]
+    int64_t R;                 // cache rows per CTA
+    int* seg_base;             // [B + 1]
+    uint32_t* cand_so;         // [slots][k] ordered scores (see topk_select.cuh)
     int32_t* cand_ix;
-    int* cand_cnt;             // [max_chunks]
+    int* cand_cnt;             // [slots]
 };
 
-// chunk_start[b] for b in [0, B].  A sequence whose rows are empty or do not
-// lie inside [0, total_n) owns no chunk and records DSA_DEVERR_INDEX (its
+__device__ __forceinline__ bool seq_ok(const Params& p, int b) {
+    const int64_t lo = p.cache_off[b], hi = p.cache_off[b + 1];
+    return lo >= 0 && hi > lo && hi <= p.total_n;
+}
+
+// seg_base[b] for b in [0, B].  A sequence whose rows are empty or do not lie
+// inside [0, total_n) owns no segment and records DSA_DEVERR_INDEX (its
 // output is then all zeros), so no later phase reads outside the caches or
 // the workspace.
 __global__ void __launch_bounds__(1024) prep_kernel(const Params p) {
@@ -63,10 +75,12 @@ __global__ void __launch_bounds__(1024) prep_kernel(const Params p) {
         const int b = b0 + tid;
         int c = 0;
         if (b < p.B) {
-            const int64_t lo = p.cache_off[b], hi = p.cache_off[b + 1];
-            const bool good = lo >= 0 && hi > lo && hi <= p.total_n;
-            if (!good) record_device_error(2);
-            c = good ? (int)((hi - lo + p.ck - 1) / p.ck) : 0;
+            if (seq_ok(p, b)) {
+                const int64_t lo = p.cache_off[b], hi = p.cache_off[b + 1];
+                c = (int)((hi - 1) / p.R - lo / p.R + 1);
+            } else {
+                record_device_error(2);
+            }
         }
         int incl = c;
         for (int o = 1; o < 32; o <<= 1) {
@@ -80,52 +94,83 @@ __global__ void __launch_bounds__(1024) prep_kernel(const Params p) {
             before += wv < warp ? wsum[wv] : 0;
             total += wsum[wv];
         }
-        if (b < p.B) p.chunk_start[b] = carry + before + incl - c;
+        if (b < p.B) p.seg_base[b] = carry + before + incl - c;
         carry += total;
         __syncthreads();
     }
-    if (tid == 0) p.chunk_start[p.B] = carry;
+    if (tid == 0) p.seg_base[p.B] = carry;
 }
 
 struct Misc {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t qfull;
+    uint64_t qfree;
     uint64_t accfull[4][2];
     uint64_t accempty[4][2];
     uint64_t mma_done;
-    uint64_t red64[4][4];
-    uint64_t red64_all[16];
-    int wcnt[4][2][4];
-    int scratch[4][4];
-    int wsum_all[16];
-    int scratch_all[4];
+    alignas(16) int wcnt[4][2][idx::kBatch][4];  // rows read as int4 by WgTopk::offer
     int cnt[4];
-    int seq, chunk_in_seq;
     uint32_t tmem_base;
     volatile int abort_flag;
 };
 
+static_assert(offsetof(Misc, wcnt) % 16 == 0, "wcnt rows are read as int4");
+
 struct Layout {
-    int q, stage, w, cs, ci, hist, misc, total;
+    int q, stage, w, cs, ci, scratch, scratch_all, misc, total;
     __host__ __device__ explicit Layout(int k) {
         const int cap = cand_capacity(k);
         q = 0;
         stage = HI * DI;                       // 8 KB, 1024-aligned
-        w = stage + kStages * kKeyTile * DI;
-        cs = w + HI * 4;
+        w = stage + kStages * kKeyTile * DI;   // one copy of the head weights per warpgroup
+        cs = w + 4 * HI * 4;
         ci = cs + 4 * cap * 4;
-        hist = ci + 4 * cap * 4;
-        misc = hist + 4 * 256 * 4;
-        total = misc + 1024;
+        scratch = (ci + 4 * cap * 4 + 15) / 16 * 16;
+        scratch_all = scratch + 4 * (int)sizeof(Scratch<128>);
+        misc = (scratch_all + (int)sizeof(Scratch<512>) + 15) / 16 * 16;
+        total = misc + (int)sizeof(Misc);
     }
 };
 
-// Tiles of warpgroup w in a chunk of `len` keys split into quarters of `sub`.
-__device__ __forceinline__ int quarter_tiles(int len, int sub, int w) {
-    int l = len - w * sub;
-    l = l < 0 ? 0 : (l > sub ? sub : l);
-    return (l + kKeyTile - 1) / kKeyTile;
+// One piece of a sequence inside this CTA's row range.
+struct Segment {
+    int b;            // sequence
+    int64_t base;     // first cache row of the sequence
+    int64_t lo, len;  // sequence-local first key and length of the piece
+    int sub;          // keys per quarter (a multiple of the tile)
+    // tiles of quarter w
+    __device__ __forceinline__ int tiles(int w) const {
+        int64_t l = len - (int64_t)w * sub;
+        l = l < 0 ? 0 : (l > sub ? sub : l);
+        return (int)((l + kKeyTile - 1) / kKeyTile);
+    }
+};
+
+// Segments of CTA c are the valid sequences overlapping [r0, r1), in order.
+// first_seq: the last b with cache_off[b] <= r0.
+__device__ __forceinline__ int first_seq(const Params& p, int64_t r0) {
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.cache_off[mid] <= r0) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ bool make_segment(const Params& p, int b, int64_t r0, int64_t r1,
+                                             Segment& g) {
+    if (!seq_ok(p, b)) return false;
+    const int64_t off = p.cache_off[b], end = p.cache_off[b + 1];
+    const int64_t a = off > r0 ? off : r0, z = end < r1 ? end : r1;
+    if (z <= a) return false;
+    g.b = b;
+    g.base = off;
+    g.lo = a - off;
+    g.len = z - a;
+    g.sub = (int)((g.len + 4 * kKeyTile - 1) / (4 * kKeyTile) * kKeyTile);
+    return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -137,7 +182,9 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     constexpr uint32_t IDESC = idesc_e4m3_f32(N);
 
     const int c = blockIdx.x;
-    if (c >= p.chunk_start[p.B]) return;  // more CTAs than chunks: nothing to do
+    const int64_t r0 = (int64_t)c * p.R;
+    const int64_t r1 = r0 + p.R < p.total_n ? r0 + p.R : p.total_n;
+    if (r0 >= r1) return;  // more CTAs than ranges: nothing to do
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -145,23 +192,15 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     const Layout lay(p.k);
     const int cap = cand_capacity(p.k);
     Misc* misc = reinterpret_cast<Misc*>(smem + lay.misc);
-    float* w_s = reinterpret_cast<float*>(smem + lay.w);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        int lo = 0, hi = p.B - 1;  // last b with chunk_start[b] <= c
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (p.chunk_start[mid] <= c) lo = mid;
-            else hi = mid - 1;
-        }
-        misc->seq = lo;
-        misc->chunk_in_seq = c - p.chunk_start[lo];
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&misc->full[s]), 1);
             mbar_init(smem_u32(&misc->empty[s]), 1);
         }
         mbar_init(smem_u32(&misc->qfull), 1);
+        mbar_init(smem_u32(&misc->qfree), 1);
         for (int w = 0; w < 4; ++w)
             for (int b = 0; b < 2; ++b) {
                 mbar_init(smem_u32(&misc->accfull[w][b]), 1);
@@ -171,7 +210,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         misc->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 2) {
+    if (warp == kProducerWarp) {
         tmem_alloc(smem_u32(&misc->tmem_base), TMEM_COLS);
         tmem_relinquish();
     }
@@ -179,193 +218,264 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc->tmem_base;
-    const int b = misc->seq;
-    const int64_t base = p.cache_off[b];
-    const int64_t n_b = p.cache_off[b + 1] - base;
-    const int64_t key0 = (int64_t)misc->chunk_in_seq * p.ck;
-    const int len = (int)(n_b - key0 < p.ck ? n_b - key0 : p.ck);
-    const int sub = p.ck / 4;
-    for (int e = threadIdx.x; e < HI; e += kThreads) w_s[e] = p.w[(int64_t)b * HI + e];
-    int nt[4];
-#pragma unroll
-    for (int w = 0; w < 4; ++w) nt[w] = quarter_tiles(len, sub, w);
-    const int umax = nt[0];  // quarter 0 has the most tiles
-    __syncthreads();
+    const int b_first = first_seq(p, r0);
 
-    if (warp == 0) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tensormap(&tmap_q);
             prefetch_tensormap(&tmap_k);
             const uint32_t qbar = smem_u32(&misc->qfull);
-            mbar_arrive_expect_tx(qbar, HI * DI);
-            tma_load_2d(smem_u32(smem + lay.q), &tmap_q, qbar, 0, b * HI);
-            int i = 0;
+            int i = 0, nseg = 0;
             bool ok = true;
-            for (int u = 0; ok && u < umax; ++u)
-                for (int w = 0; w < 4; ++w) {
-                    if (u >= nt[w]) continue;
-                    if (misc->abort_flag) { ok = false; break; }
-                    const int s = i % kStages;
-                    if (i >= kStages && !mbar_wait(smem_u32(&misc->empty[s]), ((i / kStages) - 1) & 1)) {
-                        misc->abort_flag = 1;
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = smem_u32(&misc->full[s]);
-                    mbar_arrive_expect_tx(fb, KT_BYTES);
-                    const int64_t row = base + key0 + (int64_t)w * sub + (int64_t)u * kKeyTile;
-                    tma_load_2d(smem_u32(smem + lay.stage + s * KT_BYTES), &tmap_k, fb, 0, (int32_t)row);
-                    ++i;
+            Segment g;
+            for (int b = b_first; ok && b < p.B && p.cache_off[b] < r1; ++b) {
+                if (!make_segment(p, b, r0, r1, g)) continue;
+                // the previous segment's MMAs must be done with the query block
+                if (nseg > 0 && !mbar_wait(smem_u32(&misc->qfree), (nseg - 1) & 1)) {
+                    misc->abort_flag = 1;
+                    break;
                 }
-            mbar_wait(qbar, 0);
+                mbar_arrive_expect_tx(qbar, HI * DI);
+                tma_load_2d(smem_u32(smem + lay.q), &tmap_q, qbar, 0, g.b * HI);
+                ++nseg;
+                const int nt0 = g.tiles(0);
+                for (int u = 0; ok && u < nt0; ++u)
+                    for (int w = 0; w < 4; ++w) {
+                        if (u >= g.tiles(w)) continue;
+                        if (misc->abort_flag) { ok = false; break; }
+                        const int s = i % kStages;
+                        if (i >= kStages &&
+                            !mbar_wait(smem_u32(&misc->empty[s]), ((i / kStages) - 1) & 1)) {
+                            misc->abort_flag = 1;
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t fb = smem_u32(&misc->full[s]);
+                        mbar_arrive_expect_tx(fb, KT_BYTES);
+                        const int64_t row = g.base + g.lo + (int64_t)w * g.sub + (int64_t)u * kKeyTile;
+                        tma_load_2d(smem_u32(smem + lay.stage + s * KT_BYTES), &tmap_k, fb, 0,
+                                    (int32_t)row);
+                        ++i;
+                    }
+            }
+            // Never leave with a copy in flight.
+            if (nseg > 0) mbar_wait(qbar, (nseg - 1) & 1);
             for (int e = i - kStages < 0 ? 0 : i - kStages; e < i; ++e)
                 mbar_wait(smem_u32(&misc->full[e % kStages]), (e / kStages) & 1);
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            bool ok = mbar_wait(smem_u32(&misc->qfull), 0);
             const uint64_t bdesc = smem_desc_kmajor(smem_u32(smem + lay.q), DI);
-            int i = 0;
-            for (int u = 0; ok && u < umax; ++u)
-                for (int w = 0; w < 4; ++w) {
-                    if (u >= nt[w]) continue;
-                    if (misc->abort_flag) { ok = false; break; }
-                    const int s = i % kStages;
-                    const int buf = u & 1;
-                    ok = mbar_wait(smem_u32(&misc->full[s]), (i / kStages) & 1);
-                    if (ok && u >= 2) ok = mbar_wait(smem_u32(&misc->accempty[w][buf]), ((u >> 1) - 1) & 1);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint64_t adesc = smem_desc_kmajor(smem_u32(smem + lay.stage + s * KT_BYTES), DI);
-                    const uint32_t d_tmem = tmem_base + (uint32_t)((w * 2 + buf) * N);
+            int i = 0, nseg = 0;
+            int uses[4] = {0, 0, 0, 0};
+            bool ok = true;
+            Segment g;
+            for (int b = b_first; ok && b < p.B && p.cache_off[b] < r1; ++b) {
+                if (!make_segment(p, b, r0, r1, g)) continue;
+                ok = mbar_wait(smem_u32(&misc->qfull), nseg & 1);
+                ++nseg;
+                const int nt0 = g.tiles(0);
+                for (int u = 0; ok && u < nt0; ++u)
 #pragma unroll
-                    for (int kk = 0; kk < DI / 32; ++kk)
-                        umma_f8f6f4(d_tmem, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk),
-                                    IDESC, kk > 0 ? 1u : 0u);
-                    umma_commit(smem_u32(&misc->empty[s]));
-                    umma_commit(smem_u32(&misc->accfull[w][buf]));
-                    ++i;
-                }
+                    for (int w = 0; w < 4; ++w) {
+                        if (!ok || u >= g.tiles(w)) continue;
+                        if (misc->abort_flag) { ok = false; continue; }
+                        const int s = i % kStages;
+                        const int use = uses[w]++;
+                        const int buf = use & 1;
+                        ok = mbar_wait(smem_u32(&misc->full[s]), (i / kStages) & 1);
+                        if (ok && use >= 2)
+                            ok = mbar_wait(smem_u32(&misc->accempty[w][buf]), ((use >> 1) - 1) & 1);
+                        if (!ok) continue;
+                        tc_fence_after();
+                        const uint64_t adesc =
+                            smem_desc_kmajor(smem_u32(smem + lay.stage + s * KT_BYTES), DI);
+                        const uint32_t d_tmem = tmem_base + (uint32_t)((w * 2 + buf) * N);
+#pragma unroll
+                        for (int kk = 0; kk < DI / 32; ++kk)
+                            umma_f8f6f4(d_tmem, adesc + (uint64_t)(2 * kk),
+                                        bdesc + (uint64_t)(2 * kk), IDESC, kk > 0 ? 1u : 0u);
+                        umma_commit(smem_u32(&misc->empty[s]));
+                        umma_commit(smem_u32(&misc->accfull[w][buf]));
+                        ++i;
+                    }
+                umma_commit(smem_u32(&misc->qfree));  // query block free once these retire
+            }
             if (!ok) misc->abort_flag = 1;
             umma_commit(smem_u32(&misc->mma_done));
             mbar_wait(smem_u32(&misc->mma_done), 0);
         }
-    } else if (warp >= 4) {
-        // ------------------------------------------------ epilogue
-        const int w = (warp - 4) >> 2;         // quarter of the chunk
+    } else {
+        // ------------------------------------------------ epilogue (warps 0-15)
+        const int w = warp >> 2;               // quarter of each segment
         const int q = warp & 3;                // TMEM lane quarter
-        const int tid = threadIdx.x - 128 - w * 128;
+        const int tid = threadIdx.x - w * 128;
+        const int t512 = threadIdx.x;
         const uint32_t bar = 1 + w;
-        float* sc = reinterpret_cast<float*>(smem + lay.cs) + w * cap;
+        uint32_t* so = reinterpret_cast<uint32_t*>(smem + lay.cs) + w * cap;
         int32_t* ix = reinterpret_cast<int32_t*>(smem + lay.ci) + w * cap;
-        int* hist = reinterpret_cast<int*>(smem + lay.hist) + w * 256;
-        WgTopk tk{sc, ix, hist, misc->scratch[w], misc->red64[w], misc->wcnt[w], cap, p.k, bar,
-                  tid, -INFINITY, 0};
-        const int64_t qend = key0 + (int64_t)((w + 1) * sub < len ? (w + 1) * sub : len);
-        bool ok = true;
-        for (int u = 0; u < nt[w]; ++u) {
-            const int buf = u & 1;
-            bool got = mbar_wait(smem_u32(&misc->accfull[w][buf]), (u >> 1) & 1);
-            if (!named_bar_and(bar, 128, got && !misc->abort_flag)) {
-                ok = false;
-                break;
+        float* w_s = reinterpret_cast<float*>(smem + lay.w) + w * HI;
+        Scratch<128>* S = reinterpret_cast<Scratch<128>*>(smem + lay.scratch) + w;
+        constexpr int T = idx::kBatch;
+        int use = 0;
+        Segment g;
+        for (int b = b_first; b < p.B && p.cache_off[b] < r1; ++b) {
+            if (!make_segment(p, b, r0, r1, g)) continue;
+            if (tid < HI) w_s[tid] = p.w[(int64_t)g.b * HI + tid];
+            named_bar_sync(bar, 128);
+            WgTopk<T> tk{so, ix, S, misc->wcnt[w], cap, p.k, bar, tid, 0u, 0, 0};
+            const int64_t qlo = g.lo + (int64_t)w * g.sub;
+            const int64_t qend = g.lo + ((int64_t)(w + 1) * g.sub < g.len ? (int64_t)(w + 1) * g.sub
+                                                                          : g.len);
+            const int ntw = g.tiles(w);
+            for (int u0 = 0; u0 < ntw; u0 += T) {
+                bool take[T];
+                uint32_t o[T];
+                int32_t sk[T];
+#pragma unroll
+                for (int v = 0; v < T; ++v) {
+                    const int u = u0 + v;
+                    take[v] = false;
+                    o[v] = 0;
+                    sk[v] = 0;
+                    if (u >= ntw) continue;
+                    const int buf = use & 1;
+                    if (!misc->abort_flag &&
+                        !mbar_wait(smem_u32(&misc->accfull[w][buf]), (use >> 1) & 1))
+                        misc->abort_flag = 1;
+                    tc_fence_after();
+                    const uint32_t taddr =
+                        tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((w * 2 + buf) * N);
+                    const float score = idx::head_sum<HI>(taddr, w_s);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&misc->accempty[w][buf]));
+                    ++use;
+                    const int64_t s = qlo + (int64_t)u * kKeyTile + q * 32 + lane;
+                    take[v] = s < qend;
+                    o[v] = sel::ord_f32(score);
+                    sk[v] = (int32_t)s;
+                }
+                tk.offer(take, o, sk, ntw - u0 < T ? ntw - u0 : T);
             }
-            tc_fence_after();
-            const uint32_t taddr =
-                tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)((w * 2 + buf) * N);
-            const float score = idx::head_sum<HI>(taddr, w_s);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&misc->accempty[w][buf]));
-            const int64_t s = key0 + (int64_t)w * sub + (int64_t)u * kKeyTile + q * 32 + lane;
-            tk.offer(s < qend, score, (int32_t)s, u & 1);
-        }
-        int cnt = 0;
-        if (ok) cnt = tk.finish();
-        if (tid == 0) misc->cnt[w] = ok ? cnt : -1;
-        // ---- merge the four quarter lists into the chunk's top-k
-        const int t512 = threadIdx.x - 128;
-        named_bar_sync(5, 512);
-        const bool all_ok = misc->cnt[0] >= 0 && misc->cnt[1] >= 0 && misc->cnt[2] >= 0 &&
-                            misc->cnt[3] >= 0;
-        if (all_ok) {
+            tk.reduce(false);
+            if (tid == 0) misc->cnt[w] = tk.cnt;
+            // ---- merge the four quarter lists into the segment's top-k
+            named_bar_sync(5, 512);
             SegAccess a;
             a.start[0] = 0;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-                a.sc[v] = reinterpret_cast<float*>(smem + lay.cs) + v * cap;
+                a.so[v] = reinterpret_cast<uint32_t*>(smem + lay.cs) + v * cap;
                 a.ix[v] = reinterpret_cast<int32_t*>(smem + lay.ci) + v * cap;
                 a.start[v + 1] = a.start[v] + misc->cnt[v];
             }
             const int n = a.start[4];
-            float* osc = p.cand_sc + (int64_t)c * p.k;
-            int32_t* oix = p.cand_ix + (int64_t)c * p.k;
+            const int slot = p.seg_base[g.b] + (int)(r0 / p.R - g.base / p.R);
+            uint32_t* oso = p.cand_so + (int64_t)slot * p.k;
+            int32_t* oix = p.cand_ix + (int64_t)slot * p.k;
             int outn;
             if (n <= p.k) {
                 for (int e = t512; e < n; e += 512) {
-                    osc[e] = a.score(e);
+                    oso[e] = a.ord(e);
                     oix[e] = a.index(e);
                 }
                 outn = n;
             } else {
-                int* hist0 = reinterpret_cast<int*>(smem + lay.hist);
-                const uint64_t kth = idx::blk_kth_largest<512>(a, n, p.k, hist0, misc->scratch_all,
-                                                               misc->red64_all, 5, t512);
-                outn = idx::blk_compact<512>(a, n, kth, osc, oix, misc->wsum_all, 5, t512);
+                Scratch<512>* SA = reinterpret_cast<Scratch<512>*>(smem + lay.scratch_all);
+                const uint64_t kth = sel::kth_largest<512, 16>(a, n, p.k, 0u, *SA, 5, t512);
+                outn = sel::compact<512>(a, n, kth, oso, oix, *SA, 5, t512);
             }
-            if (t512 == 0) p.cand_cnt[c] = outn;
-        } else if (t512 == 0) {
-            p.cand_cnt[c] = 0;
-            misc->abort_flag = 1;
+            if (t512 == 0) p.cand_cnt[slot] = misc->abort_flag ? 0 : outn;
+            named_bar_sync(5, 512);  // the lists are read before the next segment refills them
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == kProducerWarp) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
 
-// Per-sequence top-k of its chunks' lists -> idx[b][0..k) ascending, -1 pad.
-// Stages the lists in shared memory when they fit (smem_cap entries).
+// Per-sequence top-k of its slots' lists -> idx[b][0..k) ascending, -1 pad.
+// The lists are gathered into one run (shared memory when they fit in
+// smem_cap entries, else in place in the candidate arrays), then selected.
 __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* idx_out,
                                                       int smem_cap) {
     extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ int hist[256];
-    __shared__ int scratch[4];
-    __shared__ int wsum[32];
-    __shared__ uint64_t red64[32];
+    __shared__ Scratch<1024> S;
+    __shared__ int total_s;
     const int b = blockIdx.x, tid = threadIdx.x;
-    const int c0 = p.chunk_start[b], c1 = p.chunk_start[b + 1];
+    const int s0 = p.seg_base[b], s1 = p.seg_base[b + 1];
     int32_t* out = idx_out + (int64_t)b * p.k;
-    if (c1 <= c0) {
+    if (s1 <= s0) {
         for (int e = tid; e < p.k; e += 1024) out[e] = -1;
         return;
     }
-    const int n = (c1 - 1 - c0) * p.k + p.cand_cnt[c1 - 1];
-    const float* gsc = p.cand_sc + (int64_t)c0 * p.k;
-    const int32_t* gix = p.cand_ix + (int64_t)c0 * p.k;
+    if (tid == 0) {
+        int t = 0;
+        for (int s = s0; s < s1; ++s) t += p.cand_cnt[s];
+        total_s = t;
+    }
+    __syncthreads();
+    const int n = total_s;
+    uint32_t* gsc = p.cand_so + (int64_t)s0 * p.k;
+    int32_t* gix = p.cand_ix + (int64_t)s0 * p.k;
     FlatAccess a{gsc, gix};
     if (n <= smem_cap) {
-        float* ssc = reinterpret_cast<float*>(smem);
+        uint32_t* ssc = reinterpret_cast<uint32_t*>(smem);
         int32_t* six = reinterpret_cast<int32_t*>(smem + (size_t)smem_cap * 4);
-        for (int e = tid; e < n; e += 1024) {
-            ssc[e] = gsc[e];
-            six[e] = gix[e];
+        int at = 0;
+        for (int s = s0; s < s1; ++s) {
+            const int cnt = p.cand_cnt[s];
+            const uint32_t* fs = p.cand_so + (int64_t)s * p.k;
+            const int32_t* fi = p.cand_ix + (int64_t)s * p.k;
+            for (int e = tid; e < cnt; e += 1024) {
+                ssc[at + e] = fs[e];
+                six[at + e] = fi[e];
+            }
+            at += cnt;
         }
         __syncthreads();
         a = FlatAccess{ssc, six};
+    } else {
+        // Close the gaps between the slots, leftwards, one slot at a time.
+        int at = 0;
+        for (int s = s0; s < s1; ++s) {
+            const int cnt = p.cand_cnt[s];
+            const int from = (s - s0) * p.k;
+            uint32_t v[2];
+            int32_t x[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int e = tid + r * 1024;
+                if (e < cnt) {
+                    v[r] = gsc[from + e];
+                    x[r] = gix[from + e];
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int e = tid + r * 1024;
+                if (e < cnt) {
+                    gsc[at + e] = v[r];
+                    gix[at + e] = x[r];
+                }
+            }
+            __syncthreads();
+            at += cnt;
+        }
     }
     int cnt = n;
     if (n > p.k) {
-        const uint64_t kth = idx::blk_kth_largest<1024>(a, n, p.k, hist, scratch, red64, 0, tid);
-        // Out-of-place into the index row: only the selected k entries land there.
-        cnt = idx::blk_compact<1024>(a, n, kth, static_cast<float*>(nullptr), out, wsum, 0,
-                                     tid);
+        const uint64_t kth = sel::kth_largest<1024, 24>(a, n, p.k, 0u, S, 0, tid);
+        // Only the selected k entries land in the index row.
+        cnt = sel::compact<1024>(a, n, kth, static_cast<uint32_t*>(nullptr), out, S, 0, tid);
     } else {
         for (int e = tid; e < n; e += 1024) out[e] = a.index(e);
     }

@@ -237,31 +237,34 @@ dsa_status_t dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V
 // ------------------------------------------------------------ decode
 
 namespace {
-constexpr int kMinChunk = 4096;
+constexpr int64_t kMinRange = 4096;  // cache rows per CTA at least
 
 struct DecodePlan {
-    int ck, max_chunks, nsplit;
-    size_t off_cs, off_sc, off_ix, off_cnt, off_idx, off_po, off_pml, total;
+    int64_t R;          // cache rows per CTA of the indexer scan
+    int ctas, max_slots, nsplit;
+    size_t off_sb, off_sc, off_ix, off_cnt, off_idx, off_po, off_pml, total;
 };
 
 DecodePlan plan_decode(int B, int64_t total_n, int k, int Hq, int d, int sms) {
     DecodePlan pl;
-    // about two chunk CTAs per SM, each quarter a whole number of 128-key tiles
-    int64_t ck = (total_n + 2 * sms - 1) / (2 * sms);
-    ck = (ck + 511) / 512 * 512;
-    if (ck < kMinChunk) ck = kMinChunk;
-    if (ck > 131072) ck = 131072;
-    pl.ck = (int)ck;
-    pl.max_chunks = (int)((total_n + kMinChunk - 1) / kMinChunk) + B;
-    int ns = (2 * sms + B - 1) / B;
+    // one wave: at most one CTA per SM, each scanning an equal row range
+    int64_t ctas = (total_n + kMinRange - 1) / kMinRange;
+    if (ctas > sms) ctas = sms;
+    if (ctas < 1) ctas = 1;
+    pl.R = (total_n + ctas - 1) / ctas;
+    pl.ctas = (int)((total_n + pl.R - 1) / pl.R);
+    pl.max_slots = pl.ctas + B;  // each range boundary splits at most one sequence
+    // split the index rows so that B * nsplit attention CTAs fill one wave
+    // (two resident CTAs per SM)
+    int ns = (2 * sms) / B;
     if (ns < 1) ns = 1;
     if (ns > 16) ns = 16;
     pl.nsplit = ns;
     size_t o = 0;
-    pl.off_cs = o;  o = align256(o + (size_t)(B + 1) * 4);
-    pl.off_sc = o;  o = align256(o + (size_t)pl.max_chunks * k * 4);
-    pl.off_ix = o;  o = align256(o + (size_t)pl.max_chunks * k * 4);
-    pl.off_cnt = o; o = align256(o + (size_t)pl.max_chunks * 4);
+    pl.off_sb = o;  o = align256(o + (size_t)(B + 1) * 4);
+    pl.off_sc = o;  o = align256(o + (size_t)pl.max_slots * k * 4);
+    pl.off_ix = o;  o = align256(o + (size_t)pl.max_slots * k * 4);
+    pl.off_cnt = o; o = align256(o + (size_t)pl.max_slots * 4);
     pl.off_idx = o; o = align256(o + (size_t)B * k * 4);
     pl.off_po = o;  o = align256(o + (size_t)B * ns * Hq * d * 4);
     pl.off_pml = o; o = align256(o + (size_t)B * ns * Hq * 2 * 4);
@@ -321,9 +324,9 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     dp.B = B;
     dp.total_n = total_n;
     dp.k = k;
-    dp.ck = pl.ck;
-    dp.chunk_start = reinterpret_cast<int*>(ws + pl.off_cs);
-    dp.cand_sc = reinterpret_cast<float*>(ws + pl.off_sc);
+    dp.R = pl.R;
+    dp.seg_base = reinterpret_cast<int*>(ws + pl.off_sb);
+    dp.cand_so = reinterpret_cast<uint32_t*>(ws + pl.off_sc);
     dp.cand_ix = reinterpret_cast<int32_t*>(ws + pl.off_ix);
     dp.cand_cnt = reinterpret_cast<int*>(ws + pl.off_cnt);
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + pl.off_idx);
@@ -340,8 +343,7 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     CUDA_TRY(cudaGetLastError());
     CUDA_TRY(cudaFuncSetAttribute(dsa::dec::index_kernel,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem_idx));
-    const int grid_idx = (int)((total_n + pl.ck - 1) / pl.ck) + B;
-    dsa::dec::index_kernel<<<grid_idx, dsa::dec::kThreads, smem_idx, st>>>(mq, mk, dp);
+    dsa::dec::index_kernel<<<pl.ctas, dsa::dec::kThreads, smem_idx, st>>>(mq, mk, dp);
     CUDA_TRY(cudaGetLastError());
 
     const int merge_smem_cap = 24576;  // entries staged in shared memory (192 KB)
@@ -364,8 +366,8 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     ap.part_ml = reinterpret_cast<float*>(ws + pl.off_pml);
     dsa_status_t r = launch_attn<128, 4, 8, true>(fn, ap, (int64_t)B * pl.nsplit, st);
     if (r != DSA_OK) return r;
-    dsa::attn::combine_kernel<128, 32><<<B, 256, 0, st>>>(ap.part_o, ap.part_ml, pl.nsplit,
-                                                          static_cast<__nv_bfloat16*>(O));
+    dsa::attn::combine_kernel<128, 32><<<B * 32, 128, 0, st>>>(ap.part_o, ap.part_ml, pl.nsplit,
+                                                                static_cast<__nv_bfloat16*>(O));
     CUDA_TRY(cudaGetLastError());
     return ok();
 }

@@ -304,24 +304,23 @@ attn_kernel(const Params p) {
 
 // Merges the nsplit partial results of each (sequence, head):
 //   M = max_j m_j,  l = sum_j l_j 2^(m_j - M),  O = sum_j O_j 2^(m_j - M) / l.
+// One CTA per (sequence, head), one thread per output dimension.
 template <int D, int HQ>
-__global__ void __launch_bounds__(256) combine_kernel(const float* part_o, const float* part_ml,
-                                                      int nsplit, __nv_bfloat16* O) {
-    const int64_t b = blockIdx.x;
-    for (int e = threadIdx.x; e < HQ * D; e += blockDim.x) {
-        const int h = e / D, c = e % D;
-        float M = -INFINITY;
-        for (int j = 0; j < nsplit; ++j) M = fmaxf(M, part_ml[((b * nsplit + j) * HQ + h) * 2]);
-        const float Mu = M == -INFINITY ? 0.f : M;
-        float l = 0.f, acc = 0.f;
-        for (int j = 0; j < nsplit; ++j) {
-            const float* ml = part_ml + ((b * nsplit + j) * HQ + h) * 2;
-            const float f = ex2(ml[0] - Mu);
-            l += ml[1] * f;
-            acc += part_o[((b * nsplit + j) * HQ + h) * D + c] * f;
-        }
-        O[(b * HQ + h) * D + c] = __float2bfloat16_rn(l > 0.f ? acc / l : 0.f);
+__global__ void __launch_bounds__(D) combine_kernel(const float* part_o, const float* part_ml,
+                                                    int nsplit, __nv_bfloat16* O) {
+    const int64_t b = blockIdx.x / HQ;
+    const int h = blockIdx.x % HQ, c = threadIdx.x;
+    float M = -INFINITY;
+    for (int j = 0; j < nsplit; ++j) M = fmaxf(M, part_ml[((b * nsplit + j) * HQ + h) * 2]);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float l = 0.f, acc = 0.f;
+    for (int j = 0; j < nsplit; ++j) {
+        const float* ml = part_ml + ((b * nsplit + j) * HQ + h) * 2;
+        const float f = ex2(ml[0] - Mu);
+        l += ml[1] * f;
+        acc += part_o[((b * nsplit + j) * HQ + h) * D + c] * f;
     }
+    O[(b * HQ + h) * D + c] = __float2bfloat16_rn(l > 0.f ? acc / l : 0.f);
 }
 
 }  // namespace attn

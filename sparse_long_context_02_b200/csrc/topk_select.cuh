@@ -1,0 +1,360 @@
+// Exact top-k selection pieces shared by the prefill and decode indexers.
+//
+// Order (Kwai Keye-VL-2.0 technical-report summary, section 1: each query
+// keeps its k best positions; section 8: the selection is deterministic):
+// higher score first, then lower key index.  Scores are kept as ord(score),
+// a monotone map of IEEE floats to unsigned integers, so the whole order is
+// one 64-bit key, larger = better:
+//     key = ord(score) << 32 | ~index
+// Keys are unique, so "the k largest keys" is one well-defined set.
+//
+// Collectives run over NT threads that share a named barrier.  The k-th
+// largest key is found by searching, first on ord(score) (the largest s with
+// at least k entries scoring >= s) with three pivots per pass over scores
+// cached in registers, then, among the entries scoring exactly s, on the
+// index.  Each pass is compares, warp reductions and one barrier: no
+// atomics, no histogram.  Compaction keeps the entries whose key is >= the
+// k-th, in their original order.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace dsa {
+namespace sel {
+
+__device__ __forceinline__ uint32_t ord_f32(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ uint64_t make_key(uint32_t ord, int32_t s) {
+    return ((uint64_t)ord << 32) | (uint64_t)(~(uint32_t)s);
+}
+
+// Candidates are read through an accessor: ord(e), index(e) for logical
+// entry e.  The arrays may live in shared or global memory.
+struct FlatAccess {
+    const uint32_t* so;
+    const int32_t* ix;
+    __device__ __forceinline__ uint32_t ord(int e) const { return so[e]; }
+    __device__ __forceinline__ int32_t index(int e) const { return ix[e]; }
+};
+
+// Up to four lists, logically concatenated (list j holds start[j+1]-start[j]
+// entries).
+struct SegAccess {
+    const uint32_t* so[4];
+    const int32_t* ix[4];
+    int start[5];
+    __device__ __forceinline__ int seg(int e) const {
+        return (e >= start[1]) + (e >= start[2]) + (e >= start[3]);
+    }
+    __device__ __forceinline__ uint32_t ord(int e) const {
+        const int j = seg(e);
+        return so[j][e - start[j]];
+    }
+    __device__ __forceinline__ int32_t index(int e) const {
+        const int j = seg(e);
+        return ix[j][e - start[j]];
+    }
+};
+
+// Shared-memory scratch of one collective group.
+template <int NT>
+struct Scratch {
+    uint32_t red[2][NT / 32];   // per-warp partials, double-buffered by step parity
+    uint32_t red2[2][NT / 32];
+    uint32_t red3[2][NT / 32];
+    int csum[8 * (NT / 32)];    // compaction counts
+    int total;
+};
+
+// Sum of v over the NT threads; `parity` alternates between calls so one
+// barrier per call suffices.
+template <int NT>
+__device__ __forceinline__ uint32_t blk_sum(uint32_t v, Scratch<NT>& S, int& parity, uint32_t bar,
+                                            int tid) {
+    v = __reduce_add_sync(0xffffffffu, v);
+    if ((tid & 31) == 0) S.red[parity][tid >> 5] = v;
+    named_bar_sync(bar, NT);
+    uint32_t s = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) s += S.red[parity][w];
+    parity ^= 1;
+    return s;
+}
+
+// Min of a and max of b over the NT threads (one barrier).
+template <int NT>
+__device__ __forceinline__ void blk_minmax(uint32_t& a, uint32_t& b, Scratch<NT>& S, int& parity,
+                                           uint32_t bar, int tid) {
+    a = __reduce_min_sync(0xffffffffu, a);
+    b = __reduce_max_sync(0xffffffffu, b);
+    if ((tid & 31) == 0) {
+        S.red[parity][tid >> 5] = a;
+        S.red2[parity][tid >> 5] = b;
+    }
+    named_bar_sync(bar, NT);
+    a = S.red[parity][0];
+    b = S.red2[parity][0];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) {
+        a = min(a, S.red[parity][w]);
+        b = max(b, S.red2[parity][w]);
+    }
+    parity ^= 1;
+}
+
+// Per-thread register cache of the ordered scores: entry e = tid + r * NT
+// for r < R (0 beyond n: below every real ord, so it never counts).
+template <int NT, int R, class A>
+__device__ __forceinline__ void load_ords(const A& a, int n, int tid, uint32_t (&oc)[R]) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = tid + r * NT;
+        oc[r] = e < n ? a.ord(e) : 0u;
+    }
+}
+
+// The k-th largest key among entries [0, n) (n >= k >= 1).  `floor`: an ord
+// that at least k entries reach (0 if unknown) — the search starts there.
+// Each pass counts three pivots at once (two bits of the answer per pass)
+// over scores cached in registers (R per thread; entries beyond R * NT are
+// read from memory).
+template <int NT, int R, class A>
+__device__ uint64_t kth_largest(const A& a, int n, int k, uint32_t floor, Scratch<NT>& S,
+                                uint32_t bar, int tid) {
+    int parity = 0;
+    uint32_t oc[R];
+    load_ords<NT, R>(a, n, tid, oc);
+    const int tail0 = R * NT;
+    // ---- score: the largest s with count(ord >= s) >= k
+    uint32_t lo = 0xffffffffu, hi = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if (tid + r * NT < n) lo = min(lo, oc[r]);
+        hi = max(hi, oc[r]);
+    }
+    for (int e = tail0 + tid; e < n; e += NT) {
+        const uint32_t o = a.ord(e);
+        lo = min(lo, o);
+        hi = max(hi, o);
+    }
+    blk_minmax<NT>(lo, hi, S, parity, bar, tid);
+    lo = max(lo, min(floor, hi));
+    while (lo < hi) {  // count(>= lo) >= k always holds; the answer is in [lo, hi]
+        const uint64_t span = (uint64_t)(hi - lo) + 1;
+        const uint32_t m1 = lo + (uint32_t)(span / 4), m2 = lo + (uint32_t)(span / 2),
+                       m3 = lo + (uint32_t)(3 * span / 4);
+        uint32_t c1 = 0, c2 = 0, c3 = 0;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            c1 += oc[r] >= m1;
+            c2 += oc[r] >= m2;
+            c3 += oc[r] >= m3;
+        }
+        for (int e = tail0 + tid; e < n; e += NT) {
+            const uint32_t o = a.ord(e);
+            c1 += o >= m1;
+            c2 += o >= m2;
+            c3 += o >= m3;
+        }
+        c1 = __reduce_add_sync(0xffffffffu, c1);
+        c2 = __reduce_add_sync(0xffffffffu, c2);
+        c3 = __reduce_add_sync(0xffffffffu, c3);
+        if ((tid & 31) == 0) {
+            S.red[parity][tid >> 5] = c1;
+            S.red2[parity][tid >> 5] = c2;
+            S.red3[parity][tid >> 5] = c3;
+        }
+        named_bar_sync(bar, NT);
+        uint32_t t1 = 0, t2 = 0, t3 = 0;
+#pragma unroll
+        for (int w = 0; w < NT / 32; ++w) {
+            t1 += S.red[parity][w];
+            t2 += S.red2[parity][w];
+            t3 += S.red3[parity][w];
+        }
+        parity ^= 1;
+        const uint32_t K = (uint32_t)k;
+        if (t3 >= K) lo = m3;                        // m3 > lo whenever span >= 2
+        else if (t2 >= K) { lo = m2; hi = m3 - 1; }
+        else if (t1 >= K) { lo = m1; hi = m2 - 1; }
+        else hi = m1 - 1;                            // t1 < K implies m1 > lo
+    }
+    const uint32_t s = lo;
+    // ---- index: among entries scoring exactly s, the need-th lowest index
+    uint32_t gt = 0, eq = 0;
+    int32_t imin = 0x7fffffff, imax = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        gt += oc[r] > s;
+        if (oc[r] == s && tid + r * NT < n) {
+            eq += 1;
+            const int32_t i = a.index(tid + r * NT);
+            imin = min(imin, i);
+            imax = max(imax, i);
+        }
+    }
+    for (int e = tail0 + tid; e < n; e += NT) {
+        const uint32_t o = a.ord(e);
+        gt += o > s;
+        if (o == s) {
+            eq += 1;
+            const int32_t i = a.index(e);
+            imin = min(imin, i);
+            imax = max(imax, i);
+        }
+    }
+    const uint32_t need = (uint32_t)k - blk_sum<NT>(gt, S, parity, bar, tid);
+    const uint32_t neq = blk_sum<NT>(eq, S, parity, bar, tid);
+    uint32_t ilo = (uint32_t)imin, ihi = (uint32_t)imax;
+    blk_minmax<NT>(ilo, ihi, S, parity, bar, tid);
+    if (need == neq) return make_key(s, (int32_t)ihi);  // every tie is selected
+    // smallest m with count(ord == s && index <= m) >= need
+    while (ilo < ihi) {
+        const uint32_t mid = ilo + (ihi - ilo) / 2;
+        uint32_t c = 0;
+        for (int e = tid; e < n; e += NT) c += a.ord(e) == s && (uint32_t)a.index(e) <= mid;
+        if (blk_sum<NT>(c, S, parity, bar, tid) >= need) ihi = mid;
+        else ilo = mid + 1;
+    }
+    return make_key(s, (int32_t)ilo);
+}
+
+// Writes, in order, the entries of [0, n) whose key is >= kth to out_so /
+// out_ix (out_so may be null) and returns their count.  A round covers 8 * NT
+// consecutive entries, thread tid holding entries tid, tid + NT, ... (so the
+// reads are bank-conflict free); every read of a round lands in registers
+// before the round writes anything, and a round never writes past the end of
+// its own range, so the output may alias a flat input.
+template <int NT, class A>
+__device__ int compact(const A& a, int n, uint64_t kth, uint32_t* out_so, int32_t* out_ix,
+                       Scratch<NT>& S, uint32_t bar, int tid) {
+    constexpr int NW = NT / 32;
+    constexpr int NC = 8 * NW;            // counts per round, u-major then warp
+    const int lane = tid & 31, warp = tid >> 5;
+    const uint32_t below = (1u << lane) - 1u;
+    int out_base = 0;
+    for (int r0 = 0; r0 < n; r0 += 8 * NT) {
+        uint32_t o8[8];
+        int32_t i8[8];
+        uint32_t bal[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = r0 + u * NT + tid;
+            bool keep = false;
+            o8[u] = 0;
+            i8[u] = 0;
+            if (e < n) {
+                o8[u] = a.ord(e);
+                i8[u] = a.index(e);
+                keep = make_key(o8[u], i8[u]) >= kth;
+            }
+            bal[u] = __ballot_sync(0xffffffffu, keep);
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) S.csum[u * NW + warp] = __popc(bal[u]);
+        }
+        named_bar_sync(bar, NT);
+        if (warp == 0) {  // exclusive scan of the NC counts, in place
+            constexpr int PER = (NC + 31) / 32;
+            int v[PER], s = 0;
+#pragma unroll
+            for (int q = 0; q < PER; ++q) {
+                const int i = lane * PER + q;
+                v[q] = i < NC ? S.csum[i] : 0;
+                s += v[q];
+            }
+            int incl = s;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int run = incl - s;
+#pragma unroll
+            for (int q = 0; q < PER; ++q) {
+                const int i = lane * PER + q;
+                if (i < NC) S.csum[i] = run;
+                run += v[q];
+            }
+            if (lane == 31) S.total = incl;  // kept entries in the round
+        }
+        named_bar_sync(bar, NT);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if ((bal[u] >> lane) & 1u) {
+                const int pos = out_base + S.csum[u * NW + warp] + __popc(bal[u] & below);
+                if (out_so) out_so[pos] = o8[u];
+                out_ix[pos] = i8[u];
+            }
+        }
+        out_base += S.total;
+        named_bar_sync(bar, NT);
+    }
+    return out_base;
+}
+
+// Streaming top-k of one query over keys offered in batches of up to T tiles
+// of 128 (one key per thread of a warpgroup per tile, warp q holding keys
+// 32q..32q+31 of each tile), in ascending key order across batches.
+// Candidates that beat the threshold go to a buffer in key order; when it
+// fills, the k best are kept in order and the threshold rises to the k-th
+// score.  A later key that only ties the threshold can never enter (it would
+// lose the tie on its higher index), so `ord > theta` is exact.  One
+// warpgroup barrier per batch.
+template <int T>
+struct WgTopk {
+    uint32_t* so;
+    int32_t* ix;
+    Scratch<128>* S;
+    int (*wcnt)[T][4];  // [2][T][4] per-warp append counts, double-buffered by batch
+    int cap, k;
+    uint32_t bar;
+    int tid;
+    uint32_t theta;     // ord of the threshold score (0: take everything)
+    int cnt;
+    int parity;
+
+    // take[u]: key of tile u is visible; ord[u], s[u]: its score and index.
+    __device__ __forceinline__ void offer(const bool (&take_in)[T], const uint32_t (&o)[T],
+                                          const int32_t (&s)[T], int ntile) {
+        const int lane = tid & 31, q = tid >> 5;
+        uint32_t bal[T];
+#pragma unroll
+        for (int u = 0; u < T; ++u) {
+            bal[u] = __ballot_sync(0xffffffffu, u < ntile && take_in[u] && o[u] > theta);
+            if (lane == 0) wcnt[parity][u][q] = __popc(bal[u]);
+        }
+        named_bar_sync(bar, 128);
+        const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+        for (int u = 0; u < T; ++u) {
+            const int4 c = *reinterpret_cast<const int4*>(wcnt[parity][u]);
+            const int before = (q > 0 ? c.x : 0) + (q > 1 ? c.y : 0) + (q > 2 ? c.z : 0);
+            if ((bal[u] >> lane) & 1u) {
+                const int pos = cnt + before + __popc(bal[u] & below);
+                so[pos] = o[u];
+                ix[pos] = s[u];
+            }
+            cnt += c.x + c.y + c.z + c.w;
+        }
+        parity ^= 1;
+        if (cnt > cap - T * 128) reduce(true);
+    }
+
+    // Keeps the k best of the buffer (if it holds more), in key order.
+    __device__ void reduce(bool raise_theta) {
+        named_bar_sync(bar, 128);
+        if (cnt <= k) return;
+        const FlatAccess a{so, ix};
+        const uint64_t kth = kth_largest<128, 32>(a, cnt, k, theta, *S, bar, tid);
+        cnt = compact<128>(a, cnt, kth, so, ix, *S, bar, tid);
+        if (raise_theta) theta = (uint32_t)(kth >> 32);
+    }
+};
+
+}  // namespace sel
+}  // namespace dsa
