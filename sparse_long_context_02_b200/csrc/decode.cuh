@@ -109,7 +109,8 @@ struct Misc {
     uint64_t accfull[4][2];
     uint64_t accempty[4][2];
     uint64_t mma_done;
-    alignas(16) int wcnt[4][2][idx::kBatch][4];  // rows read as int4 by WgTopk::offer
+    alignas(16) int wcnt[2][4][idx::kBatch][4];  // rows read as int4 by WgTopk::offer
+    int cnts[2][4];
     int cnt[4];
     uint32_t tmem_base;
     volatile int abort_flag;
@@ -325,12 +326,15 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             if (!make_segment(p, b, r0, r1, g)) continue;
             if (tid < HI) w_s[tid] = p.w[(int64_t)g.b * HI + tid];
             named_bar_sync(bar, 128);
-            WgTopk<T> tk{so, ix, S, misc->wcnt[w], cap, p.k, bar, tid, 0u, 0, 0};
+            WgTopk<T, 4> tk{so, ix, S, misc->wcnt, misc->cnts, w, cap, p.k, bar, 5, tid, 0u, 0, 0};
+            tk.start();
             const int64_t qlo = g.lo + (int64_t)w * g.sub;
             const int64_t qend = g.lo + ((int64_t)(w + 1) * g.sub < g.len ? (int64_t)(w + 1) * g.sub
                                                                           : g.len);
             const int ntw = g.tiles(w);
-            for (int u0 = 0; u0 < ntw; u0 += T) {
+            const int nt0 = g.tiles(0);  // quarter 0 has the most tiles: every warpgroup
+                                         // runs its batch count, offering nothing at the end
+            for (int u0 = 0; u0 < nt0; u0 += T) {
                 bool take[T];
                 uint32_t o[T];
                 int32_t sk[T];
@@ -358,9 +362,9 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                     o[v] = sel::ord_f32(score);
                     sk[v] = (int32_t)s;
                 }
-                tk.offer(take, o, sk, ntw - u0 < T ? ntw - u0 : T);
+                tk.offer(take, o, sk, ntw - u0 < T ? (ntw - u0 > 0 ? ntw - u0 : 0) : T);
             }
-            tk.reduce(false);
+            tk.reduce(true);
             if (tid == 0) misc->cnt[w] = tk.cnt;
             // ---- merge the four quarter lists into the segment's top-k
             named_bar_sync(5, 512);

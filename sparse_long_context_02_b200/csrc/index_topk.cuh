@@ -30,7 +30,7 @@ namespace dsa {
 namespace idx {
 
 using sel::Scratch;
-using sel::WgTopk;
+using sel::WgTopk;  // WgTopk<T, G>
 
 constexpr int kTokens = 4;        // query tokens per CTA
 constexpr int kKeyTile = 128;     // keys per tile (MMA M)
@@ -39,7 +39,8 @@ constexpr int kEpiWarps = 16;     // warps 0-15
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 18 * 32;
-constexpr int kBatch = 4;         // tiles offered to the top-k per warpgroup barrier
+constexpr int kBatch = 4;         // tiles offered to the top-k per barrier
+constexpr uint32_t kAllEpilogueBar = 5;  // named barrier over the 512 epilogue threads
 
 // Candidate buffer entries per query: room for the k kept plus at least one
 // full batch of offers (and 2k, so that a compaction frees at least k).
@@ -56,7 +57,8 @@ struct Misc {
     uint64_t accfull[2];
     uint64_t accempty[2];
     uint64_t mma_done;
-    alignas(16) int wcnt[kTokens][2][kBatch][4];  // rows read as int4 by WgTopk::offer
+    alignas(16) int wcnt[2][kTokens][kBatch][4];  // rows read as int4 by WgTopk::offer
+    int cnts[2][kTokens];
     uint32_t tmem_base;
     volatile int abort_flag;
 };
@@ -267,7 +269,9 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         int32_t* ix = reinterpret_cast<int32_t*>(smem + lay.ci) + j * cap;
         Scratch<128>* S = reinterpret_cast<Scratch<128>*>(smem + lay.scratch) + j;
         const float* wj = w_s + j * HI;
-        WgTopk<kBatch> tk{so, ix, S, misc->wcnt[j], cap, p.k, bar, tid, 0u, 0, 0};
+        WgTopk<kBatch, kTokens> tk{so, ix, S, misc->wcnt, misc->cnts, j, cap, p.k, bar,
+                                   kAllEpilogueBar, tid, 0u, 0, 0};
+        tk.start();
 
         // A wait that times out sets abort_flag; the loop then runs on
         // without waiting (results are discarded), so every warp of the
@@ -307,7 +311,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         }
 
         if constexpr (TOPK) {
-            tk.reduce(false);
+            tk.reduce(true);
             if (trow && !misc->abort_flag) {
                 int32_t* out = p.idx + t * p.k;
                 for (int e = tid; e < p.k; e += 128) out[e] = e < tk.cnt ? ix[e] : -1;

@@ -67,6 +67,7 @@ struct Scratch {
     uint32_t red3[2][NT / 32];
     int csum[8 * (NT / 32)];    // compaction counts
     int total;
+    alignas(16) uint32_t samp[NT];  // one sampled score per thread
 };
 
 // Sum of v over the NT threads; `parity` alternates between calls so one
@@ -103,6 +104,73 @@ __device__ __forceinline__ void blk_minmax(uint32_t& a, uint32_t& b, Scratch<NT>
         b = max(b, S.red2[parity][w]);
     }
     parity ^= 1;
+}
+
+// Index of the need-th entry (1-based, in position order) whose ord equals s.
+// One pass over rounds of NT entries with warp ballots and a scan of the
+// per-(round, warp) counts by warp 0.
+template <int NT, class A>
+__device__ int32_t nth_in_order(const A& a, int n, uint32_t s, uint32_t need, Scratch<NT>& S,
+                                uint32_t bar, int tid) {
+    constexpr int NW = NT / 32;
+    const int lane = tid & 31, warp = tid >> 5;
+    uint32_t before = 0;  // ties in earlier chunks
+    for (int c0 = 0; c0 < n; c0 += 8 * NT) {
+        uint32_t bal[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = c0 + u * NT + tid;
+            bal[u] = __ballot_sync(0xffffffffu, e < n && a.ord(e) == s);
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) S.csum[u * NW + warp] = __popc(bal[u]);
+        }
+        named_bar_sync(bar, NT);
+        if (warp == 0) {  // exclusive scan of the 8 * NW counts, in place
+            constexpr int NC = 8 * NW, PER = (NC + 31) / 32;
+            int v[PER], t = 0;
+#pragma unroll
+            for (int q = 0; q < PER; ++q) {
+                const int i = lane * PER + q;
+                v[q] = i < NC ? S.csum[i] : 0;
+                t += v[q];
+            }
+            int incl = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int run = incl - t;
+#pragma unroll
+            for (int q = 0; q < PER; ++q) {
+                const int i = lane * PER + q;
+                if (i < NC) S.csum[i] = run;
+                run += v[q];
+            }
+            if (lane == 31) S.total = incl;
+        }
+        named_bar_sync(bar, NT);
+        const uint32_t chunk = (uint32_t)S.total;
+        if (before + chunk >= need) {  // the need-th tie is in this chunk
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if ((bal[u] >> lane) & 1u) {
+                    const uint32_t rank = before + (uint32_t)S.csum[u * NW + warp] +
+                                          (uint32_t)__popc(bal[u] & ((1u << lane) - 1u));
+                    if (rank + 1 == need) S.red[0][0] = (uint32_t)a.index(c0 + u * NT + tid);
+                }
+            }
+            named_bar_sync(bar, NT);
+            const int32_t r = (int32_t)S.red[0][0];
+            named_bar_sync(bar, NT);
+            return r;
+        }
+        before += chunk;
+        named_bar_sync(bar, NT);
+    }
+    return 0x7fffffff;  // not reached: need <= number of ties
 }
 
 // Per-thread register cache of the ordered scores: entry e = tid + r * NT
@@ -211,15 +279,9 @@ __device__ uint64_t kth_largest(const A& a, int n, int k, uint32_t floor, Scratc
     uint32_t ilo = (uint32_t)imin, ihi = (uint32_t)imax;
     blk_minmax<NT>(ilo, ihi, S, parity, bar, tid);
     if (need == neq) return make_key(s, (int32_t)ihi);  // every tie is selected
-    // smallest m with count(ord == s && index <= m) >= need
-    while (ilo < ihi) {
-        const uint32_t mid = ilo + (ihi - ilo) / 2;
-        uint32_t c = 0;
-        for (int e = tid; e < n; e += NT) c += a.ord(e) == s && (uint32_t)a.index(e) <= mid;
-        if (blk_sum<NT>(c, S, parity, bar, tid) >= need) ihi = mid;
-        else ilo = mid + 1;
-    }
-    return make_key(s, (int32_t)ilo);
+    // Entries are in ascending index order, so the need-th lowest index among
+    // the ties is the index of the need-th tie in position order.
+    return make_key(s, nth_in_order<NT>(a, n, s, need, S, bar, tid));
 }
 
 // Writes, in order, the entries of [0, n) whose key is >= kth to out_so /
@@ -297,28 +359,88 @@ __device__ int compact(const A& a, int n, uint64_t kth, uint32_t* out_so, int32_
     return out_base;
 }
 
+// A threshold ord th with k <= count(ord >= th) <= max_keep, found from a
+// sample: each thread contributes one cached score, the sample's rank that
+// matches k plus a margin of three standard errors gives th, and one counting
+// pass checks both bounds.  Returns 0 when the check fails (the caller then
+// selects exactly).
+// Keeping every entry with ord >= th is a valid compaction: at least k kept
+// entries beat any later key whose ord is <= th.
+template <int R>
+__device__ uint32_t sampled_threshold(const uint32_t (&oc)[R], int n, int k, int max_keep,
+                                      Scratch<128>& S, int& parity, uint32_t bar, int tid) {
+    const int rounds = (n + 127) / 128;
+    const int pick = tid % rounds;
+    uint32_t mine = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) mine = r == pick ? oc[r] : mine;
+    if (tid + pick * 128 >= n) mine = 0;
+    S.samp[tid] = mine;
+    named_bar_sync(bar, 128);
+    // rank of this sample (descending; ties by thread id)
+    int rank = 0;
+    const uint4* s4 = reinterpret_cast<const uint4*>(S.samp);
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {
+        const uint4 v = s4[i];
+        rank += (v.x > mine) || (v.x == mine && 4 * i + 0 < tid);
+        rank += (v.y > mine) || (v.y == mine && 4 * i + 1 < tid);
+        rank += (v.z > mine) || (v.z == mine && 4 * i + 2 < tid);
+        rank += (v.w > mine) || (v.w == mine && 4 * i + 3 < tid);
+    }
+    // target: k plus 3 sigma of the sample quantile, in entries
+    const float pk = (float)k / (float)n;
+    const float sig = sqrtf(pk * (1.f - pk) / 128.f);
+    int target = (int)(128.f * (pk + 3.f * sig));
+    target = target > 127 ? 127 : target;
+    named_bar_sync(bar, 128);  // every rank read the samples before they are overwritten
+    if (rank == target) S.samp[0] = mine;
+    named_bar_sync(bar, 128);
+    const uint32_t th = S.samp[0];
+    uint32_t c = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) c += oc[r] >= th;
+    const uint32_t tot = blk_sum<128>(c, S, parity, bar, tid);
+    return (th != 0 && tot >= (uint32_t)k && (int)tot <= max_keep) ? th : 0u;
+}
+
 // Streaming top-k of one query over keys offered in batches of up to T tiles
 // of 128 (one key per thread of a warpgroup per tile, warp q holding keys
 // 32q..32q+31 of each tile), in ascending key order across batches.
 // Candidates that beat the threshold go to a buffer in key order; when it
 // fills, the k best are kept in order and the threshold rises to the k-th
 // score.  A later key that only ties the threshold can never enter (it would
-// lose the tie on its higher index), so `ord > theta` is exact.  One
-// warpgroup barrier per batch.
-template <int T>
+// lose the tie on its higher index), so `ord > theta` is exact.
+//
+// Several such streams (one per warpgroup, G of them) run in lockstep: each
+// batch ends with one barrier over all G * 128 threads, after which every
+// stream sees every stream's counts, and if any buffer is near full they all
+// compact at once (each with its own warpgroup barrier), so the compactions
+// overlap instead of stalling the shared MMA pipeline one after another.
+template <int T, int G>
 struct WgTopk {
     uint32_t* so;
     int32_t* ix;
     Scratch<128>* S;
-    int (*wcnt)[T][4];  // [2][T][4] per-warp append counts, double-buffered by batch
+    int (*wcnt)[G][T][4];  // [2][G][T][4] per-warp append counts of the batch
+    int (*cnts)[G];        // [2][G] buffer counts at the start of the batch
+    int j;                 // this stream
     int cap, k;
-    uint32_t bar;
+    uint32_t bar;          // this warpgroup's barrier
+    uint32_t gbar;         // barrier over all G warpgroups
     int tid;
-    uint32_t theta;     // ord of the threshold score (0: take everything)
+    uint32_t theta;        // ord of the threshold score (0: take everything)
     int cnt;
-    int parity;
+    int parity;            // batch parity: both shared arrays are double-buffered by it
 
-    // take[u]: key of tile u is visible; ord[u], s[u]: its score and index.
+    // Call once, before the first offer, from every thread of the stream.
+    __device__ __forceinline__ void start() {
+        cnt = 0;
+        theta = 0u;
+        if (tid == 0) cnts[parity][j] = 0;
+    }
+
+    // take[u]: key of tile u is visible; o[u], s[u]: its ordered score and index.
     __device__ __forceinline__ void offer(const bool (&take_in)[T], const uint32_t (&o)[T],
                                           const int32_t (&s)[T], int ntile) {
         const int lane = tid & 31, q = tid >> 5;
@@ -326,33 +448,66 @@ struct WgTopk {
 #pragma unroll
         for (int u = 0; u < T; ++u) {
             bal[u] = __ballot_sync(0xffffffffu, u < ntile && take_in[u] && o[u] > theta);
-            if (lane == 0) wcnt[parity][u][q] = __popc(bal[u]);
+            if (lane == 0) wcnt[parity][j][u][q] = __popc(bal[u]);
         }
-        named_bar_sync(bar, 128);
+        // One barrier per batch: the writes of batch b land in slot b % 2 and
+        // are read only between this barrier and the next one, which no
+        // thread passes before every thread has finished reading.
+        named_bar_sync(gbar, G * 128);
         const uint32_t below = (1u << lane) - 1u;
+        bool full = false;
 #pragma unroll
-        for (int u = 0; u < T; ++u) {
-            const int4 c = *reinterpret_cast<const int4*>(wcnt[parity][u]);
-            const int before = (q > 0 ? c.x : 0) + (q > 1 ? c.y : 0) + (q > 2 ? c.z : 0);
-            if ((bal[u] >> lane) & 1u) {
-                const int pos = cnt + before + __popc(bal[u] & below);
-                so[pos] = o[u];
-                ix[pos] = s[u];
+        for (int g = 0; g < G; ++g) {
+            int c = cnts[parity][g];
+#pragma unroll
+            for (int u = 0; u < T; ++u) {
+                const int4 w4 = *reinterpret_cast<const int4*>(wcnt[parity][g][u]);
+                if (g == j && ((bal[u] >> lane) & 1u)) {
+                    const int before = (q > 0 ? w4.x : 0) + (q > 1 ? w4.y : 0) + (q > 2 ? w4.z : 0);
+                    const int pos = c + before + __popc(bal[u] & below);
+                    so[pos] = o[u];
+                    ix[pos] = s[u];
+                }
+                c += w4.x + w4.y + w4.z + w4.w;
             }
-            cnt += c.x + c.y + c.z + c.w;
+            if (g == j) cnt = c;
+            full |= c > cap - T * 128;
         }
         parity ^= 1;
-        if (cnt > cap - T * 128) reduce(true);
+        if (full) reduce(false);  // every stream at once
+        else if (tid == 0) cnts[parity][j] = cnt;
     }
 
-    // Keeps the k best of the buffer (if it holds more), in key order.
-    __device__ void reduce(bool raise_theta) {
+    // Shrinks the buffer and publishes the count for the next batch.  The
+    // final call (exact = true) keeps exactly the k best, in key order; the
+    // intermediate ones keep every entry at or above a sampled threshold
+    // (at least k of them), which is cheaper and equally safe.
+    __device__ void reduce(bool exact) {
         named_bar_sync(bar, 128);
-        if (cnt <= k) return;
-        const FlatAccess a{so, ix};
-        const uint64_t kth = kth_largest<128, 32>(a, cnt, k, theta, *S, bar, tid);
-        cnt = compact<128>(a, cnt, kth, so, ix, *S, bar, tid);
-        if (raise_theta) theta = (uint32_t)(kth >> 32);
+        if (cnt > k) {
+            const FlatAccess a{so, ix};
+            uint32_t th = 0;
+            if (!exact) {
+                uint32_t oc[32];
+                load_ords<128, 32>(a, cnt, tid, oc);
+                int par = 0;
+                // keep at most half-way between k and the compaction trigger, so
+                // the next batch always fits and the compaction frees real room
+                const int max_keep = (k + (cap - T * 128)) / 2;
+                th = sampled_threshold<32>(oc, cnt, k, max_keep, *S, par, bar, tid);
+            }
+            uint64_t kth;
+            if (th != 0) {
+                kth = make_key(th, 0x7fffffff);  // every entry with ord >= th
+            } else {
+                if (!exact) named_bar_sync(bar, 128);  // the sampler's partials are read
+                kth = kth_largest<128, 32>(a, cnt, k, theta, *S, bar, tid);
+                th = (uint32_t)(kth >> 32);
+            }
+            cnt = compact<128>(a, cnt, kth, so, ix, *S, bar, tid);
+            if (!exact) theta = th;
+        }
+        if (tid == 0) cnts[parity][j] = cnt;
     }
 };
 

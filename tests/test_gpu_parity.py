@@ -227,3 +227,49 @@ def test_decode_equals_prefill_last_row():
     assert torch.equal(idx_d, idx_p[tt])
     diff = (O_d.float() - O_p[tt].float()).abs()
     assert diff.max().item() <= 2 ** -7  # same keys, split vs one-pass softmax order
+
+
+def _ascending_case(L, H, d, seed):
+    """Indexer inputs whose scores rise with the key index (with ties): q = 1
+    everywhere, key s holds a count of +1 entries that grows with s."""
+    rng = np.random.default_rng(seed)
+    q = np.ones((L, H, d))
+    kI = -np.ones((L, d))
+    ones = np.minimum((np.arange(L) * d) // L + rng.integers(0, 2, L), d)
+    for s in range(L):
+        kI[s, :ones[s]] = 1.0
+    w = rng.integers(0, 4, (L, H)).astype(np.float32)
+    return gen.encode_e4m3(q), gen.encode_e4m3(kI), w
+
+
+@pytest.mark.parametrize("L,k", [(4000, 256), (5000, 2048), (3001, 64)])
+def test_index_topk_ascending_scores_stress(L, k):
+    q, kI, w = _ascending_case(L, 64, 128, seed=L + k)
+    rows = np.array(sorted({0, k - 1, k, L // 2, L - 2, L - 1} | set(range(0, L, 97))), np.int64)
+    ref = oracle.index_topk(q, kI, w, k, rows=rows)
+    got = dsa.index_topk(dev(q), dev(kI), dev(w), k).cpu().numpy()[rows]
+    no_device_error()
+    assert np.array_equal(got, ref)
+
+
+def test_decode_ascending_scores_stress():
+    L = 70000
+    q, kI, w = _ascending_case(L, 64, 128, seed=3)
+    lens = np.array([L, 30000, 5], np.int64)
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    kI_c = np.concatenate([kI[:n] for n in lens])
+    cfg = gen.Config(0, "stress", "decode", k=2048, H_I=64, d_I=128, Hq=32, Hkv=4, d=128, B=3,
+                     seed=5)
+    Q = gen.normal_bf16(5, 4, 0, 3 * 32 * 128).reshape(3, 32, 128)
+    N = int(off[-1])
+    K = gen.normal_bf16(5, 5, 0, N * 512).reshape(N, 4, 128)
+    V = gen.normal_bf16(5, 6, 0, N * 512).reshape(N, 4, 128)
+    qd, wd = q[lens - 1], w[lens - 1]
+    r_idx, r_O = oracle.decode(qd, wd, Q, kI_c, K, V, off, cfg.k, cfg.scale)
+    idx = torch.empty((3, cfg.k), dtype=torch.int32, device="cuda")
+    O, _ = dsa.sparse_attn_decode(dev(qd), dev(wd), dev(Q, torch.bfloat16), dev(kI_c),
+                                  dev(K, torch.bfloat16), dev(V, torch.bfloat16), dev(off), cfg.k,
+                                  cfg.scale, idx_out=idx)
+    no_device_error()
+    assert np.array_equal(idx.cpu().numpy(), r_idx)
+    check_attn(O, r_O)
