@@ -188,8 +188,10 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     if (r0 >= r1) return;  // more CTAs than ranges: nothing to do
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Aligned by pointer arithmetic on the shared array itself (not through an
+    // integer), so that the compiler keeps every access in the shared window
+    // (ld/st.shared with 32-bit addresses instead of generic ones).
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const Layout lay(p.k);
     const int cap = cand_capacity(p.k);
     Misc* misc = reinterpret_cast<Misc*>(smem + lay.misc);

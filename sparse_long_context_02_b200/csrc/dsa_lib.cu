@@ -109,6 +109,13 @@ dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, cons
     if (smem > max_optin_smem())
         return fail(DSA_ERR_UNSUPPORTED, "%s: needs %d bytes of shared memory", fn, smem);
     auto kern = dsa::idx::index_kernel<HI, DI, TOPK>;
+    // The kernel re-splits its registers between warpgroups (setmaxnreg);
+    // the split adds up only if every thread starts with exactly 96.
+    cudaFuncAttributes fa;
+    CUDA_TRY(cudaFuncGetAttributes(&fa, kern));
+    if (fa.numRegs != 96)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: kernel built with %d registers per thread, not 96",
+                    fn, fa.numRegs);
     CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     dsa::idx::Params p;
     p.w = w;

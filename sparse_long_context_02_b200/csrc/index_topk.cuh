@@ -38,7 +38,13 @@ constexpr int kStages = 3;        // depth of the key-tile ring
 constexpr int kEpiWarps = 16;     // warps 0-15
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
-constexpr int kThreads = 18 * 32;
+constexpr int kThreads = 20 * 32;  // warps 18-19 idle: warpgroup 4 is whole for setmaxnreg
+// Register split (setmaxnreg): the launch gives every thread 96 registers
+// (640 * 96 = 61440); warpgroup 4 drops to 32 and the four epilogue
+// warpgroups rise to 112: 4 * 128 * 112 + 128 * 32 = 61440.
+constexpr int kEpiRegs = 112;
+constexpr int kCtlRegs = 32;
+static_assert(4 * 128 * kEpiRegs + 128 * kCtlRegs <= kThreads * 96, "register split");
 constexpr int kBatch = 4;         // tiles offered to the top-k per barrier
 constexpr uint32_t kAllEpilogueBar = 5;  // named barrier over the 512 epilogue threads
 
@@ -159,8 +165,10 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     static_assert(DI == 64 || DI == 128, "d_I");
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Aligned by pointer arithmetic on the shared array itself (not through an
+    // integer), so that the compiler keeps every access in the shared window
+    // (ld/st.shared with 32-bit addresses instead of generic ones).
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const Layout lay(HI, DI, p.k, TOPK);
     const int cap = TOPK ? cand_capacity(p.k) : 0;
     Misc* misc = reinterpret_cast<Misc*>(smem + lay.misc);
@@ -201,6 +209,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem_base = misc->tmem_base;
 
+    if (warp >= kEpiWarps) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -257,8 +266,9 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             umma_commit(smem_u32(&misc->mma_done));
             mbar_wait(smem_u32(&misc->mma_done), 0);
         }
-    } else {
+    } else if (warp < kEpiWarps) {
         // ------------------------------------------------ epilogue (warps 0-15)
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
         const int j = warp >> 2;              // token of this warpgroup
         const int q = warp & 3;               // TMEM lane quarter
         const int tid = threadIdx.x - j * 128;

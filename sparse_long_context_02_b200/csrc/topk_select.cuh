@@ -454,24 +454,38 @@ struct WgTopk {
         // are read only between this barrier and the next one, which no
         // thread passes before every thread has finished reading.
         named_bar_sync(gbar, G * 128);
+        static_assert(G * T <= 32, "one lane per (stream, tile)");
         const uint32_t below = (1u << lane) - 1u;
-        bool full = false;
+        // Lane g * T + u reads the four warp counts of stream g, tile u; a
+        // segmented scan over u gives every stream's count after the batch
+        // and, for this warp's stream, where its offers of each tile go.
+        const int gl = lane / T, ul = lane % T;
+        int tot = 0, bq = 0, c0 = 0;
+        if (lane < G * T) {
+            const int4 w4 = *reinterpret_cast<const int4*>(wcnt[parity][gl][ul]);
+            tot = w4.x + w4.y + w4.z + w4.w;
+            bq = (q > 0 ? w4.x : 0) + (q > 1 ? w4.y : 0) + (q > 2 ? w4.z : 0);
+            c0 = cnts[parity][gl];
+        }
+        int incl = tot;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            int c = cnts[parity][g];
+        for (int d = 1; d < T; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (ul >= d) incl += y;
+        }
+        const int base = c0 + incl - tot + bq;  // first slot of this warp's offers of (g, u)
+        const int after = c0 + __shfl_sync(0xffffffffu, incl, (gl * T + T - 1) & 31);
+        const bool full =
+            __any_sync(0xffffffffu, lane < G * T && ul == T - 1 && after > cap - T * 128);
+        cnt = __shfl_sync(0xffffffffu, after, j * T);
 #pragma unroll
-            for (int u = 0; u < T; ++u) {
-                const int4 w4 = *reinterpret_cast<const int4*>(wcnt[parity][g][u]);
-                if (g == j && ((bal[u] >> lane) & 1u)) {
-                    const int before = (q > 0 ? w4.x : 0) + (q > 1 ? w4.y : 0) + (q > 2 ? w4.z : 0);
-                    const int pos = c + before + __popc(bal[u] & below);
-                    so[pos] = o[u];
-                    ix[pos] = s[u];
-                }
-                c += w4.x + w4.y + w4.z + w4.w;
+        for (int u = 0; u < T; ++u) {
+            const int bu = __shfl_sync(0xffffffffu, base, j * T + u);
+            if ((bal[u] >> lane) & 1u) {
+                const int pos = bu + __popc(bal[u] & below);
+                so[pos] = o[u];
+                ix[pos] = s[u];
             }
-            if (g == j) cnt = c;
-            full |= c > cap - T * 128;
         }
         parity ^= 1;
         if (full) reduce(false);  // every stream at once
