@@ -141,6 +141,26 @@ __device__ __forceinline__ float head_sum(uint32_t taddr, const float* wj) {
     }
 }
 
+
+// Weighted head sum with the token's 64 weights held in registers as f32
+// pairs: no shared-memory reads beside the tensor core's operand fetches,
+// which are what the tile rate depends on.  Same arithmetic and exactness as
+// head_sum above.
+__device__ __forceinline__ float head_sum_w2(uint32_t taddr, const uint64_t (&w2)[32]) {
+    uint64_t acc[2] = {0ull, 0ull};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float v[16];
+        tmem_ld_32x32b_x16(taddr + c * 16, v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            fma2(acc[0], w2[c * 8 + 2 * q], pack2(fmaxf(v[4 * q], 0.f), fmaxf(v[4 * q + 1], 0.f)));
+            fma2(acc[1], w2[c * 8 + 2 * q + 1], pack2(fmaxf(v[4 * q + 2], 0.f), fmaxf(v[4 * q + 3], 0.f)));
+        }
+    }
+    return (sum2(acc[0]) + sum2(acc[1])) + 0.0f;
+}
+
 // ---------------------------------------------------------------- kernel
 
 struct Params {
@@ -287,6 +307,16 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         // without waiting (results are discarded), so every warp of the
         // warpgroup still meets every barrier.
         for (int i0 = 0; i0 < ntiles; i0 += kBatch) {
+            uint64_t w2[32];  // the token's weights, reloaded per batch: dead across offers,
+                              // so the compactions have the registers
+            if constexpr (HI == 64) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const float4 f = reinterpret_cast<const float4*>(wj)[c];
+                    w2[2 * c] = pack2(f.x, f.y);
+                    w2[2 * c + 1] = pack2(f.z, f.w);
+                }
+            }
             bool take[kBatch];
             uint32_t o[kBatch];
             int32_t sk[kBatch];
@@ -303,7 +333,9 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 tc_fence_after();
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * N + j * HI);
-                const float score = head_sum<HI>(taddr, wj);
+                float score;
+                if constexpr (HI == 64) score = head_sum_w2(taddr, w2);
+                else score = head_sum<HI>(taddr, wj);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&misc->accempty[buf]));

@@ -404,6 +404,101 @@ __device__ uint32_t sampled_threshold(const uint32_t (&oc)[R], int n, int k, int
     return (th != 0 && tot >= (uint32_t)k && (int)tot <= max_keep) ? th : 0u;
 }
 
+// Intermediate compaction of a flat buffer of n <= 32 * 128 entries: keeps,
+// in order, every entry whose ord is at least th, where th is the element of
+// descending rank `target` of a 128-entry sample (one cached score per
+// thread), provided that leaves between k and max_keep entries; otherwise
+// returns false with the buffer untouched.  One warp (sel_warp) finds th by
+// a bitwise search over the sample; the counts per (round, warp) go through
+// one barrier, and the indices of kept entries are read before it, so the
+// writes after it may land on entries that other threads have read already:
+// the compaction runs in place with three barriers.
+__device__ bool compact_sampled(uint32_t* so, int32_t* ix, int& n_io, int k, int max_keep,
+                                Scratch<128>& S, uint32_t bar, int tid, int sel_warp,
+                                uint32_t& th_out) {
+    constexpr int R = 32;
+    const int n = n_io;
+    const int lane = tid & 31, warp = tid >> 5;
+    uint32_t oc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = tid + r * 128;
+        oc[r] = e < n ? so[e] : 0u;
+    }
+    // ---- sample: entry tid + pick * 128 of every thread
+    const int rounds = (n + 127) / 128;
+    const int pick = tid % rounds;
+    uint32_t mine = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) mine = r == pick ? oc[r] : mine;
+    if (tid + pick * 128 >= n) mine = 0;
+    S.samp[tid] = mine;
+    // target rank: k plus three standard errors of the sample quantile
+    const float pk = (float)k / (float)n;
+    const float sig = sqrtf(pk * (1.f - pk) / 128.f);
+    int target = (int)(128.f * (pk + 3.f * sig));
+    target = target > 127 ? 127 : target;
+    named_bar_sync(bar, 128);
+    if (warp == sel_warp) {
+        // the largest x with at least target + 1 samples >= x: that sample
+        const uint4 v = reinterpret_cast<const uint4*>(S.samp)[lane];
+        uint32_t x = 0;
+#pragma unroll 4
+        for (int b = 31; b >= 0; --b) {
+            const uint32_t c = x | (1u << b);
+            const uint32_t m = __reduce_add_sync(
+                0xffffffffu, (uint32_t)(v.x >= c) + (uint32_t)(v.y >= c) + (uint32_t)(v.z >= c) +
+                                 (uint32_t)(v.w >= c));
+            if (m >= (uint32_t)target + 1u) x = c;
+        }
+        if (lane == 0) S.total = (int)x;
+    }
+    named_bar_sync(bar, 128);
+    const uint32_t th = (uint32_t)S.total;
+    // ---- kept entries per (round, warp); indices of kept entries to registers
+    int32_t ic[R];
+    int* cnt4 = reinterpret_cast<int*>(S.samp);  // the sample is no longer read
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = tid + r * 128;
+        const bool keep = e < n && oc[r] >= th;
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) cnt4[r * 4 + warp] = __popc(bal);
+        ic[r] = keep ? ix[e] : 0;
+    }
+    named_bar_sync(bar, 128);
+    // lane r scans round r: exclusive prefix of the rounds before it, plus
+    // the warps before this one within the round
+    const int4 c4 = reinterpret_cast<const int4*>(cnt4)[lane];
+    const int tot = c4.x + c4.y + c4.z + c4.w;
+    int incl = tot;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    const int basew =
+        incl - tot + (warp > 0 ? c4.x : 0) + (warp > 1 ? c4.y : 0) + (warp > 2 ? c4.z : 0);
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (th == 0 || total < k || total > max_keep) return false;  // same answer in every thread
+    const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int b = __shfl_sync(0xffffffffu, basew, r);
+        const int e = tid + r * 128;
+        const bool keep = e < n && oc[r] >= th;
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+            const int pos = b + __popc(bal & below);
+            so[pos] = oc[r];
+            ix[pos] = ic[r];
+        }
+    }
+    n_io = total;
+    th_out = th;
+    return true;
+}
+
 // Streaming top-k of one query over keys offered in batches of up to T tiles
 // of 128 (one key per thread of a warpgroup per tile, warp q holding keys
 // 32q..32q+31 of each tile), in ascending key order across batches.
@@ -499,27 +594,22 @@ struct WgTopk {
     __device__ void reduce(bool exact) {
         named_bar_sync(bar, 128);
         if (cnt > k) {
-            const FlatAccess a{so, ix};
-            uint32_t th = 0;
-            if (!exact) {
-                uint32_t oc[32];
-                load_ords<128, 32>(a, cnt, tid, oc);
-                int par = 0;
+            bool done = false;
+            if (!exact && cnt <= 32 * 128) {
                 // keep at most half-way between k and the compaction trigger, so
                 // the next batch always fits and the compaction frees real room
                 const int max_keep = (k + (cap - T * 128)) / 2;
-                th = sampled_threshold<32>(oc, cnt, k, max_keep, *S, par, bar, tid);
+                uint32_t th = 0;
+                done = compact_sampled(so, ix, cnt, k, max_keep, *S, bar, tid, j & 3, th);
+                if (done) theta = th;
+                else named_bar_sync(bar, 128);  // every thread is past the sampler
             }
-            uint64_t kth;
-            if (th != 0) {
-                kth = make_key(th, 0x7fffffff);  // every entry with ord >= th
-            } else {
-                if (!exact) named_bar_sync(bar, 128);  // the sampler's partials are read
-                kth = kth_largest<128, 32>(a, cnt, k, theta, *S, bar, tid);
-                th = (uint32_t)(kth >> 32);
+            if (!done) {
+                const FlatAccess a{so, ix};
+                const uint64_t kth = kth_largest<128, 32>(a, cnt, k, theta, *S, bar, tid);
+                cnt = compact<128>(a, cnt, kth, so, ix, *S, bar, tid);
+                if (!exact) theta = (uint32_t)(kth >> 32);
             }
-            cnt = compact<128>(a, cnt, kth, so, ix, *S, bar, tid);
-            if (!exact) theta = th;
         }
         if (tid == 0) cnts[parity][j] = cnt;
     }
