@@ -31,7 +31,6 @@ namespace dsa {
 namespace dec {
 
 using idx::kKeyTile;
-using idx::cand_capacity;
 using sel::FlatAccess;
 using sel::Scratch;
 using sel::SegAccess;
@@ -40,6 +39,13 @@ using sel::WgTopk;
 constexpr int HI = 64;
 constexpr int DI = 128;
 constexpr int kStages = 5;        // HBM-bound: keep more key tiles in flight
+constexpr int kBatch = 4;         // tiles offered to the top-k per barrier
+// Candidate buffer entries per query: room for the k kept plus one batch of
+// offers, and 2k so that a compaction frees at least k.
+__host__ __device__ constexpr int cand_capacity(int k) {
+    const int c = 2 * k > k + kBatch * kKeyTile ? 2 * k : k + kBatch * kKeyTile;
+    return (c + 127) / 128 * 128;
+}
 constexpr int kEpiWarps = 16;     // warps 0-15: four warpgroups, one per chunk quarter
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
@@ -109,7 +115,7 @@ struct Misc {
     uint64_t accfull[4][2];
     uint64_t accempty[4][2];
     uint64_t mma_done;
-    alignas(16) int wcnt[2][4][idx::kBatch][4];  // rows read as int4 by WgTopk::offer
+    alignas(16) int wcnt[2][4][kBatch][4];  // rows read as int4 by WgTopk::offer
     int cnts[2][4];
     int cnt[4];
     uint32_t tmem_base;
@@ -321,7 +327,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         int32_t* ix = reinterpret_cast<int32_t*>(smem + lay.ci) + w * cap;
         float* w_s = reinterpret_cast<float*>(smem + lay.w) + w * HI;
         Scratch<128>* S = reinterpret_cast<Scratch<128>*>(smem + lay.scratch) + w;
-        constexpr int T = idx::kBatch;
+        constexpr int T = kBatch;
         int use = 0;
         Segment g;
         for (int b = b_first; b < p.B && p.cache_off[b] < r1; ++b) {
@@ -337,15 +343,11 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             const int nt0 = g.tiles(0);  // quarter 0 has the most tiles: every warpgroup
                                          // runs its batch count, offering nothing at the end
             for (int u0 = 0; u0 < nt0; u0 += T) {
-                bool take[T];
-                uint32_t o[T];
-                int32_t sk[T];
+                uint32_t o[T];  // ord of this thread's key in each tile; 0 = not offered
 #pragma unroll
                 for (int v = 0; v < T; ++v) {
                     const int u = u0 + v;
-                    take[v] = false;
                     o[v] = 0;
-                    sk[v] = 0;
                     if (u >= ntw) continue;
                     const int buf = use & 1;
                     if (!misc->abort_flag &&
@@ -360,11 +362,10 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                     if (lane == 0) mbar_arrive(smem_u32(&misc->accempty[w][buf]));
                     ++use;
                     const int64_t s = qlo + (int64_t)u * kKeyTile + q * 32 + lane;
-                    take[v] = s < qend;
-                    o[v] = sel::ord_f32(score);
-                    sk[v] = (int32_t)s;
+                    if (s < qend) o[v] = sel::ord_f32(score);
                 }
-                tk.offer(take, o, sk, ntw - u0 < T ? (ntw - u0 > 0 ? ntw - u0 : 0) : T);
+                tk.offer(o, (int32_t)(qlo + (int64_t)u0 * kKeyTile + q * 32 + lane),
+                         ntw - u0 < T ? (ntw - u0 > 0 ? ntw - u0 : 0) : T);
             }
             tk.reduce(true);
             if (tid == 0) misc->cnt[w] = tk.cnt;

@@ -34,7 +34,7 @@ using sel::WgTopk;  // WgTopk<T, G>
 
 constexpr int kTokens = 4;        // query tokens per CTA
 constexpr int kKeyTile = 128;     // keys per tile (MMA M)
-constexpr int kStages = 3;        // depth of the key-tile ring
+constexpr int kStages = 2;        // depth of the key-tile ring (kI is L2-resident)
 constexpr int kEpiWarps = 16;     // warps 0-15
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
@@ -45,14 +45,18 @@ constexpr int kThreads = 20 * 32;  // warps 18-19 idle: warpgroup 4 is whole for
 constexpr int kEpiRegs = 112;
 constexpr int kCtlRegs = 32;
 static_assert(4 * 128 * kEpiRegs + 128 * kCtlRegs <= kThreads * 96, "register split");
-constexpr int kBatch = 4;         // tiles offered to the top-k per barrier
+constexpr int kBatch = 8;         // tiles offered to the top-k per barrier
 constexpr uint32_t kAllEpilogueBar = 5;  // named barrier over the 512 epilogue threads
 
-// Candidate buffer entries per query: room for the k kept plus at least one
-// full batch of offers (and 2k, so that a compaction frees at least k).
-__host__ __device__ constexpr int cand_capacity(int k) {
-    int c = 2 * k > k + kBatch * kKeyTile ? 2 * k : k + kBatch * kKeyTile;
-    return (c + 127) / 128 * 128;
+// Candidate buffer entries per query.  A compaction starts once a batch
+// leaves more than cap - kBatch * 128 entries (so the next batch always
+// fits) and keeps at most half-way between k and that mark, so cap should
+// exceed k by well over one batch: 2k + 512 for the usual k (4608 entries
+// at k = 2048, which the shared-memory budget allows with a two-stage key
+// ring), and at least k + one batch + 512 for small k.
+__host__ __device__ constexpr int cand_capacity(int k, int batch) {
+    const int a = 2 * k + 512, b = k + batch * kKeyTile + 512;
+    return ((a > b ? a : b) + 127) / 128 * 128;
 }
 
 // Misc block: barriers and the small shared state.
@@ -76,7 +80,7 @@ struct Layout {
     int q, stage, w, cs, ci, scratch, misc, total;
     __host__ __device__ Layout(int HI, int DI, int k, bool topk) {
         const int n = kTokens * HI;
-        const int cap = topk ? cand_capacity(k) : 0;
+        const int cap = topk ? cand_capacity(k, kBatch) : 0;
         q = 0;
         stage = (n * DI + 1023) / 1024 * 1024;
         w = stage + kStages * kKeyTile * DI;
@@ -190,7 +194,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     // (ld/st.shared with 32-bit addresses instead of generic ones).
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const Layout lay(HI, DI, p.k, TOPK);
-    const int cap = TOPK ? cand_capacity(p.k) : 0;
+    const int cap = TOPK ? cand_capacity(p.k, kBatch) : 0;
     Misc* misc = reinterpret_cast<Misc*>(smem + lay.misc);
     float* w_s = reinterpret_cast<float*>(smem + lay.w);
 
@@ -317,15 +321,11 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                     w2[2 * c + 1] = pack2(f.z, f.w);
                 }
             }
-            bool take[kBatch];
-            uint32_t o[kBatch];
-            int32_t sk[kBatch];
+            uint32_t o[kBatch];  // ord of this thread's key in each tile; 0 = not visible
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
                 const int i = i0 + u;
-                take[u] = false;
                 o[u] = 0;
-                sk[u] = 0;
                 if (i >= ntiles) continue;
                 const int buf = i & 1;
                 if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->accfull[buf]), (i >> 1) & 1))
@@ -341,15 +341,14 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 if (lane == 0) mbar_arrive(smem_u32(&misc->accempty[buf]));
                 const int64_t s = (int64_t)i * kKeyTile + q * 32 + lane;
                 if constexpr (TOPK) {
-                    take[u] = trow && s <= t;
-                    o[u] = sel::ord_f32(score);
-                    sk[u] = (int32_t)s;
+                    if (trow && s <= t) o[u] = sel::ord_f32(score);
                 } else {
                     if (trow && s < L) p.scores[t * L + s] = s <= t ? score : -INFINITY;
                 }
             }
             if constexpr (TOPK)
-                tk.offer(take, o, sk, ntiles - i0 < kBatch ? ntiles - i0 : kBatch);
+                tk.offer(o, (int32_t)(i0 * kKeyTile + q * 32 + lane),
+                         ntiles - i0 < kBatch ? ntiles - i0 : kBatch);
         }
 
         if constexpr (TOPK) {

@@ -535,14 +535,15 @@ struct WgTopk {
         if (tid == 0) cnts[parity][j] = 0;
     }
 
-    // take[u]: key of tile u is visible; o[u], s[u]: its ordered score and index.
-    __device__ __forceinline__ void offer(const bool (&take_in)[T], const uint32_t (&o)[T],
-                                          const int32_t (&s)[T], int ntile) {
+    // o[u]: ordered score of this thread's key in tile u of the batch, 0 when
+    // the key is not visible (0 is below every threshold); its index is
+    // s0 + 128 u.
+    __device__ __forceinline__ void offer(const uint32_t (&o)[T], int32_t s0, int ntile) {
         const int lane = tid & 31, q = tid >> 5;
         uint32_t bal[T];
 #pragma unroll
         for (int u = 0; u < T; ++u) {
-            bal[u] = __ballot_sync(0xffffffffu, u < ntile && take_in[u] && o[u] > theta);
+            bal[u] = __ballot_sync(0xffffffffu, u < ntile && o[u] > theta);
             if (lane == 0) wcnt[parity][j][u][q] = __popc(bal[u]);
         }
         // One barrier per batch: the writes of batch b land in slot b % 2 and
@@ -579,7 +580,7 @@ struct WgTopk {
             if ((bal[u] >> lane) & 1u) {
                 const int pos = bu + __popc(bal[u] & below);
                 so[pos] = o[u];
-                ix[pos] = s[u];
+                ix[pos] = s0 + u * 128;
             }
         }
         parity ^= 1;
