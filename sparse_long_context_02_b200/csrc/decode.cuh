@@ -334,7 +334,9 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             if (!make_segment(p, b, r0, r1, g)) continue;
             if (tid < HI) w_s[tid] = p.w[(int64_t)g.b * HI + tid];
             named_bar_sync(bar, 128);
-            WgTopk<T, 4> tk{so, ix, S, misc->wcnt, misc->cnts, w, cap, p.k, bar, 5, tid, 0u, 0, 0};
+            // the four quarters split one query's keys: one threshold for the union
+            WgTopk<T, 4, true> tk{so, ix, S, misc->wcnt, misc->cnts, w, cap, p.k, bar, 5, tid,
+                                  0u, 0, 0, reinterpret_cast<Scratch<512>*>(smem + lay.scratch_all)};
             tk.start();
             const int64_t qlo = g.lo + (int64_t)w * g.sub;
             const int64_t qend = g.lo + ((int64_t)(w + 1) * g.sub < g.len ? (int64_t)(w + 1) * g.sub
@@ -367,7 +369,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 tk.offer(o, (int32_t)(qlo + (int64_t)u0 * kKeyTile + q * 32 + lane),
                          ntw - u0 < T ? (ntw - u0 > 0 ? ntw - u0 : 0) : T);
             }
-            tk.reduce(true);
+            tk.shrink_union();
             if (tid == 0) misc->cnt[w] = tk.cnt;
             // ---- merge the four quarter lists into the segment's top-k
             named_bar_sync(5, 512);

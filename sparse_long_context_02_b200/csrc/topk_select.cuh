@@ -499,6 +499,113 @@ __device__ bool compact_sampled(uint32_t* so, int32_t* ix, int& n_io, int k, int
     return true;
 }
 
+// Compaction of G streams at once (all G * 128 threads, stream j being
+// warpgroup j) whose keys are disjoint parts of ONE query's key set: a key
+// that k keys of the union beat can be dropped from any stream, so all
+// streams share one threshold th taken at the union's rank k (plus a margin)
+// from a 128-entry sample of each stream, weighted by the streams' sizes
+// ng[].  Each stream keeps its entries >= th, in order (its count may fall
+// below k).  Returns false, with nothing written, if th would leave fewer
+// than k or more than max_keep entries in the union.  Streams hold at most
+// 32 * 128 entries each.
+template <int G>
+__device__ bool compact_union(uint32_t* so, int32_t* ix, int& n_io, const int (&ng)[G], int k,
+                              int max_keep, Scratch<128>& S, Scratch<G * 128>& SA, uint32_t bar,
+                              uint32_t gbar, int j, int tid, uint32_t& th_out) {
+    constexpr int R = 32, NT = G * 128;
+    static_assert(NT / 32 == 4 * G && G <= 4, "one sampling lane group per stream");
+    const int n = n_io;
+    const int lane = tid & 31, warp = tid >> 5;
+    uint32_t oc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = tid + r * 128;
+        oc[r] = e < n ? so[e] : 0u;
+    }
+    const int rounds = n > 0 ? (n + 127) / 128 : 1;
+    const int pick = tid % rounds;
+    uint32_t mine = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) mine = r == pick ? oc[r] : mine;
+    SA.samp[j * 128 + tid] = mine;  // 0 (below everything) where there is no entry
+    int ntot = 0;
+#pragma unroll
+    for (int g = 0; g < G; ++g) ntot += ng[g];
+    // union rank to aim at: k plus three standard errors of the sample quantile
+    const float pk = (float)k / (float)ntot;
+    const float sig = sqrtf(pk * (1.f - pk) / (float)NT);
+    const float tgt = (pk + 3.f * sig) * (float)ntot;
+    const uint32_t target128 = (uint32_t)(tgt * 128.f);  // sample weights are ng / 128
+    named_bar_sync(gbar, NT);
+    if (j == 0 && warp == 0) {
+        // lane l holds samples PER l .. PER l + PER - 1, all of stream PER l / 128
+        constexpr int PER = NT / 32;
+        uint32_t v[PER];
+#pragma unroll
+        for (int i = 0; i < PER / 4; ++i) {
+            const uint4 q4 = reinterpret_cast<const uint4*>(SA.samp)[lane * (PER / 4) + i];
+            v[4 * i] = q4.x; v[4 * i + 1] = q4.y; v[4 * i + 2] = q4.z; v[4 * i + 3] = q4.w;
+        }
+        const uint32_t wt = (uint32_t)ng[(lane * PER) / 128];
+        uint32_t x = 0;
+#pragma unroll 2
+        for (int b = 31; b >= 0; --b) {
+            const uint32_t c = x | (1u << b);
+            uint32_t m = 0;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) m += (uint32_t)(v[i] >= c);
+            if (__reduce_add_sync(0xffffffffu, m * wt) >= target128) x = c;
+        }
+        if (lane == 0) SA.total = (int)x;
+    }
+    named_bar_sync(gbar, NT);
+    const uint32_t th = (uint32_t)SA.total;
+    int32_t ic[R];
+    int* cnt4 = reinterpret_cast<int*>(S.samp);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = tid + r * 128;
+        const bool keep = e < n && oc[r] >= th;
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) cnt4[r * 4 + warp] = __popc(bal);
+        ic[r] = keep ? ix[e] : 0;
+    }
+    named_bar_sync(bar, 128);
+    const int4 c4 = reinterpret_cast<const int4*>(cnt4)[lane];
+    const int tot = c4.x + c4.y + c4.z + c4.w;
+    int incl = tot;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    const int basew =
+        incl - tot + (warp > 0 ? c4.x : 0) + (warp > 1 ? c4.y : 0) + (warp > 2 ? c4.z : 0);
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (tid == 0) SA.red[0][j] = (uint32_t)total;
+    named_bar_sync(gbar, NT);
+    int utot = 0;
+#pragma unroll
+    for (int g = 0; g < G; ++g) utot += (int)SA.red[0][g];
+    if (th == 0 || utot < k || utot > max_keep) return false;  // same answer everywhere
+    const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int b = __shfl_sync(0xffffffffu, basew, r);
+        const int e = tid + r * 128;
+        const bool keep = e < n && oc[r] >= th;
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+            const int pos = b + __popc(bal & below);
+            so[pos] = oc[r];
+            ix[pos] = ic[r];
+        }
+    }
+    n_io = total;
+    th_out = th;
+    return true;
+}
+
 // Streaming top-k of one query over keys offered in batches of up to T tiles
 // of 128 (one key per thread of a warpgroup per tile, warp q holding keys
 // 32q..32q+31 of each tile), in ascending key order across batches.
@@ -512,7 +619,7 @@ __device__ bool compact_sampled(uint32_t* so, int32_t* ix, int& n_io, int k, int
 // stream sees every stream's counts, and if any buffer is near full they all
 // compact at once (each with its own warpgroup barrier), so the compactions
 // overlap instead of stalling the shared MMA pipeline one after another.
-template <int T, int G>
+template <int T, int G, bool UNION = false>
 struct WgTopk {
     uint32_t* so;
     int32_t* ix;
@@ -527,6 +634,9 @@ struct WgTopk {
     uint32_t theta;        // ord of the threshold score (0: take everything)
     int cnt;
     int parity;            // batch parity: both shared arrays are double-buffered by it
+    // UNION: the G streams split one query's keys; compactions then use one
+    // threshold for the union (compact_union), with this scratch.
+    Scratch<G * 128>* SA = nullptr;
 
     // Call once, before the first offer, from every thread of the stream.
     __device__ __forceinline__ void start() {
@@ -543,7 +653,11 @@ struct WgTopk {
         uint32_t bal[T];
 #pragma unroll
         for (int u = 0; u < T; ++u) {
-            bal[u] = __ballot_sync(0xffffffffu, u < ntile && o[u] > theta);
+            // One stream: a later key that only ties the threshold loses on its
+            // index, so it is not offered.  UNION streams interleave index
+            // ranges, so ties are kept and the final selection orders them.
+            const bool pass = UNION ? (o[u] != 0u && o[u] >= theta) : o[u] > theta;
+            bal[u] = __ballot_sync(0xffffffffu, u < ntile && pass);
             if (lane == 0) wcnt[parity][j][u][q] = __popc(bal[u]);
         }
         // One barrier per batch: the writes of batch b land in slot b % 2 and
@@ -584,8 +698,63 @@ struct WgTopk {
             }
         }
         parity ^= 1;
-        if (full) reduce(false);  // every stream at once
-        else if (tid == 0) cnts[parity][j] = cnt;
+        if (full) {  // every stream at once
+            if constexpr (UNION) {
+                int ng[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) ng[g] = __shfl_sync(0xffffffffu, after, (g * T + T - 1) & 31);
+                reduce_union(ng);
+            } else {
+                reduce(false);
+            }
+        } else if (tid == 0) {
+            cnts[parity][j] = cnt;
+        }
+    }
+
+    // Union compaction (UNION streams); falls back to each stream's own
+    // exact k-th when the shared threshold is out of bounds.
+    __device__ void reduce_union(const int (&ng)[G]) {
+        named_bar_sync(bar, 128);
+        bool done = false, small = true;
+#pragma unroll
+        for (int g = 0; g < G; ++g) small = small && ng[g] <= 32 * 128;
+        if (small) {
+            const int max_keep = (k + (cap - T * 128)) / 2;
+            uint32_t th = 0;
+            done = compact_union<G>(so, ix, cnt, ng, k, max_keep, *S, *SA, bar, gbar, j, tid, th);
+            if (done) theta = th;
+            else named_bar_sync(bar, 128);  // this stream's threads are past the counts
+        }
+        if (!done && cnt > k) {
+            const FlatAccess a{so, ix};
+            const uint64_t kth = kth_largest<128, 32>(a, cnt, k, theta, *S, bar, tid);
+            cnt = compact<128>(a, cnt, kth, so, ix, *S, bar, tid);
+            theta = (uint32_t)(kth >> 32);
+        }
+        if (tid == 0) cnts[parity][j] = cnt;
+    }
+
+    // UNION streams at the end of their keys: one more union compaction when
+    // the union holds more than max_keep entries (all G * 128 threads).
+    __device__ void shrink_union() {
+        named_bar_sync(gbar, G * 128);
+        int ng[G], ntot = 0;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            ng[g] = cnts[parity][g];
+            ntot += ng[g];
+        }
+        const int max_keep = (k + (cap - T * 128)) / 2;
+        bool small = true;
+#pragma unroll
+        for (int g = 0; g < G; ++g) small = small && ng[g] <= 32 * 128;
+        if (ntot > max_keep && small) {
+            uint32_t th = 0;
+            if (compact_union<G>(so, ix, cnt, ng, k, max_keep, *S, *SA, bar, gbar, j, tid, th))
+                theta = th;
+        }
+        named_bar_sync(gbar, G * 128);
     }
 
     // Shrinks the buffer and publishes the count for the next batch.  The
