@@ -90,6 +90,39 @@ def decode_bytes(cfg, lens) -> float:
             + cfg.B * (cfg.H_I * cfg.d_I + cfg.H_I * 4 + 2 * 2 * cfg.Hq * cfg.d))
 
 
+# ------------------------------------------------------------------ DRAM traffic
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch,
+# from one ncu capture of the prefill L=32768 case (its summary under
+# profiles/ncu_prefill32k_decode4_index_attn.md), per prefill query token:
+# the indexer's DRAM traffic is its queries, weights and index rows (the keys
+# stay in L2), so it grows with L.  Valid only for the CUDA sources the
+# counters were taken on (their SHA-256 below); otherwise null.
+TRAFFIC = {
+    "dsa_index_topk": dict(bytes_per_query_token=510171392 / 32768,
+                           src_sha256="769e3ff4e88fa327a5869516cac6d167a837a4fd10ed054d7e3a1249e9eef442"),
+}
+
+
+def csrc_sha256() -> str:
+    import glob
+    import hashlib
+    root = os.path.join(ROOT, "sparse_long_context_02_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(root, "*.cu")) + glob.glob(os.path.join(root, "*.cuh"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def dram_traffic(kernel: str, pcfg):
+    t = TRAFFIC.get(kernel)
+    if t is None or pcfg is None or t["src_sha256"] != csrc_sha256():
+        return None
+    return t["bytes_per_query_token"] * pcfg.L
+
+
 # ------------------------------------------------------------------ ranks
 
 def rank_workloads(pcfg, dcfg, rank: int, world: int):
@@ -336,13 +369,7 @@ def run_ours(args, rank, world, local_rank):
         v["frac"] = v["achieved"] / v["peak"]
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     dk = kernels[dom]
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            traffic = json.load(open(tpath)).get(dom)
-        except ValueError:
-            traffic = None
+    traffic = dram_traffic(dom, pcfg)
     roofline = dict(bound=dk["bound"], achieved=dk["achieved"], peak=dk["peak"], unit=dk["unit"],
                     frac=dk["frac"], traffic=traffic, kernel=dom,
                     peak_source=f"{pk['src']} ({'2 x sustained bf16' if dk['bound'] == 'tensor' else 'hbm copy'})")
