@@ -506,8 +506,8 @@ __device__ bool compact_sampled(uint32_t* so, int32_t* ix, int& n_io, int k, int
 // from a 128-entry sample of each stream, weighted by the streams' sizes
 // ng[].  Each stream keeps its entries >= th, in order (its count may fall
 // below k).  Returns false, with nothing written, if th would leave fewer
-// than k or more than max_keep entries in the union.  Streams hold at most
-// 32 * 128 entries each.
+// than k entries in the union or more than max_keep in any one stream.
+// Streams hold at most 32 * 128 entries each.
 template <int G>
 __device__ bool compact_union(uint32_t* so, int32_t* ix, int& n_io, const int (&ng)[G], int k,
                               int max_keep, Scratch<128>& S, Scratch<G * 128>& SA, uint32_t bar,
@@ -584,10 +584,15 @@ __device__ bool compact_union(uint32_t* so, int32_t* ix, int& n_io, const int (&
     const int total = __shfl_sync(0xffffffffu, incl, 31);
     if (tid == 0) SA.red[0][j] = (uint32_t)total;
     named_bar_sync(gbar, NT);
-    int utot = 0;
+    int utot = 0, umax = 0;
 #pragma unroll
-    for (int g = 0; g < G; ++g) utot += (int)SA.red[0][g];
-    if (th == 0 || utot < k || utot > max_keep) return false;  // same answer everywhere
+    for (int g = 0; g < G; ++g) {
+        utot += (int)SA.red[0][g];
+        umax = max(umax, (int)SA.red[0][g]);
+    }
+    // valid when the union keeps at least k; useful when no stream keeps
+    // more than max_keep (each keeps about a G-th of the union)
+    if (th == 0 || utot < k || umax > max_keep) return false;  // same answer everywhere
     const uint32_t below = (1u << lane) - 1u;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
