@@ -46,6 +46,10 @@ __host__ __device__ constexpr int cand_capacity(int k) {
     const int c = 2 * k > k + kBatch * kKeyTile ? 2 * k : k + kBatch * kKeyTile;
     return (c + 127) / 128 * 128;
 }
+// Entries of one chunk slot in the workspace: a chunk hands its union of
+// candidates (at or above a shared threshold, at least k) to the per-sequence
+// merge as it is when it fits, and selects exactly k itself only when not.
+__host__ __device__ constexpr int slot_capacity(int k) { return (k + k / 2 + 127) / 128 * 128; }
 constexpr int kEpiWarps = 16;     // warps 0-15: four warpgroups, one per chunk quarter
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
@@ -383,10 +387,10 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             }
             const int n = a.start[4];
             const int slot = p.seg_base[g.b] + (int)(r0 / p.R - g.base / p.R);
-            uint32_t* oso = p.cand_so + (int64_t)slot * p.k;
-            int32_t* oix = p.cand_ix + (int64_t)slot * p.k;
+            uint32_t* oso = p.cand_so + (int64_t)slot * slot_capacity(p.k);
+            int32_t* oix = p.cand_ix + (int64_t)slot * slot_capacity(p.k);
             int outn;
-            if (n <= p.k) {
+            if (n <= slot_capacity(p.k)) {  // the merge selects the k
                 for (int e = t512; e < n; e += 512) {
                     oso[e] = a.ord(e);
                     oix[e] = a.index(e);
@@ -432,8 +436,9 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
     }
     __syncthreads();
     const int n = total_s;
-    uint32_t* gsc = p.cand_so + (int64_t)s0 * p.k;
-    int32_t* gix = p.cand_ix + (int64_t)s0 * p.k;
+    const int sc = slot_capacity(p.k);
+    uint32_t* gsc = p.cand_so + (int64_t)s0 * sc;
+    int32_t* gix = p.cand_ix + (int64_t)s0 * sc;
     FlatAccess a{gsc, gix};
     if (n <= smem_cap) {
         uint32_t* ssc = reinterpret_cast<uint32_t*>(smem);
@@ -441,8 +446,8 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
         int at = 0;
         for (int s = s0; s < s1; ++s) {
             const int cnt = p.cand_cnt[s];
-            const uint32_t* fs = p.cand_so + (int64_t)s * p.k;
-            const int32_t* fi = p.cand_ix + (int64_t)s * p.k;
+            const uint32_t* fs = p.cand_so + (int64_t)s * sc;
+            const int32_t* fi = p.cand_ix + (int64_t)s * sc;
             for (int e = tid; e < cnt; e += 1024) {
                 ssc[at + e] = fs[e];
                 six[at + e] = fi[e];
@@ -452,31 +457,29 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
         __syncthreads();
         a = FlatAccess{ssc, six};
     } else {
-        // Close the gaps between the slots, leftwards, one slot at a time.
+        // Close the gaps between the slots, leftwards, one slot and one chunk
+        // of 1024 entries at a time (a chunk's writes end at or before the
+        // next chunk's first read, so ascending chunks never overwrite
+        // unread entries).
         int at = 0;
         for (int s = s0; s < s1; ++s) {
             const int cnt = p.cand_cnt[s];
-            const int from = (s - s0) * p.k;
-            uint32_t v[2];
-            int32_t x[2];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int e = tid + r * 1024;
+            const int from = (s - s0) * sc;
+            for (int c0 = 0; c0 < cnt; c0 += 1024) {
+                const int e = c0 + tid;
+                uint32_t v = 0;
+                int32_t x = 0;
                 if (e < cnt) {
-                    v[r] = gsc[from + e];
-                    x[r] = gix[from + e];
+                    v = gsc[from + e];
+                    x = gix[from + e];
                 }
-            }
-            __syncthreads();
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int e = tid + r * 1024;
+                __syncthreads();
                 if (e < cnt) {
-                    gsc[at + e] = v[r];
-                    gix[at + e] = x[r];
+                    gsc[at + e] = v;
+                    gix[at + e] = x;
                 }
+                __syncthreads();
             }
-            __syncthreads();
             at += cnt;
         }
     }

@@ -269,8 +269,9 @@ DecodePlan plan_decode(int B, int64_t total_n, int k, int Hq, int d, int sms) {
     pl.nsplit = ns;
     size_t o = 0;
     pl.off_sb = o;  o = align256(o + (size_t)(B + 1) * 4);
-    pl.off_sc = o;  o = align256(o + (size_t)pl.max_slots * k * 4);
-    pl.off_ix = o;  o = align256(o + (size_t)pl.max_slots * k * 4);
+    const size_t sc = (size_t)dsa::dec::slot_capacity(k);
+    pl.off_sc = o;  o = align256(o + (size_t)pl.max_slots * sc * 4);
+    pl.off_ix = o;  o = align256(o + (size_t)pl.max_slots * sc * 4);
     pl.off_cnt = o; o = align256(o + (size_t)pl.max_slots * 4);
     pl.off_idx = o; o = align256(o + (size_t)B * k * 4);
     pl.off_po = o;  o = align256(o + (size_t)B * ns * Hq * d * 4);
