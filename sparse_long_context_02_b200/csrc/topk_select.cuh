@@ -62,6 +62,7 @@ struct SegAccess {
 // Shared-memory scratch of one collective group.
 template <int NT>
 struct Scratch {
+    static_assert(NT % 32 == 0 && NT <= 1024, "one partial per warp, at most one per lane");
     uint32_t red[2][NT / 32];   // per-warp partials, double-buffered by step parity
     uint32_t red2[2][NT / 32];
     uint32_t red3[2][NT / 32];
@@ -78,9 +79,9 @@ __device__ __forceinline__ uint32_t blk_sum(uint32_t v, Scratch<NT>& S, int& par
     v = __reduce_add_sync(0xffffffffu, v);
     if ((tid & 31) == 0) S.red[parity][tid >> 5] = v;
     named_bar_sync(bar, NT);
-    uint32_t s = 0;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) s += S.red[parity][w];
+    // every warp reduces the NT / 32 partials itself: one load per lane
+    const int lane = tid & 31;
+    const uint32_t s = __reduce_add_sync(0xffffffffu, lane < NT / 32 ? S.red[parity][lane] : 0u);
     parity ^= 1;
     return s;
 }
@@ -96,13 +97,9 @@ __device__ __forceinline__ void blk_minmax(uint32_t& a, uint32_t& b, Scratch<NT>
         S.red2[parity][tid >> 5] = b;
     }
     named_bar_sync(bar, NT);
-    a = S.red[parity][0];
-    b = S.red2[parity][0];
-#pragma unroll
-    for (int w = 1; w < NT / 32; ++w) {
-        a = min(a, S.red[parity][w]);
-        b = max(b, S.red2[parity][w]);
-    }
+    const int lane = tid & 31;
+    a = __reduce_min_sync(0xffffffffu, lane < NT / 32 ? S.red[parity][lane] : 0xffffffffu);
+    b = __reduce_max_sync(0xffffffffu, lane < NT / 32 ? S.red2[parity][lane] : 0u);
     parity ^= 1;
 }
 
@@ -236,13 +233,11 @@ __device__ uint64_t kth_largest(const A& a, int n, int k, uint32_t floor, Scratc
             S.red3[parity][tid >> 5] = c3;
         }
         named_bar_sync(bar, NT);
-        uint32_t t1 = 0, t2 = 0, t3 = 0;
-#pragma unroll
-        for (int w = 0; w < NT / 32; ++w) {
-            t1 += S.red[parity][w];
-            t2 += S.red2[parity][w];
-            t3 += S.red3[parity][w];
-        }
+        const int ln = tid & 31;
+        const bool has = ln < NT / 32;
+        const uint32_t t1 = __reduce_add_sync(0xffffffffu, has ? S.red[parity][ln] : 0u);
+        const uint32_t t2 = __reduce_add_sync(0xffffffffu, has ? S.red2[parity][ln] : 0u);
+        const uint32_t t3 = __reduce_add_sync(0xffffffffu, has ? S.red3[parity][ln] : 0u);
         parity ^= 1;
         const uint32_t K = (uint32_t)k;
         if (t3 >= K) lo = m3;                        // m3 > lo whenever span >= 2
