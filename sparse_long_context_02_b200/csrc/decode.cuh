@@ -63,9 +63,11 @@ struct Params {
     int k;
     int64_t R;                 // cache rows per CTA
     int* seg_base;             // [B + 1]
-    uint32_t* cand_so;         // [slots][k] ordered scores (see topk_select.cuh)
+    uint32_t* cand_so;         // [slots][slot_capacity(k)] ordered scores (topk_select.cuh)
     int32_t* cand_ix;
     int* cand_cnt;             // [slots]
+    uint32_t* cand_th;         // [slots] an ord that at least k of the slot's entries reach
+                               // (0 when the slot holds fewer than k or none is known)
 };
 
 __device__ __forceinline__ bool seq_ok(const Params& p, int b) {
@@ -122,6 +124,7 @@ struct Misc {
     alignas(16) int wcnt[2][4][kBatch][4];  // rows read as int4 by WgTopk::offer
     int cnts[2][4];
     int cnt[4];
+    uint32_t thr[4];
     uint32_t tmem_base;
     volatile int abort_flag;
 };
@@ -374,7 +377,10 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                          ntw - u0 < T ? (ntw - u0 > 0 ? ntw - u0 : 0) : T);
             }
             tk.shrink_union();
-            if (tid == 0) misc->cnt[w] = tk.cnt;
+            if (tid == 0) {
+                misc->cnt[w] = tk.cnt;
+                misc->thr[w] = tk.theta;
+            }
             // ---- merge the four quarter lists into the segment's top-k
             named_bar_sync(5, 512);
             SegAccess a;
@@ -401,7 +407,15 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 const uint64_t kth = sel::kth_largest<512, 16>(a, n, p.k, 0u, *SA, 5, t512);
                 outn = sel::compact<512>(a, n, kth, oso, oix, *SA, 5, t512);
             }
-            if (t512 == 0) p.cand_cnt[slot] = misc->abort_flag ? 0 : outn;
+            if (t512 == 0) {
+                p.cand_cnt[slot] = misc->abort_flag ? 0 : outn;
+                // each quarter's threshold is one that k entries of the union
+                // reach (a shared one, or the quarter's own exact k-th), and
+                // every entry at or above it is in the slot
+                uint32_t th = 0;
+                for (int v = 0; v < 4; ++v) th = max(th, misc->thr[v]);
+                p.cand_th[slot] = outn >= p.k ? th : 0u;
+            }
             named_bar_sync(5, 512);  // the lists are read before the next segment refills them
         }
     }
@@ -422,6 +436,7 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ Scratch<1024> S;
     __shared__ int total_s;
+    __shared__ uint32_t floor_s;
     const int b = blockIdx.x, tid = threadIdx.x;
     const int s0 = p.seg_base[b], s1 = p.seg_base[b + 1];
     int32_t* out = idx_out + (int64_t)b * p.k;
@@ -431,8 +446,13 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
     }
     if (tid == 0) {
         int t = 0;
-        for (int s = s0; s < s1; ++s) t += p.cand_cnt[s];
+        uint32_t f = 0;
+        for (int s = s0; s < s1; ++s) {
+            t += p.cand_cnt[s];
+            f = max(f, p.cand_th[s]);  // k entries of that slot reach it
+        }
         total_s = t;
+        floor_s = f;
     }
     __syncthreads();
     const int n = total_s;
@@ -485,7 +505,7 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
     }
     int cnt = n;
     if (n > p.k) {
-        const uint64_t kth = sel::kth_largest<1024, 24>(a, n, p.k, 0u, S, 0, tid);
+        const uint64_t kth = sel::kth_largest<1024, 24>(a, n, p.k, floor_s, S, 0, tid);
         // Only the selected k entries land in the index row.
         cnt = sel::compact<1024>(a, n, kth, static_cast<uint32_t*>(nullptr), out, S, 0, tid);
     } else {

@@ -249,7 +249,7 @@ constexpr int64_t kMinRange = 4096;  // cache rows per CTA at least
 struct DecodePlan {
     int64_t R;          // cache rows per CTA of the indexer scan
     int ctas, max_slots, nsplit;
-    size_t off_sb, off_sc, off_ix, off_cnt, off_idx, off_po, off_pml, total;
+    size_t off_sb, off_sc, off_ix, off_cnt, off_th, off_idx, off_po, off_pml, total;
 };
 
 DecodePlan plan_decode(int B, int64_t total_n, int k, int Hq, int d, int sms) {
@@ -273,6 +273,7 @@ DecodePlan plan_decode(int B, int64_t total_n, int k, int Hq, int d, int sms) {
     pl.off_sc = o;  o = align256(o + (size_t)pl.max_slots * sc * 4);
     pl.off_ix = o;  o = align256(o + (size_t)pl.max_slots * sc * 4);
     pl.off_cnt = o; o = align256(o + (size_t)pl.max_slots * 4);
+    pl.off_th = o;  o = align256(o + (size_t)pl.max_slots * 4);
     pl.off_idx = o; o = align256(o + (size_t)B * k * 4);
     pl.off_po = o;  o = align256(o + (size_t)B * ns * Hq * d * 4);
     pl.off_pml = o; o = align256(o + (size_t)B * ns * Hq * 2 * 4);
@@ -337,6 +338,7 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     dp.cand_so = reinterpret_cast<uint32_t*>(ws + pl.off_sc);
     dp.cand_ix = reinterpret_cast<int32_t*>(ws + pl.off_ix);
     dp.cand_cnt = reinterpret_cast<int*>(ws + pl.off_cnt);
+    dp.cand_th = reinterpret_cast<uint32_t*>(ws + pl.off_th);
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + pl.off_idx);
 
     CUtensorMap mq, mk;
