@@ -80,6 +80,7 @@ __device__ __forceinline__ bool seq_ok(const Params& p, int b) {
 // output is then all zeros), so no later phase reads outside the caches or
 // the workspace.
 __global__ void __launch_bounds__(1024) prep_kernel(const Params p) {
+    pdl_launch_dependents();
     __shared__ int wsum[32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int carry = 0;
@@ -195,6 +196,8 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     constexpr uint32_t TMEM_COLS = 512;  // 4 warpgroups x 2 accumulators x 64 columns
     constexpr uint32_t IDESC = idesc_e4m3_f32(N);
 
+    pdl_wait();  // the slot bases come from prep_kernel
+    pdl_launch_dependents();
     const int c = blockIdx.x;
     const int64_t r0 = (int64_t)c * p.R;
     const int64_t r1 = r0 + p.R < p.total_n ? r0 + p.R : p.total_n;
@@ -437,6 +440,8 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
     __shared__ Scratch<1024> S;
     __shared__ int total_s;
     __shared__ uint32_t floor_s;
+    pdl_wait();  // the slots come from index_kernel
+    pdl_launch_dependents();
     const int b = blockIdx.x, tid = threadIdx.x;
     const int s0 = p.seg_base[b], s1 = p.seg_base[b + 1];
     int32_t* out = idx_out + (int64_t)b * p.k;

@@ -9,6 +9,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <utility>
+
 #include "dsa.h"
 #include "decode.cuh"
 #include "index_topk.cuh"
@@ -147,13 +149,35 @@ dsa_status_t dispatch_index(const char* fn, const void* q_I, const void* k_I, co
 
 // ------------------------------------------------------------ attention
 
+// Launches `kern` so that it may start while the previous kernel on the
+// stream finishes (it calls pdl_wait() before touching that kernel's output).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <int D, int HKV, int G, bool SPLIT>
 dsa_status_t launch_attn(const char* fn, const dsa::attn::Params& p, int64_t grid,
                          cudaStream_t st) {
     using C = dsa::attn::Cfg<D, HKV>;
     auto kern = dsa::attn::attn_kernel<D, HKV, G, SPLIT>;
     CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
-    kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(p);
+    if (SPLIT) {  // decode: chained behind the merge kernel
+        CUDA_TRY(launch_chained(kern, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM, st, p));
+    } else {
+        kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(p);
+    }
     CUDA_TRY(cudaGetLastError());
     return DSA_OK;
 }
@@ -353,14 +377,16 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     CUDA_TRY(cudaGetLastError());
     CUDA_TRY(cudaFuncSetAttribute(dsa::dec::index_kernel,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem_idx));
-    dsa::dec::index_kernel<<<pl.ctas, dsa::dec::kThreads, smem_idx, st>>>(mq, mk, dp);
+    CUDA_TRY(launch_chained(dsa::dec::index_kernel, dim3(pl.ctas), dim3(dsa::dec::kThreads),
+                            smem_idx, st, mq, mk, dp));
     CUDA_TRY(cudaGetLastError());
 
     const int merge_smem_cap = 24576;  // entries staged in shared memory (192 KB)
     const int smem_merge = merge_smem_cap * 8;
     CUDA_TRY(cudaFuncSetAttribute(dsa::dec::merge_kernel,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem_merge));
-    dsa::dec::merge_kernel<<<B, 1024, smem_merge, st>>>(dp, idx, merge_smem_cap);
+    CUDA_TRY(launch_chained(dsa::dec::merge_kernel, dim3(B), dim3(1024), smem_merge, st, dp, idx,
+                            merge_smem_cap));
     CUDA_TRY(cudaGetLastError());
 
     dsa::attn::Params ap{};
@@ -376,8 +402,9 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     ap.part_ml = reinterpret_cast<float*>(ws + pl.off_pml);
     dsa_status_t r = launch_attn<128, 4, 8, true>(fn, ap, (int64_t)B * pl.nsplit, st);
     if (r != DSA_OK) return r;
-    dsa::attn::combine_kernel<128, 32><<<B * 32, 128, 0, st>>>(ap.part_o, ap.part_ml, pl.nsplit,
-                                                                static_cast<__nv_bfloat16*>(O));
+    CUDA_TRY(launch_chained(dsa::attn::combine_kernel<128, 32>, dim3(B * 32), dim3(128), 0, st,
+                            static_cast<const float*>(ap.part_o), static_cast<const float*>(ap.part_ml),
+                            pl.nsplit, static_cast<__nv_bfloat16*>(O)));
     CUDA_TRY(cudaGetLastError());
     return ok();
 }

@@ -89,6 +89,8 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
 template <int D, int HKV, int G, bool SPLIT>
 __global__ void __launch_bounds__(Cfg<D, HKV>::THREADS)
 attn_kernel(const Params p) {
+    pdl_wait();  // decode: the index rows come from the merge kernel
+    pdl_launch_dependents();
     using C = Cfg<D, HKV>;
     constexpr int HQ = HKV * G;
     static_assert(G <= 8, "at most 8 query heads per KV group");
@@ -308,6 +310,7 @@ attn_kernel(const Params p) {
 template <int D, int HQ>
 __global__ void __launch_bounds__(D) combine_kernel(const float* part_o, const float* part_ml,
                                                     int nsplit, __nv_bfloat16* O) {
+    pdl_wait();  // the partials come from the split attention
     const int64_t b = blockIdx.x / HQ;
     const int h = blockIdx.x % HQ, c = threadIdx.x;
     float M = -INFINITY;
