@@ -9,16 +9,17 @@
 // wave: CTA c covers packed-cache rows [c R, (c+1) R).  A range may hold the
 // tail of one sequence, whole short sequences and the head of another; each
 // such piece is a "segment".
-// Phase 1 (prep): seg_base[b] = number of segments of the sequences before b
-//          (sequence b's segments are the CTAs its rows touch, in order).
-// Phase 2 (index): per segment the CTA loads that sequence's query block,
+// Phase 1 (index): per segment the CTA loads that sequence's query block,
 //          its four epilogue warpgroups each scan a contiguous quarter of the
 //          segment (the MMA thread interleaves their tiles into eight TMEM
-//          accumulators, N = 64 indexer heads of the one query) keeping the
-//          top-k of the quarter, and the CTA merges the four ordered lists
-//          into the segment's top-k, written to slot seg_base[b] + (c - first
-//          CTA of b).
-// Phase 3 (merge): one CTA per sequence selects the top-k of its slots'
+//          accumulators, N = 64 indexer heads of the one query); the quarters
+//          share union thresholds, and the segment's candidates (every key at
+//          or above a threshold that k of them reach) go to slot c + b.
+//          Sequences and chunks are both in row order, so (c, b) pairs of
+//          overlapping chunks and sequences have distinct sums c + b, and the
+//          slots of sequence b are the contiguous range from
+//          cache_off[b] / R + b to (cache_off[b+1] - 1) / R + b.
+// Phase 2 (merge): one CTA per sequence selects the top-k of its slots'
 //          lists (in key order) into the index row.
 // Attention (split over index-row slices) and the split merge live in
 // sparse_attn.cuh.
@@ -62,7 +63,6 @@ struct Params {
     int64_t total_n;           // rows of the packed caches
     int k;
     int64_t R;                 // cache rows per CTA
-    int* seg_base;             // [B + 1]
     uint32_t* cand_so;         // [slots][slot_capacity(k)] ordered scores (topk_select.cuh)
     int32_t* cand_ix;
     int* cand_cnt;             // [slots]
@@ -75,44 +75,6 @@ __device__ __forceinline__ bool seq_ok(const Params& p, int b) {
     return lo >= 0 && hi > lo && hi <= p.total_n;
 }
 
-// seg_base[b] for b in [0, B].  A sequence whose rows are empty or do not lie
-// inside [0, total_n) owns no segment and records DSA_DEVERR_INDEX (its
-// output is then all zeros), so no later phase reads outside the caches or
-// the workspace.
-__global__ void __launch_bounds__(1024) prep_kernel(const Params p) {
-    pdl_launch_dependents();
-    __shared__ int wsum[32];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int carry = 0;
-    for (int b0 = 0; b0 < p.B; b0 += 1024) {
-        const int b = b0 + tid;
-        int c = 0;
-        if (b < p.B) {
-            if (seq_ok(p, b)) {
-                const int64_t lo = p.cache_off[b], hi = p.cache_off[b + 1];
-                c = (int)((hi - 1) / p.R - lo / p.R + 1);
-            } else {
-                record_device_error(2);
-            }
-        }
-        int incl = c;
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (lane == 31) wsum[warp] = incl;
-        __syncthreads();
-        int before = 0, total = 0;
-        for (int wv = 0; wv < 32; ++wv) {
-            before += wv < warp ? wsum[wv] : 0;
-            total += wsum[wv];
-        }
-        if (b < p.B) p.seg_base[b] = carry + before + incl - c;
-        carry += total;
-        __syncthreads();
-    }
-    if (tid == 0) p.seg_base[p.B] = carry;
-}
 
 struct Misc {
     uint64_t full[kStages];
@@ -196,7 +158,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     constexpr uint32_t TMEM_COLS = 512;  // 4 warpgroups x 2 accumulators x 64 columns
     constexpr uint32_t IDESC = idesc_e4m3_f32(N);
 
-    pdl_wait();  // the slot bases come from prep_kernel
+    pdl_wait();  // the caches and queries may come from the previous kernel
     pdl_launch_dependents();
     const int c = blockIdx.x;
     const int64_t r0 = (int64_t)c * p.R;
@@ -395,7 +357,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 a.start[v + 1] = a.start[v] + misc->cnt[v];
             }
             const int n = a.start[4];
-            const int slot = p.seg_base[g.b] + (int)(r0 / p.R - g.base / p.R);
+            const int slot = (int)(r0 / p.R) + g.b;  // distinct over (chunk, sequence) pairs
             uint32_t* oso = p.cand_so + (int64_t)slot * slot_capacity(p.k);
             int32_t* oix = p.cand_ix + (int64_t)slot * slot_capacity(p.k);
             int outn;
@@ -443,8 +405,18 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
     pdl_wait();  // the slots come from index_kernel
     pdl_launch_dependents();
     const int b = blockIdx.x, tid = threadIdx.x;
-    const int s0 = p.seg_base[b], s1 = p.seg_base[b + 1];
     int32_t* out = idx_out + (int64_t)b * p.k;
+    // A sequence whose rows are empty, out of [0, total_n) or not after the
+    // previous sequence's owns no slot: it records DSA_DEVERR_INDEX and its
+    // index row is all -1 (its output all zeros).
+    const bool ordered = b == 0 || p.cache_off[b] >= p.cache_off[b - 1];
+    int s0 = 0, s1 = 0;
+    if (seq_ok(p, b) && ordered) {
+        s0 = (int)(p.cache_off[b] / p.R) + b;
+        s1 = (int)((p.cache_off[b + 1] - 1) / p.R) + b + 1;
+    } else if (tid == 0) {
+        record_device_error(2);
+    }
     if (s1 <= s0) {
         for (int e = tid; e < p.k; e += 1024) out[e] = -1;
         return;

@@ -273,7 +273,7 @@ constexpr int64_t kMinRange = 4096;  // cache rows per CTA at least
 struct DecodePlan {
     int64_t R;          // cache rows per CTA of the indexer scan
     int ctas, max_slots, nsplit;
-    size_t off_sb, off_sc, off_ix, off_cnt, off_th, off_idx, off_po, off_pml, total;
+    size_t off_sc, off_ix, off_cnt, off_th, off_idx, off_po, off_pml, total;
 };
 
 DecodePlan plan_decode(int B, int64_t total_n, int k, int Hq, int d, int sms) {
@@ -284,7 +284,7 @@ DecodePlan plan_decode(int B, int64_t total_n, int k, int Hq, int d, int sms) {
     if (ctas < 1) ctas = 1;
     pl.R = (total_n + ctas - 1) / ctas;
     pl.ctas = (int)((total_n + pl.R - 1) / pl.R);
-    pl.max_slots = pl.ctas + B;  // each range boundary splits at most one sequence
+    pl.max_slots = pl.ctas + B;  // slot = chunk + sequence of an overlapping pair
     // split the index rows so that B * nsplit attention CTAs fill one wave
     // (two resident CTAs per SM)
     int ns = (2 * sms) / B;
@@ -292,7 +292,6 @@ DecodePlan plan_decode(int B, int64_t total_n, int k, int Hq, int d, int sms) {
     if (ns > 16) ns = 16;
     pl.nsplit = ns;
     size_t o = 0;
-    pl.off_sb = o;  o = align256(o + (size_t)(B + 1) * 4);
     const size_t sc = (size_t)dsa::dec::slot_capacity(k);
     pl.off_sc = o;  o = align256(o + (size_t)pl.max_slots * sc * 4);
     pl.off_ix = o;  o = align256(o + (size_t)pl.max_slots * sc * 4);
@@ -358,7 +357,6 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     dp.total_n = total_n;
     dp.k = k;
     dp.R = pl.R;
-    dp.seg_base = reinterpret_cast<int*>(ws + pl.off_sb);
     dp.cand_so = reinterpret_cast<uint32_t*>(ws + pl.off_sc);
     dp.cand_ix = reinterpret_cast<int32_t*>(ws + pl.off_ix);
     dp.cand_cnt = reinterpret_cast<int*>(ws + pl.off_cnt);
@@ -373,8 +371,6 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     if (smem_idx > max_optin_smem())
         return fail(DSA_ERR_UNSUPPORTED, "%s: needs %d bytes of shared memory", fn, smem_idx);
 
-    dsa::dec::prep_kernel<<<1, 1024, 0, st>>>(dp);
-    CUDA_TRY(cudaGetLastError());
     CUDA_TRY(cudaFuncSetAttribute(dsa::dec::index_kernel,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem_idx));
     CUDA_TRY(launch_chained(dsa::dec::index_kernel, dim3(pl.ctas), dim3(dsa::dec::kThreads),
