@@ -295,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
                                D["V_cache"], D["cache_off"], dcfg.k, dcfg.scale, O=D["O"],
                                idx_out=D["idx"], workspace=D["ws"], stream=stream)
 
-    launches_per_step = (2 if pcfg else 0) + (5 if dcfg else 0)
+    launches_per_step = (2 if pcfg else 0) + (4 if dcfg else 0)  # decode: index, merge, attention, combine
 
     def step(ev=None):
         if ev is not None:
