@@ -95,6 +95,26 @@ DSA_API dsa_status_t dsa_index_topk(const void* q_I, const void* k_I, const floa
                             int H_I, int d_I, int k, int32_t* idx, dsa_stream_t stream);
 
 /*
+ * dsa_index_topk_varlen - dsa_index_topk over a packed batch of sequences
+ * (the pages' varlen mode and sequence packing, Kwai Keye-VL-2.0 technical
+ * report summary, sections 1 and 8).  Row t of sequence b, with
+ * cu_seqlens[b] <= t < cu_seqlens[b+1], sees only the keys
+ * s in [cu_seqlens[b], t]: the causal mask restarts at every sequence.
+ *
+ *   cu_seqlens [nseq+1] int32  device; 0 = cu_seqlens[0] <= ... <=
+ *                              cu_seqlens[nseq] = L (caller's contract; a
+ *                              first or last entry other than 0 and L
+ *                              records DSA_DEVERR_INDEX)
+ *   q_I, k_I, w, idx           as dsa_index_topk over the packed rows; idx
+ *                              holds packed (global) key positions, so
+ *                              dsa_sparse_attn_prefill runs on it unchanged
+ * Same shape support as dsa_index_topk.
+ */
+DSA_API dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, const float* w,
+                                   const int32_t* cu_seqlens, int nseq, int64_t L, int H_I,
+                                   int d_I, int k, int32_t* idx, dsa_stream_t stream);
+
+/*
  * dsa_index_scores - the same indexer, writing the dense causal score
  * matrix instead of selecting (for small L: checks and training losses that
  * need the whole score distribution).

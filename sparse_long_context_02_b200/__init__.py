@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_index_topk.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp]
         L.dsa_index_scores.restype = i32
         L.dsa_index_scores.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
+        L.dsa_index_topk_varlen.restype = i32
+        L.dsa_index_topk_varlen.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, vp]
         L.dsa_sparse_attn_prefill.restype = i32
         L.dsa_sparse_attn_prefill.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, f32, vp,
                                               vp]
@@ -105,6 +107,25 @@ def index_topk(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, k: int,
         idx = torch.empty((L, k), dtype=torch.int32, device=q_I.device)
     _check(lib().dsa_index_topk(_dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), L, H, d,
                                 k, _dev(idx, "idx", 4), _stream(stream)), "dsa_index_topk")
+    return idx
+
+
+def index_topk_varlen(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor,
+                      cu_seqlens: torch.Tensor, k: int, idx: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """Indexer + top-k over a packed batch: cu_seqlens [nseq + 1] int32 on the
+    device (0 ... L); row t of a sequence sees only that sequence's keys up to
+    t.  idx holds packed key positions (ascending, -1 pad)."""
+    L, H, d = q_I.shape
+    if idx is None:
+        idx = torch.empty((L, k), dtype=torch.int32, device=q_I.device)
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+        raise DSAError("dsa_index_topk_varlen: cu_seqlens must be an int32 device tensor")
+    nseq = cu_seqlens.numel() - 1
+    _check(lib().dsa_index_topk_varlen(_dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4),
+                                       _dev(cu_seqlens, "cu_seqlens", 4), nseq, L, H, d, k,
+                                       _dev(idx, "idx", 4), _stream(stream)),
+           "dsa_index_topk_varlen")
     return idx
 
 

@@ -101,7 +101,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 template <int HI, int DI, bool TOPK>
 dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
-                          int64_t L, int k, int32_t* idx, float* scores, cudaStream_t st) {
+                          int64_t L, int k, int32_t* idx, float* scores, const int32_t* cu_seqlens,
+                          int nseq, cudaStream_t st) {
     CUtensorMap mq, mk;
     if (!make_map(&mq, q_I, DI, (uint64_t)L * HI, dsa::idx::kTokens * HI) ||
         !make_map(&mk, k_I, DI, (uint64_t)L, dsa::idx::kKeyTile))
@@ -126,6 +127,8 @@ dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, cons
     p.idx = idx;
     p.scores = scores;
     p.nblocks = (int)((L + dsa::idx::kTokens - 1) / dsa::idx::kTokens);
+    p.cu_seqlens = cu_seqlens;
+    p.nseq = nseq;
     kern<<<p.nblocks, dsa::idx::kThreads, smem, st>>>(mq, mk, p);
     CUDA_TRY(cudaGetLastError());
     return ok();
@@ -134,15 +137,15 @@ dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, cons
 template <bool TOPK>
 dsa_status_t dispatch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
                             int64_t L, int H_I, int d_I, int k, int32_t* idx, float* scores,
-                            cudaStream_t st) {
+                            const int32_t* cu, int nseq, cudaStream_t st) {
     if (H_I == 64 && d_I == 128)
-        return launch_index<64, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, st);
+        return launch_index<64, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, st);
     if (H_I == 64 && d_I == 64)
-        return launch_index<64, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, st);
+        return launch_index<64, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, st);
     if (H_I == 4 && d_I == 128)
-        return launch_index<4, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, st);
+        return launch_index<4, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, st);
     if (H_I == 4 && d_I == 64)
-        return launch_index<4, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, st);
+        return launch_index<4, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, st);
     return fail(DSA_ERR_UNSUPPORTED, "%s: (H_I, d_I) = (%d, %d) not in {4, 64} x {64, 128}", fn,
                 H_I, d_I);
 }
@@ -214,7 +217,26 @@ dsa_status_t dsa_index_topk(const void* q_I, const void* k_I, const float* w, in
     if (k > 2048) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > 2048", fn, k);
     if (L * H_I >= (int64_t(1) << 31))
         return fail(DSA_ERR_UNSUPPORTED, "%s: L * H_I too large", fn);
-    return dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr,
+    return dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, nullptr, 1,
+                                static_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, const float* w,
+                                   const int32_t* cu_seqlens, int nseq, int64_t L, int H_I,
+                                   int d_I, int k, int32_t* idx, dsa_stream_t stream) {
+    static const char fn[] = "dsa_index_topk_varlen";
+    CHECK_PTR(q_I);
+    CHECK_PTR(k_I);
+    CHECK_PTR(w);
+    CHECK_PTR(idx);
+    if (cu_seqlens == nullptr) return fail(DSA_ERR_INVALID_ARG, "%s: cu_seqlens is null", fn);
+    if (nseq < 1) return fail(DSA_ERR_INVALID_ARG, "%s: nseq = %d", fn, nseq);
+    if (L < 1 || L > (int64_t(1) << 30)) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (k > 2048) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > 2048", fn, k);
+    if (L * H_I >= (int64_t(1) << 31))
+        return fail(DSA_ERR_UNSUPPORTED, "%s: L * H_I too large", fn);
+    return dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, cu_seqlens, nseq,
                                 static_cast<cudaStream_t>(stream));
 }
 
@@ -227,7 +249,7 @@ dsa_status_t dsa_index_scores(const void* q_I, const void* k_I, const float* w, 
     CHECK_PTR(scores);
     if (L < 1 || L * L >= (int64_t(1) << 31))
         return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld (L * L must be < 2^31)", fn, (long long)L);
-    return dispatch_index<false>(fn, q_I, k_I, w, L, H_I, d_I, 1, nullptr, scores,
+    return dispatch_index<false>(fn, q_I, k_I, w, L, H_I, d_I, 1, nullptr, scores, nullptr, 1,
                                  static_cast<cudaStream_t>(stream));
 }
 

@@ -174,7 +174,26 @@ struct Params {
     int32_t* idx;        // [L][k]        (top-k mode)
     float* scores;       // [L][L]        (dense-score mode)
     int nblocks;
+    // Packed variable-length batch (top-k mode): query t sees keys
+    // [cu_seqlens[b], t] of its own sequence b.  Null: one sequence.
+    const int32_t* cu_seqlens;  // [nseq + 1], 0 ... L, non-decreasing
+    int nseq;
 };
+
+// Start of the sequence that holds row t: cu[b] for the last b with
+// cu[b] <= t, clamped into [0, t] (so a malformed array never reaches
+// outside the rows).
+__device__ __forceinline__ int64_t seq_start(const int32_t* cu, int nseq, int64_t t) {
+    if (cu == nullptr) return 0;
+    int lo = 0, hi = nseq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)cu[mid] <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    int64_t s = cu[lo];
+    return s < 0 ? 0 : (s > t ? t : s);
+}
 
 template <int HI, int DI, bool TOPK>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -204,7 +223,15 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     const int blk = p.nblocks - 1 - (int)blockIdx.x;  // longest rows first
     const int64_t t0 = (int64_t)blk * kTokens;
     const int64_t tmax = (t0 + kTokens - 1 < L ? t0 + kTokens - 1 : L - 1);
-    const int ntiles = TOPK ? (int)(tmax / kKeyTile) + 1 : (int)((L + kKeyTile - 1) / kKeyTile);
+    // token t0 + j sees keys [seq_start(t0 + j), t0 + j]; the CTA's tiles run
+    // from the tile of the lowest start (the first token's: starts grow with t)
+    const int64_t lo_min = TOPK ? seq_start(p.cu_seqlens, p.nseq, t0) : 0;
+    const int tile0 = TOPK ? (int)(lo_min / kKeyTile) : 0;  // first key tile of the CTA
+    const int ntiles = TOPK ? (int)(tmax / kKeyTile) + 1 - tile0
+                            : (int)((L + kKeyTile - 1) / kKeyTile);  // tiles tile0, tile0 + 1, ...
+    if (TOPK && p.cu_seqlens != nullptr && blockIdx.x == 0 && threadIdx.x == 0 &&
+        (p.cu_seqlens[0] != 0 || (int64_t)p.cu_seqlens[p.nseq] != L))
+        record_device_error(2);  // cu_seqlens must run from 0 to L
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -254,7 +281,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 const uint32_t fb = smem_u32(&misc->full[s]);
                 mbar_arrive_expect_tx(fb, KT_BYTES);
                 tma_load_2d(smem_u32(smem + lay.stage + s * KT_BYTES), &tmap_k, fb, 0,
-                            i * kKeyTile);
+                            (tile0 + i) * kKeyTile);
                 issued = i + 1;
             }
             // Never leave with a copy in flight.
@@ -299,6 +326,11 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         const uint32_t bar = 1 + j;
         const int64_t t = t0 + j;
         const bool trow = t < L;
+        // key s of tile i is kb + 128 i; it is visible iff s - lo_t < vis_n
+        // (unsigned), i.e. lo_t <= s <= t, with L <= 2^30 in 32 bits
+        const int lo_t = TOPK && trow ? (int)seq_start(p.cu_seqlens, p.nseq, t) : 0;
+        const uint32_t vis_n = trow ? (uint32_t)(t - lo_t + 1) : 0u;
+        const int kb = tile0 * kKeyTile + q * 32 + lane;
         uint32_t* so = reinterpret_cast<uint32_t*>(smem + lay.cs) + j * cap;
         int32_t* ix = reinterpret_cast<int32_t*>(smem + lay.ci) + j * cap;
         Scratch<128>* S = reinterpret_cast<Scratch<128>*>(smem + lay.scratch) + j;
@@ -339,15 +371,15 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&misc->accempty[buf]));
-                const int64_t s = (int64_t)i * kKeyTile + q * 32 + lane;
                 if constexpr (TOPK) {
-                    if (trow && s <= t) o[u] = sel::ord_f32(score);
+                    if ((uint32_t)(kb + i * kKeyTile - lo_t) < vis_n) o[u] = sel::ord_f32(score);
                 } else {
+                    const int64_t s = (int64_t)i * kKeyTile + q * 32 + lane;
                     if (trow && s < L) p.scores[t * L + s] = s <= t ? score : -INFINITY;
                 }
             }
             if constexpr (TOPK)
-                tk.offer(o, (int32_t)(i0 * kKeyTile + q * 32 + lane),
+                tk.offer(o, kb + i0 * kKeyTile,
                          ntiles - i0 < kBatch ? ntiles - i0 : kBatch);
         }
 
