@@ -53,6 +53,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--union-stats", type=int, default=0, metavar="G",
+                    help="instead of timing: run the prefill indexer once and report how many "
+                         "distinct keys the index rows of G consecutive queries select together "
+                         "(the traffic an adjacent-query dedup would read)")
     return ap.parse_args()
 
 
@@ -507,6 +511,33 @@ def run_reference(args):
                          d2h_bytes_per_step=0))
 
 
+def union_stats(args) -> dict:
+    """Distinct keys selected by blocks of G consecutive query rows, over the
+    rows whose index sets are full (t + 1 >= k): the rows an adjacent-query
+    dedup would gather once per block instead of once per row."""
+    import torch
+    import sparse_long_context_02_b200 as dsa
+    G = args.union_stats
+    cfg = gen.CONFIGS[args.prefill_config]
+    host = gen.prefill_inputs(cfg)
+    idx = dsa.index_topk(torch.from_numpy(host["q_I"]).cuda(), torch.from_numpy(host["k_I"]).cuda(),
+                         torch.from_numpy(host["w"]).cuda(), cfg.k)
+    t0 = (cfg.k + G - 1) // G * G  # first block of full rows
+    nb = (cfg.L - t0) // G
+    fr = []
+    for b0 in range(0, nb, 1024):  # blocks in batches (sorting needs memory)
+        b1 = min(nb, b0 + 1024)
+        x = idx[t0 + b0 * G:t0 + b1 * G].reshape(b1 - b0, G * cfg.k)
+        x, _ = torch.sort(x, dim=1)
+        distinct = 1 + (x[:, 1:] != x[:, :-1]).sum(dim=1)
+        fr.append(distinct.float() / (G * cfg.k))
+    fr = torch.cat(fr).cpu().numpy()
+    return dict(metric="distinct selected keys per block of %d queries / (%d k)" % (G, G),
+                workload=cfg.name, blocks=int(nb), mean=float(fr.mean()),
+                p10=float(np.percentile(fr, 10)), p50=float(np.percentile(fr, 50)),
+                p90=float(np.percentile(fr, 90)), k=cfg.k, data="synthetic")
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -516,6 +547,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.union_stats:
+        if rank == 0:
+            print(json.dumps(union_stats(args)), flush=True)
         return
 
     import datetime
