@@ -103,8 +103,8 @@ def decode_bytes(cfg, lens) -> float:
 # stay in L2), so it grows with L.  Valid only for the CUDA sources the
 # counters were taken on (their SHA-256 below); otherwise null.
 TRAFFIC = {
-    "dsa_index_topk": dict(bytes_per_query_token=510171392 / 32768,
-                           src_sha256="769e3ff4e88fa327a5869516cac6d167a837a4fd10ed054d7e3a1249e9eef442"),
+    "dsa_index_topk": dict(bytes_per_query_token=510516224 / 32768,
+                           src_sha256="eb5cd06497475cb58d5203cda13d3b22bdb13b3991eb096de27b5d9ade8307fd"),
 }
 
 
