@@ -115,6 +115,34 @@ DSA_API dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, con
                                    int d_I, int k, int32_t* idx, dsa_stream_t stream);
 
 /*
+ * dsa_prefill_from_host - the whole prefill (A1 + A2 + A3) for inputs that
+ * sit in host memory.  The rows are handled in chunks of chunk_rows (rounded
+ * up to a multiple of 128): each chunk's rows of q_I, k_I, w, Q, K and V are
+ * copied into the caller's device buffers on h2d_stream; as soon as they are
+ * there (with every earlier key), the chunk's index rows and attention run on
+ * `stream`; its output rows go back to O_host on d2h_stream.  Copies of
+ * later chunks thus overlap the kernels of earlier ones.  Asynchronous: when
+ * `stream` reaches the end of this call's work, O_host holds the result and
+ * idx the index rows.  The copy streams first wait for the work already
+ * queued on `stream` (which may still use the device buffers).  Host buffers
+ * must be page-locked for the copies to be asynchronous; the three streams
+ * must be distinct.
+ *
+ *   *_host              host pointers, layouts as the device buffers below
+ *   q_I, k_I, w, Q, K, V, idx, O
+ *                       caller-owned device buffers, layouts as in
+ *                       dsa_index_topk and dsa_sparse_attn_prefill
+ * Same shape support as dsa_index_topk and dsa_sparse_attn_prefill.
+ */
+DSA_API dsa_status_t dsa_prefill_from_host(const void* q_I_host, const void* k_I_host,
+                                   const float* w_host, const void* Q_host, const void* K_host,
+                                   const void* V_host, void* O_host, void* q_I, void* k_I,
+                                   float* w, void* Q, void* K, void* V, int32_t* idx, void* O,
+                                   int64_t L, int H_I, int d_I, int Hq, int Hkv, int d, int k,
+                                   float scale, int64_t chunk_rows, dsa_stream_t stream,
+                                   dsa_stream_t h2d_stream, dsa_stream_t d2h_stream);
+
+/*
  * dsa_index_scores - the same indexer, writing the dense causal score
  * matrix instead of selecting (for small L: checks and training losses that
  * need the whole score distribution).

@@ -50,6 +50,9 @@ def lib() -> ctypes.CDLL:
         L.dsa_index_topk.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp]
         L.dsa_index_scores.restype = i32
         L.dsa_index_scores.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
+        L.dsa_prefill_from_host.restype = i32
+        L.dsa_prefill_from_host.argtypes = [vp] * 15 + [i64, i32, i32, i32, i32, i32, i32,
+                                                          ctypes.c_float, i64, vp, vp, vp]
         L.dsa_index_topk_varlen.restype = i32
         L.dsa_index_topk_varlen.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, vp]
         L.dsa_sparse_attn_prefill.restype = i32
@@ -156,6 +159,31 @@ def sparse_attn_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, idx: 
                                          _dev(O, "O", 2), _stream(stream)),
            "dsa_sparse_attn_prefill")
     return O
+
+
+def _host(t: torch.Tensor, name: str) -> int:
+    if t.is_cuda or not t.is_contiguous():
+        raise DSAError(f"{name} must be a contiguous host tensor")
+    return t.data_ptr()
+
+
+def prefill_from_host(host: dict, dev: dict, k: int, scale: float, chunk_rows: int = 8192,
+                      stream=None, h2d_stream=None, d2h_stream=None) -> None:
+    """Whole prefill from host inputs with copies and kernels overlapped in
+    row chunks.  host: q_I, k_I, w, Q, K, V (inputs) and O (output), pinned
+    CPU tensors; dev: device buffers of the same names plus idx [L][k].
+    Asynchronous on `stream` (host["O"] is filled when it completes)."""
+    L, H, d_I = host["q_I"].shape
+    Hq, d = host["Q"].shape[1], host["Q"].shape[2]
+    Hkv = host["K"].shape[1]
+    if h2d_stream is None or d2h_stream is None:
+        raise DSAError("dsa_prefill_from_host: pass h2d_stream and d2h_stream")
+    names = ("q_I", "k_I", "w", "Q", "K", "V")
+    args = [_host(host[n], n) for n in names] + [_host(host["O"], "O")]
+    args += [_dev(dev[n], n) for n in names] + [_dev(dev["idx"], "idx", 4), _dev(dev["O"], "O")]
+    _check(lib().dsa_prefill_from_host(*args, L, H, d_I, Hq, Hkv, d, k, float(scale), chunk_rows,
+                                       _stream(stream), _stream(h2d_stream), _stream(d2h_stream)),
+           "dsa_prefill_from_host")
 
 
 def decode_workspace_size(B: int, total_n: int, H_I: int, d_I: int, k: int, Hq: int, Hkv: int,

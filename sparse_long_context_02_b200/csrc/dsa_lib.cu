@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include <utility>
+#include <vector>
 
 #include "dsa.h"
 #include "decode.cuh"
@@ -102,7 +103,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 template <int HI, int DI, bool TOPK>
 dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
                           int64_t L, int k, int32_t* idx, float* scores, const int32_t* cu_seqlens,
-                          int nseq, cudaStream_t st) {
+                          int nseq, int64_t row0, int64_t row1, cudaStream_t st) {
     CUtensorMap mq, mk;
     if (!make_map(&mq, q_I, DI, (uint64_t)L * HI, dsa::idx::kTokens * HI) ||
         !make_map(&mk, k_I, DI, (uint64_t)L, dsa::idx::kKeyTile))
@@ -126,7 +127,9 @@ dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, cons
     p.k = k;
     p.idx = idx;
     p.scores = scores;
-    p.nblocks = (int)((L + dsa::idx::kTokens - 1) / dsa::idx::kTokens);
+    // rows [row0, row1), row0 a multiple of kTokens
+    p.blk0 = (int)(row0 / dsa::idx::kTokens);
+    p.nblocks = (int)((row1 + dsa::idx::kTokens - 1) / dsa::idx::kTokens) - p.blk0;
     p.cu_seqlens = cu_seqlens;
     p.nseq = nseq;
     kern<<<p.nblocks, dsa::idx::kThreads, smem, st>>>(mq, mk, p);
@@ -137,15 +140,17 @@ dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, cons
 template <bool TOPK>
 dsa_status_t dispatch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
                             int64_t L, int H_I, int d_I, int k, int32_t* idx, float* scores,
-                            const int32_t* cu, int nseq, cudaStream_t st) {
+                            const int32_t* cu, int nseq, cudaStream_t st, int64_t row0 = 0,
+                            int64_t row1 = -1) {
+    if (row1 < 0) row1 = L;
     if (H_I == 64 && d_I == 128)
-        return launch_index<64, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, st);
+        return launch_index<64, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, st);
     if (H_I == 64 && d_I == 64)
-        return launch_index<64, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, st);
+        return launch_index<64, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, st);
     if (H_I == 4 && d_I == 128)
-        return launch_index<4, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, st);
+        return launch_index<4, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, st);
     if (H_I == 4 && d_I == 64)
-        return launch_index<4, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, st);
+        return launch_index<4, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, st);
     return fail(DSA_ERR_UNSUPPORTED, "%s: (H_I, d_I) = (%d, %d) not in {4, 64} x {64, 128}", fn,
                 H_I, d_I);
 }
@@ -183,6 +188,30 @@ dsa_status_t launch_attn(const char* fn, const dsa::attn::Params& p, int64_t gri
     }
     CUDA_TRY(cudaGetLastError());
     return DSA_OK;
+}
+
+// Attention for query rows [row0, row1) over keys [0, L) (arguments
+// checked by the caller).
+dsa_status_t attn_prefill_rows(const char* fn, const void* Q, const void* K, const void* V,
+                               const int32_t* idx, int64_t L, int Hq, int Hkv, int d, int k,
+                               float scale, void* O, int64_t row0, int64_t row1,
+                               cudaStream_t st) {
+    const int G = Hq / Hkv;
+    dsa::attn::Params p{};
+    p.Q = static_cast<const __nv_bfloat16*>(Q) + row0 * Hq * d;
+    p.K = static_cast<const __nv_bfloat16*>(K);
+    p.V = static_cast<const __nv_bfloat16*>(V);
+    p.idx = idx + row0 * k;
+    p.nkeys = L;
+    p.k = k;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.O = static_cast<__nv_bfloat16*>(O) + row0 * Hq * d;
+    const int64_t rows = row1 - row0;
+    if (d == 128 && Hkv == 4 && G == 8) return launch_attn<128, 4, 8, false>(fn, p, rows, st);
+    if (d == 64 && Hkv == 2 && G == 4) return launch_attn<64, 2, 4, false>(fn, p, rows, st);
+    if (d == 128 && Hkv == 2 && G == 4) return launch_attn<128, 2, 4, false>(fn, p, rows, st);
+    if (d == 64 && Hkv == 4 && G == 8) return launch_attn<64, 4, 8, false>(fn, p, rows, st);
+    return fail(DSA_ERR_UNSUPPORTED, "%s: (d, Hkv, Hq/Hkv) = (%d, %d, %d)", fn, d, Hkv, G);
 }
 
 }  // namespace
@@ -240,6 +269,87 @@ dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, const float
                                 static_cast<cudaStream_t>(stream));
 }
 
+dsa_status_t dsa_prefill_from_host(const void* q_I_h, const void* k_I_h, const float* w_h,
+                                   const void* Q_h, const void* K_h, const void* V_h, void* O_h,
+                                   void* q_I, void* k_I, float* w, void* Q, void* K, void* V,
+                                   int32_t* idx, void* O, int64_t L, int H_I, int d_I, int Hq,
+                                   int Hkv, int d, int k, float scale, int64_t chunk_rows,
+                                   dsa_stream_t stream, dsa_stream_t h2d_stream,
+                                   dsa_stream_t d2h_stream) {
+    static const char fn[] = "dsa_prefill_from_host";
+    CHECK_PTR(q_I_h);
+    CHECK_PTR(k_I_h);
+    CHECK_PTR(w_h);
+    CHECK_PTR(Q_h);
+    CHECK_PTR(K_h);
+    CHECK_PTR(V_h);
+    CHECK_PTR(O_h);
+    CHECK_PTR(q_I);
+    CHECK_PTR(k_I);
+    CHECK_PTR(w);
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(idx);
+    CHECK_PTR(O);
+    if (L < 1 || L > (int64_t(1) << 30)) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (k > 2048) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > 2048", fn, k);
+    if (L * H_I >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED, "%s: L * H_I too large", fn);
+    if (Hkv < 1 || Hq < 1 || Hq % Hkv) return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d", fn, Hq, Hkv);
+    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
+    if (chunk_rows < 1) return fail(DSA_ERR_INVALID_ARG, "%s: chunk_rows = %lld", fn, (long long)chunk_rows);
+    const int64_t C = (chunk_rows + 127) / 128 * 128;  // whole 4-row blocks and key tiles
+    const int nch = (int)((L + C - 1) / C);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaStream_t sh = static_cast<cudaStream_t>(h2d_stream);
+    cudaStream_t sd = static_cast<cudaStream_t>(d2h_stream);
+    // per chunk: inputs on the device, outputs ready; then all copies back
+    std::vector<cudaEvent_t> ev(2 * nch + 2, nullptr);
+    for (auto& e : ev) CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    struct Destroy {
+        std::vector<cudaEvent_t>& v;
+        ~Destroy() {
+            for (auto e : v)
+                if (e) cudaEventDestroy(e);  // released once pending work reaches them
+        }
+    } destroy{ev};
+    auto hb = [](const void* p) { return static_cast<const uint8_t*>(p); };
+    auto db = [](void* p) { return static_cast<uint8_t*>(p); };
+    // the device buffers may still be in use by earlier work on `stream`:
+    // neither copy stream starts before it
+    CUDA_TRY(cudaEventRecord(ev[2 * nch + 1], st));
+    CUDA_TRY(cudaStreamWaitEvent(sh, ev[2 * nch + 1], 0));
+    CUDA_TRY(cudaStreamWaitEvent(sd, ev[2 * nch + 1], 0));
+    const int64_t rq = (int64_t)H_I * d_I, rk = d_I, rw = (int64_t)H_I * 4,
+                  rQ = (int64_t)Hq * d * 2, rK = (int64_t)Hkv * d * 2;
+    for (int c = 0; c < nch; ++c) {
+        const int64_t r0 = c * C, r1 = r0 + C < L ? r0 + C : L, n = r1 - r0;
+        // the chunk's new rows: queries, weights, and the keys/values they add
+        CUDA_TRY(cudaMemcpyAsync(db(q_I) + r0 * rq, hb(q_I_h) + r0 * rq, n * rq, cudaMemcpyHostToDevice, sh));
+        CUDA_TRY(cudaMemcpyAsync(db(k_I) + r0 * rk, hb(k_I_h) + r0 * rk, n * rk, cudaMemcpyHostToDevice, sh));
+        CUDA_TRY(cudaMemcpyAsync(db(w) + r0 * rw, hb(w_h) + r0 * rw, n * rw, cudaMemcpyHostToDevice, sh));
+        CUDA_TRY(cudaMemcpyAsync(db(Q) + r0 * rQ, hb(Q_h) + r0 * rQ, n * rQ, cudaMemcpyHostToDevice, sh));
+        CUDA_TRY(cudaMemcpyAsync(db(K) + r0 * rK, hb(K_h) + r0 * rK, n * rK, cudaMemcpyHostToDevice, sh));
+        CUDA_TRY(cudaMemcpyAsync(db(V) + r0 * rK, hb(V_h) + r0 * rK, n * rK, cudaMemcpyHostToDevice, sh));
+        CUDA_TRY(cudaEventRecord(ev[2 * c], sh));
+        // rows [r0, r1) need keys [0, r1): all of them are on the device now
+        CUDA_TRY(cudaStreamWaitEvent(st, ev[2 * c], 0));
+        dsa_status_t r = dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, nullptr,
+                                              1, st, r0, r1);
+        if (r != DSA_OK) return r;
+        r = attn_prefill_rows(fn, Q, K, V, idx, L, Hq, Hkv, d, k, scale, O, r0, r1, st);
+        if (r != DSA_OK) return r;
+        CUDA_TRY(cudaEventRecord(ev[2 * c + 1], st));
+        CUDA_TRY(cudaStreamWaitEvent(sd, ev[2 * c + 1], 0));
+        CUDA_TRY(cudaMemcpyAsync(db(O_h) + r0 * rQ, static_cast<const uint8_t*>(O) + r0 * rQ, n * rQ,
+                                 cudaMemcpyDeviceToHost, sd));
+    }
+    CUDA_TRY(cudaEventRecord(ev[2 * nch], sd));
+    CUDA_TRY(cudaStreamWaitEvent(st, ev[2 * nch], 0));  // `stream` ends when O_h is filled
+    return ok();
+}
+
 dsa_status_t dsa_index_scores(const void* q_I, const void* k_I, const float* w, int64_t L,
                               int H_I, int d_I, float* scores, dsa_stream_t stream) {
     static const char fn[] = "dsa_index_scores";
@@ -266,24 +376,8 @@ dsa_status_t dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V
     if (k < 1 || k > 65536) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
     if (Hkv < 1 || Hq < 1 || Hq % Hkv) return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d", fn, Hq, Hkv);
     if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
-    const int G = Hq / Hkv;
-    dsa::attn::Params p{};
-    p.Q = static_cast<const __nv_bfloat16*>(Q);
-    p.K = static_cast<const __nv_bfloat16*>(K);
-    p.V = static_cast<const __nv_bfloat16*>(V);
-    p.idx = idx;
-    p.nkeys = L;
-    p.k = k;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.O = static_cast<__nv_bfloat16*>(O);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    dsa_status_t r;
-    if (d == 128 && Hkv == 4 && G == 8) r = launch_attn<128, 4, 8, false>(fn, p, L, st);
-    else if (d == 64 && Hkv == 2 && G == 4) r = launch_attn<64, 2, 4, false>(fn, p, L, st);
-    else if (d == 128 && Hkv == 2 && G == 4) r = launch_attn<128, 2, 4, false>(fn, p, L, st);
-    else if (d == 64 && Hkv == 4 && G == 8) r = launch_attn<64, 4, 8, false>(fn, p, L, st);
-    else
-        return fail(DSA_ERR_UNSUPPORTED, "%s: (d, Hkv, Hq/Hkv) = (%d, %d, %d)", fn, d, Hkv, G);
+    const dsa_status_t r = attn_prefill_rows(fn, Q, K, V, idx, L, Hq, Hkv, d, k, scale, O, 0, L,
+                                             static_cast<cudaStream_t>(stream));
     return r == DSA_OK ? ok() : r;
 }
 

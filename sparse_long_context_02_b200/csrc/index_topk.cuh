@@ -173,7 +173,8 @@ struct Params {
     int k;
     int32_t* idx;        // [L][k]        (top-k mode)
     float* scores;       // [L][L]        (dense-score mode)
-    int nblocks;
+    int nblocks;         // blocks of kTokens rows launched
+    int blk0;            // first block: rows [4 blk0, 4 (blk0 + nblocks)) are computed
     // Packed variable-length batch (top-k mode): query t sees keys
     // [cu_seqlens[b], t] of its own sequence b.  Null: one sequence.
     const int32_t* cu_seqlens;  // [nseq + 1], 0 ... L, non-decreasing
@@ -220,7 +221,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t L = p.L;
-    const int blk = p.nblocks - 1 - (int)blockIdx.x;  // longest rows first
+    const int blk = p.blk0 + p.nblocks - 1 - (int)blockIdx.x;  // longest rows first
     const int64_t t0 = (int64_t)blk * kTokens;
     const int64_t tmax = (t0 + kTokens - 1 < L ? t0 + kTokens - 1 : L - 1);
     // token t0 + j sees keys [seq_start(t0 + j), t0 + j]; the CTA's tiles run

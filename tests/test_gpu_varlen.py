@@ -80,3 +80,29 @@ def test_index_topk_varlen_flags_bad_ends():
     dsa.index_topk_varlen(dev(q), dev(kI), dev(w), dev(cu), cfg.k)
     assert dsa.device_error() == dsa.DEVERR_INDEX
     assert dsa.device_error() == dsa.DEVERR_NONE  # read and cleared
+
+
+def test_prefill_from_host_matches_device_path():
+    """The chunked host-to-device prefill computes exactly what the device
+    calls compute (same kernels on the same rows), with a ragged last chunk."""
+    cfg = gen.custom(L=3000, H_I=64, d_I=128, k=256, Hq=32, Hkv=4, d=128, seed=15)
+    inp = gen.prefill_inputs(cfg)
+    host = {"q_I": torch.from_numpy(inp["q_I"]).pin_memory(),
+            "k_I": torch.from_numpy(inp["k_I"]).pin_memory(),
+            "w": torch.from_numpy(inp["w"]).pin_memory(),
+            "Q": torch.from_numpy(inp["Q"].view(np.int16)).view(torch.bfloat16).pin_memory(),
+            "K": torch.from_numpy(inp["K"].view(np.int16)).view(torch.bfloat16).pin_memory(),
+            "V": torch.from_numpy(inp["V"].view(np.int16)).view(torch.bfloat16).pin_memory()}
+    host["O"] = torch.empty_like(host["Q"]).pin_memory()
+    devb = {n: torch.empty_like(host[n], device="cuda") for n in ("q_I", "k_I", "w", "Q", "K", "V", "O")}
+    devb["idx"] = torch.empty((cfg.L, cfg.k), dtype=torch.int32, device="cuda")
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    dsa.prefill_from_host(host, devb, cfg.k, cfg.scale, chunk_rows=1000, h2d_stream=s1,
+                          d2h_stream=s2)
+    torch.cuda.synchronize()
+    idx = dsa.index_topk(dev(inp["q_I"]), dev(inp["k_I"]), dev(inp["w"]), cfg.k)
+    O = dsa.sparse_attn_prefill(dev(inp["Q"], torch.bfloat16), dev(inp["K"], torch.bfloat16),
+                                dev(inp["V"], torch.bfloat16), idx, cfg.scale)
+    assert torch.equal(devb["idx"], idx)
+    assert torch.equal(host["O"], O.cpu())
+    assert dsa.device_error() == dsa.DEVERR_NONE
