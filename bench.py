@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--attn", default="auto", choices=["auto", "rows", "dedup"],
+                    help="prefill attention kernel: one CTA per query row, the adjacent-query "
+                         "dedup kernel, or auto (dedup on the video workload)")
     ap.add_argument("--union-stats", type=int, default=0, metavar="G",
                     help="instead of timing: run the prefill indexer once and report how many "
                          "distinct keys the index rows of G consecutive queries select together "
@@ -288,11 +291,13 @@ def run_ours(args, rank, world, local_rank):
             return
         dsa.index_topk(P["q_I"], P["k_I"], P["w"], pcfg.k, idx=P["idx"], stream=stream)
 
+    use_dedup = pcfg is not None and (args.attn == "dedup" or (args.attn == "auto" and pcfg.video))
+
     def attn():
         if pcfg is None:
             return
-        dsa.sparse_attn_prefill(P["Q"], P["K"], P["V"], P["idx"], pcfg.scale, O=P["O"],
-                                stream=stream)
+        f = dsa.sparse_attn_prefill_dedup if use_dedup else dsa.sparse_attn_prefill
+        f(P["Q"], P["K"], P["V"], P["idx"], pcfg.scale, O=P["O"], stream=stream)
 
     def decode():
         if dcfg is None:

@@ -115,6 +115,23 @@ DSA_API dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, con
                                    int d_I, int k, int32_t* idx, dsa_stream_t stream);
 
 /*
+ * dsa_sparse_attn_prefill_dedup - the result of dsa_sparse_attn_prefill,
+ * computed for blocks of 6 adjacent query tokens that load the union of
+ * their index rows once (adjacent-query dedup, Kwai Keye-VL-2.0 technical
+ * report summary, section 8).  Each key a block selects is gathered once;
+ * each query keeps only its own keys through a mask in the products.  It
+ * pays when adjacent rows overlap strongly (clustered video tokens); its
+ * products grow with the union, so on unclustered rows it is slower.
+ * Arguments and layouts as dsa_sparse_attn_prefill; an index row must not
+ * repeat a key (a repeat counts once here).  Supported: (d, Hkv, Hq/Hkv) in
+ * {(128, 4, 8), (64, 2, 4)}, k <= 2048, L <= 262144.
+ */
+DSA_API dsa_status_t dsa_sparse_attn_prefill_dedup(const void* Q, const void* K, const void* V,
+                                           const int32_t* idx, int64_t L, int Hq, int Hkv,
+                                           int d, int k, float scale, void* O,
+                                           dsa_stream_t stream);
+
+/*
  * dsa_prefill_from_host - the whole prefill (A1 + A2 + A3) for inputs that
  * sit in host memory.  The rows are handled in chunks of chunk_rows (rounded
  * up to a multiple of 128): each chunk's rows of q_I, k_I, w, Q, K and V are

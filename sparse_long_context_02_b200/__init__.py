@@ -50,6 +50,9 @@ def lib() -> ctypes.CDLL:
         L.dsa_index_topk.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp]
         L.dsa_index_scores.restype = i32
         L.dsa_index_scores.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
+        L.dsa_sparse_attn_prefill_dedup.restype = i32
+        L.dsa_sparse_attn_prefill_dedup.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32,
+                                                    ctypes.c_float, vp, vp]
         L.dsa_prefill_from_host.restype = i32
         L.dsa_prefill_from_host.argtypes = [vp] * 15 + [i64, i32, i32, i32, i32, i32, i32,
                                                           ctypes.c_float, i64, vp, vp, vp]
@@ -184,6 +187,23 @@ def prefill_from_host(host: dict, dev: dict, k: int, scale: float, chunk_rows: i
     _check(lib().dsa_prefill_from_host(*args, L, H, d_I, Hq, Hkv, d, k, float(scale), chunk_rows,
                                        _stream(stream), _stream(h2d_stream), _stream(d2h_stream)),
            "dsa_prefill_from_host")
+
+
+def sparse_attn_prefill_dedup(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                              idx: torch.Tensor, scale: float, O: Optional[torch.Tensor] = None,
+                              stream=None) -> torch.Tensor:
+    """sparse_attn_prefill for blocks of 6 adjacent queries that gather the
+    union of their index rows once (pays when adjacent rows overlap)."""
+    L, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    k = idx.shape[1]
+    if O is None:
+        O = torch.empty_like(Q)
+    _check(lib().dsa_sparse_attn_prefill_dedup(_dev(Q, "Q", 2), _dev(K, "K", 2), _dev(V, "V", 2),
+                                               _dev(idx, "idx", 4), L, Hq, Hkv, d, k,
+                                               float(scale), _dev(O, "O", 2), _stream(stream)),
+           "dsa_sparse_attn_prefill_dedup")
+    return O
 
 
 def decode_workspace_size(B: int, total_n: int, H_I: int, d_I: int, k: int, Hq: int, Hkv: int,

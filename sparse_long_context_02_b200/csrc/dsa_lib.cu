@@ -14,6 +14,7 @@
 
 #include "dsa.h"
 #include "decode.cuh"
+#include "sparse_attn_dedup.cuh"
 #include "index_topk.cuh"
 #include "sparse_attn.cuh"
 
@@ -190,6 +191,19 @@ dsa_status_t launch_attn(const char* fn, const dsa::attn::Params& p, int64_t gri
     return DSA_OK;
 }
 
+template <int D, int HKV, int G>
+dsa_status_t launch_dedup(const char* fn, const dsa::attn::Params& p, int64_t L, cudaStream_t st) {
+    using C = dsa::attn::DedupCfg<D, HKV>;
+    auto kern = dsa::attn::dedup_kernel<D, HKV, G>;
+    if (C::SMEM > max_optin_smem())
+        return fail(DSA_ERR_UNSUPPORTED, "%s: needs %d bytes of shared memory", fn, C::SMEM);
+    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    const int64_t grid = (L + dsa::attn::kDedupQB - 1) / dsa::attn::kDedupQB;
+    kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(p);
+    CUDA_TRY(cudaGetLastError());
+    return DSA_OK;
+}
+
 // Attention for query rows [row0, row1) over keys [0, L) (arguments
 // checked by the caller).
 dsa_status_t attn_prefill_rows(const char* fn, const void* Q, const void* K, const void* V,
@@ -267,6 +281,41 @@ dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, const float
         return fail(DSA_ERR_UNSUPPORTED, "%s: L * H_I too large", fn);
     return dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, cu_seqlens, nseq,
                                 static_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_sparse_attn_prefill_dedup(const void* Q, const void* K, const void* V,
+                                           const int32_t* idx, int64_t L, int Hq, int Hkv, int d,
+                                           int k, float scale, void* O, dsa_stream_t stream) {
+    static const char fn[] = "dsa_sparse_attn_prefill_dedup";
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(idx);
+    CHECK_PTR(O);
+    if (L < 1) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
+    if (L > dsa::attn::kDedupMaxKeys)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: L = %lld > %d", fn, (long long)L, dsa::attn::kDedupMaxKeys);
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (k > dsa::attn::kDedupMaxK) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > %d", fn, k, dsa::attn::kDedupMaxK);
+    if (Hkv < 1 || Hq < 1 || Hq % Hkv) return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d", fn, Hq, Hkv);
+    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
+    const int G = Hq / Hkv;
+    dsa::attn::Params p{};
+    p.Q = static_cast<const __nv_bfloat16*>(Q);
+    p.K = static_cast<const __nv_bfloat16*>(K);
+    p.V = static_cast<const __nv_bfloat16*>(V);
+    p.idx = idx;
+    p.nkeys = L;
+    p.k = k;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.O = static_cast<__nv_bfloat16*>(O);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    dsa_status_t r;
+    if (d == 128 && Hkv == 4 && G == 8) r = launch_dedup<128, 4, 8>(fn, p, L, st);
+    else if (d == 64 && Hkv == 2 && G == 4) r = launch_dedup<64, 2, 4>(fn, p, L, st);
+    else
+        return fail(DSA_ERR_UNSUPPORTED, "%s: (d, Hkv, Hq/Hkv) = (%d, %d, %d)", fn, d, Hkv, G);
+    return r == DSA_OK ? ok() : r;
 }
 
 dsa_status_t dsa_prefill_from_host(const void* q_I_h, const void* k_I_h, const float* w_h,
