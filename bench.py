@@ -105,29 +105,29 @@ def decode_bytes(cfg, lens) -> float:
 # from one ncu capture of the prefill L=32768 case (its summary under
 # profiles/ncu_prefill32k_decode4_index_attn.md), per prefill query token:
 # the indexer's DRAM traffic is its queries, weights and index rows (the keys
-# stay in L2), so it grows with L.  Valid only for the CUDA sources the
-# counters were taken on (their SHA-256 below); otherwise null.
+# stay in L2), so it grows with L.  Valid only for the kernel sources the
+# counters were taken on (the SHA-256 of the files listed); otherwise null.
 TRAFFIC = {
-    "dsa_index_topk": dict(bytes_per_query_token=510516224 / 32768,
-                           src_sha256="eb5cd06497475cb58d5203cda13d3b22bdb13b3991eb096de27b5d9ade8307fd"),
+    "dsa_index_topk": dict(bytes_per_query_token=(282554880 + 228671232) / 32768,
+                           sources=("index_topk.cuh", "topk_select.cuh", "ptx.cuh"),
+                           src_sha256="f56f3ee75da1563ddaf911e63c7f34293912a3187bf81711c5c279f1b18ad11c"),
 }
 
 
-def csrc_sha256() -> str:
-    import glob
+def csrc_sha256(sources) -> str:
     import hashlib
     root = os.path.join(ROOT, "sparse_long_context_02_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(root, "*.cu")) + glob.glob(os.path.join(root, "*.cuh"))):
-        h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
+    for name in sorted(sources):
+        h.update(name.encode())
+        with open(os.path.join(root, name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
 
 def dram_traffic(kernel: str, pcfg):
     t = TRAFFIC.get(kernel)
-    if t is None or pcfg is None or t["src_sha256"] != csrc_sha256():
+    if t is None or pcfg is None or t["src_sha256"] != csrc_sha256(t["sources"]):
         return None
     return t["bytes_per_query_token"] * pcfg.L
 
