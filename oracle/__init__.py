@@ -16,6 +16,9 @@ and section 8; formula readings listed in the C file's header):
 * ``dense_causal_attn`` - plain causal attention, written separately, used as
                      a pin (k >= t + 1 must reduce to it).
 * ``decode``       - one new token per sequence over a packed cache.
+* ``kl.indexer_kl`` - the indexer's dense warm-up loss (KL from the head-mean
+                     full attention to the indexer's softmax) and its
+                     gradients, in numpy float64 (``oracle/kl.py``).
 
 Parity is pinned for every function here (see tests/test_oracle_pins.py);
 the pages' own measured figures (cost ratios, dedup counts) depend on the
