@@ -252,6 +252,64 @@ DSA_API dsa_status_t dsa_sparse_attn_decode_noalloc(
     int Hq, int Hkv, int d, int k, float scale, void* O, int32_t* idx_out, dsa_stream_t stream);
 
 /*
+ * Indexer warm-up loss (dense warm-up stage: Kwai Keye-VL-2.0 technical
+ * report summary, section 1 -- the full attention is kept and only the
+ * Lightning Indexer is trained, towards the full attention's distribution,
+ * under a KL divergence).  The pages print no formula; the reading taken:
+ *
+ *   I[t,s]  = sum_j w[t,j] relu(q_I[t,j] . k_I[s])                (s <= t)
+ *   P_I[t]  = softmax_s(scale_I * I[t,s])
+ *   p[t,s]  = (1/Hq) sum_h softmax_s(scale * Q[t,h] . K[s, h / (Hq/Hkv)])
+ *   kl[t]   = sum_s p[t,s] (ln p[t,s] - ln P_I[t,s])     (0 ln 0 = 0)
+ *   G[t,s]  = d(sum_t kl[t]) / dI[t,s] = scale_I (P_I[t,s] - p[t,s])
+ *
+ * The attention side is the target and gets no gradient.
+ *
+ * dsa_indexer_kl_workspace_size - bytes of device workspace the forward
+ * needs (256-byte aligned pointer).
+ */
+DSA_API size_t dsa_indexer_kl_workspace_size(int64_t L, int Hq);
+
+/*
+ * dsa_indexer_kl_forward - the loss per token and dL/dI.
+ *
+ *   q_I  [L][H_I][d_I] e4m3,  k_I [L][d_I] e4m3,  w [L][H_I] fp32
+ *   Q    [L][Hq][d] bf16,     K   [L][Hkv][d] bf16
+ *   kl   [L]    fp32  OUT
+ *   G    [L][L] fp32  OUT: G[t,s] for s <= t, 0 above the diagonal
+ * Supported: (H_I, d_I) as dsa_index_topk; d in {64, 128}; Hkv <= 8 with
+ * Hq a multiple of Hkv; L * L < 2^31.  Work: the indexer scores (tcgen05,
+ * FP8), then two tensor-core passes over the attention scores.  Results are
+ * bit-identical run to run.  Errors: DSA_ERR_INVALID_ARG for bad sizes or
+ * null pointers, DSA_ERR_WORKSPACE if workspace_bytes is short.
+ */
+DSA_API dsa_status_t dsa_indexer_kl_forward(const void* q_I, const void* k_I, const float* w,
+                                    const void* Q, const void* K, int64_t L, int H_I, int d_I,
+                                    int Hq, int Hkv, int d, float scale, float scale_I, float* kl,
+                                    float* G, void* workspace, size_t workspace_bytes,
+                                    dsa_stream_t stream);
+
+/*
+ * dsa_indexer_kl_backward - gradients of sum_t kl[t] with respect to the
+ * indexer's inputs, from G:
+ *
+ *   dw[t,j]   = sum_{s<=t} G[t,s] relu(S)
+ *   dq_I[t,j] = w[t,j] sum_{s<=t} G[t,s] [S > 0] k_I[s]
+ *   dk_I[s]   = sum_{t>=s} sum_j G[t,s] w[t,j] [S > 0] q_I[t,j]
+ *   with S = q_I[t,j] . k_I[s] (exact in fp32 for the e4m3 inputs' range
+ *   used here; the ReLU's derivative at 0 is 0).
+ *
+ *   G     [L][L]         fp32  (only s <= t is read)
+ *   dq_I  [L][H_I][d_I]  fp32  OUT,  dk_I [L][d_I] fp32 OUT,  dw [L][H_I] fp32 OUT
+ * G [S > 0] w is rounded to bf16 for the two products with k_I and q_I (fp32
+ * accumulation); dw is fp32 throughout.  Supported: d_I in {64, 128},
+ * 1 <= H_I <= 256, L * L < 2^31.
+ */
+DSA_API dsa_status_t dsa_indexer_kl_backward(const void* q_I, const void* k_I, const float* w,
+                                     const float* G, int64_t L, int H_I, int d_I, float* dq_I,
+                                     float* dk_I, float* dw, dsa_stream_t stream);
+
+/*
  * dsa_device_error - synchronizes `stream`, then reads and clears the
  * current device's error word into *code (DSA_DEVERR_*).  Returns DSA_OK if
  * the word could be read (whatever its value), DSA_ERR_CUDA otherwise.

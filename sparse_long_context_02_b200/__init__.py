@@ -69,6 +69,13 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_attn_decode_noalloc.restype = i32
         L.dsa_sparse_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
                                                      i32, i32, i32, i32, i32, f32, vp, vp, vp]
+        L.dsa_indexer_kl_workspace_size.restype = sz
+        L.dsa_indexer_kl_workspace_size.argtypes = [i64, i32]
+        L.dsa_indexer_kl_forward.restype = i32
+        L.dsa_indexer_kl_forward.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, f32,
+                                             f32, vp, vp, vp, sz, vp]
+        L.dsa_indexer_kl_backward.restype = i32
+        L.dsa_indexer_kl_backward.argtypes = [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp]
         L.dsa_device_error.restype = i32
         L.dsa_device_error.argtypes = [ctypes.POINTER(i32), vp]
         _lib = L
@@ -126,7 +133,7 @@ def index_topk_varlen(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor,
     if idx is None:
         idx = torch.empty((L, k), dtype=torch.int32, device=q_I.device)
     if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
-        raise DSAError("dsa_index_topk_varlen: cu_seqlens must be an int32 device tensor")
+        raise ValueError("dsa_index_topk_varlen: cu_seqlens must be an int32 device tensor")
     nseq = cu_seqlens.numel() - 1
     _check(lib().dsa_index_topk_varlen(_dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4),
                                        _dev(cu_seqlens, "cu_seqlens", 4), nseq, L, H, d, k,
@@ -259,3 +266,53 @@ def device_error(stream=None) -> int:
     code = ctypes.c_int(0)
     _check(lib().dsa_device_error(ctypes.byref(code), _stream(stream)), "dsa_device_error")
     return code.value
+
+
+def indexer_kl_workspace_size(L: int, Hq: int) -> int:
+    return lib().dsa_indexer_kl_workspace_size(L, Hq)
+
+
+def indexer_kl_forward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, Q: torch.Tensor,
+                       K: torch.Tensor, scale: float, scale_I: float = 1.0,
+                       kl: Optional[torch.Tensor] = None, G: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None):
+    """Indexer warm-up loss.  Returns (kl [L] float32, G [L][L] float32 =
+    d(sum kl)/dI, zero above the diagonal).  q_I/k_I e4m3, w float32, Q/K
+    bf16 (layouts as dsa_indexer_kl_forward)."""
+    L, H_I, d_I = q_I.shape
+    _, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    dev = q_I.device
+    if kl is None:
+        kl = torch.empty(L, dtype=torch.float32, device=dev)
+    if G is None:
+        G = torch.empty((L, L), dtype=torch.float32, device=dev)
+    need = indexer_kl_workspace_size(L, Hq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check(lib().dsa_indexer_kl_forward(
+        _dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), _dev(Q, "Q", 2),
+        _dev(K, "K", 2), L, H_I, d_I, Hq, Hkv, d, float(scale), float(scale_I), _dev(kl, "kl", 4),
+        _dev(G, "G", 4), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "dsa_indexer_kl_forward")
+    return kl, G
+
+
+def indexer_kl_backward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, G: torch.Tensor,
+                        dq_I: Optional[torch.Tensor] = None, dk_I: Optional[torch.Tensor] = None,
+                        dw: Optional[torch.Tensor] = None, stream=None):
+    """Gradients of sum_t kl[t] with respect to q_I, k_I and w, from G.
+    Returns (dq_I [L][H_I][d_I], dk_I [L][d_I], dw [L][H_I]), float32."""
+    L, H_I, d_I = q_I.shape
+    dev = q_I.device
+    if dq_I is None:
+        dq_I = torch.empty((L, H_I, d_I), dtype=torch.float32, device=dev)
+    if dk_I is None:
+        dk_I = torch.empty((L, d_I), dtype=torch.float32, device=dev)
+    if dw is None:
+        dw = torch.empty((L, H_I), dtype=torch.float32, device=dev)
+    _check(lib().dsa_indexer_kl_backward(
+        _dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), _dev(G, "G", 4), L, H_I, d_I,
+        _dev(dq_I, "dq_I", 4), _dev(dk_I, "dk_I", 4), _dev(dw, "dw", 4), _stream(stream)),
+        "dsa_indexer_kl_backward")
+    return dq_I, dk_I, dw

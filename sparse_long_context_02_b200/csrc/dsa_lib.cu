@@ -17,6 +17,7 @@
 #include "sparse_attn_dedup.cuh"
 #include "index_topk.cuh"
 #include "sparse_attn.cuh"
+#include "indexer_kl.cuh"
 
 namespace {
 
@@ -649,3 +650,146 @@ extern "C" dsa_status_t dsa_sparse_attn_decode_noalloc(
                                   H_I, d_I, Hq, Hkv, d, k, scale, O, idx_out, scratch,
                                   kNoAllocScratchBytes, stream);
 }
+
+// ---------------------------------------------------------------- indexer warm-up loss
+
+namespace {
+
+struct KlWorkspace {
+    size_t lse_h, lse_I, part, total;
+    KlWorkspace(int64_t L, int Hq) {
+        const int64_t nt = (L + dsa::kl::kTile - 1) / dsa::kl::kTile;
+        lse_h = 0;
+        lse_I = align256((size_t)L * Hq * 4);
+        part = lse_I + align256((size_t)L * 4);
+        total = part + align256((size_t)L * nt * 4);
+    }
+};
+
+template <int D>
+dsa_status_t launch_kl_forward(const char* fn, const dsa::kl::Params& p, cudaStream_t st) {
+    using namespace dsa::kl;
+    const int smem_lse = 2 * BfTile<D>::BYTES;
+    const int smem_tgt = (p.Hkv + 2) * BfTile<D>::BYTES;
+    CUDA_TRY(cudaFuncSetAttribute(head_lse_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem_lse));
+    CUDA_TRY(cudaFuncSetAttribute(target_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem_tgt));
+    row_lse_kernel<<<(unsigned)((p.L + 7) / 8), 256, 0, st>>>(p);
+    head_lse_kernel<D><<<dim3(p.ntiles, p.Hq), kThreads, smem_lse, st>>>(p);
+    target_kernel<D><<<dim3(p.ntiles, p.ntiles), kThreads, smem_tgt, st>>>(p);
+    kl_reduce_kernel<<<(unsigned)((p.L + 255) / 256), 256, 0, st>>>(p);
+    CUDA_TRY(cudaGetLastError());
+    return DSA_OK;
+}
+
+template <int DI>
+dsa_status_t launch_kl_backward(const char* fn, const dsa::kl::Params& p, cudaStream_t st) {
+    using namespace dsa::kl;
+    const int smem_dq = 2 * F8Tile<DI>::BYTES;
+    const int smem_dk = 2 * F8Tile<DI>::BYTES + p.HI * kWStride * 4;
+    CUDA_TRY(cudaFuncSetAttribute(dq_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem_dq));
+    CUDA_TRY(cudaFuncSetAttribute(dk_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem_dk));
+    dq_kernel<DI><<<dim3(p.ntiles, p.HI), kThreads, smem_dq, st>>>(p);
+    dk_kernel<DI><<<p.ntiles, kThreads, smem_dk, st>>>(p);
+    CUDA_TRY(cudaGetLastError());
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dsa_indexer_kl_workspace_size(int64_t L, int Hq) {
+    if (L < 1 || Hq < 1) return 0;
+    return KlWorkspace(L, Hq).total;
+}
+
+dsa_status_t dsa_indexer_kl_forward(const void* q_I, const void* k_I, const float* w,
+                                    const void* Q, const void* K, int64_t L, int H_I, int d_I,
+                                    int Hq, int Hkv, int d, float scale, float scale_I, float* kl,
+                                    float* G, void* workspace, size_t workspace_bytes,
+                                    dsa_stream_t stream) {
+    static const char fn[] = "dsa_indexer_kl_forward";
+    CHECK_PTR(q_I);
+    CHECK_PTR(k_I);
+    CHECK_PTR(w);
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(kl);
+    CHECK_PTR(G);
+    CHECK_PTR(workspace);
+    if (L < 1 || L * L >= (int64_t(1) << 31))
+        return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld (L * L must be < 2^31)", fn, (long long)L);
+    if (Hkv < 1 || Hkv > 8 || Hq < Hkv || Hq % Hkv != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d (Hkv in 1..8 dividing Hq)", fn, Hq,
+                    Hkv);
+    if (d != 64 && d != 128) return fail(DSA_ERR_UNSUPPORTED, "%s: d = %d (64 or 128)", fn, d);
+    if (!(scale_I > 0.f) || !(scale > 0.f))
+        return fail(DSA_ERR_INVALID_ARG, "%s: scale and scale_I must be > 0", fn);
+    const KlWorkspace ws(L, Hq);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace must be 256-byte aligned", fn);
+    if (workspace_bytes < ws.total)
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace of %zu bytes, %zu needed", fn,
+                    workspace_bytes, ws.total);
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    dsa_status_t r = dispatch_index<false>(fn, q_I, k_I, w, L, H_I, d_I, 1, nullptr, G, nullptr, 1,
+                                           st);
+    if (r != DSA_OK) return r;
+    dsa::kl::Params p{};
+    p.Q = static_cast<const __nv_bfloat16*>(Q);
+    p.K = static_cast<const __nv_bfloat16*>(K);
+    p.L = L;
+    p.HI = H_I;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.ntiles = (int)((L + dsa::kl::kTile - 1) / dsa::kl::kTile);
+    p.scale_log2 = scale * dsa::kl::kLog2e;
+    p.scale_I = scale_I;
+    p.G = G;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    p.lse_h = reinterpret_cast<float*>(wsb + ws.lse_h);
+    p.lse_I = reinterpret_cast<float*>(wsb + ws.lse_I);
+    p.kl_part = reinterpret_cast<float*>(wsb + ws.part);
+    p.kl = kl;
+    r = d == 128 ? launch_kl_forward<128>(fn, p, st) : launch_kl_forward<64>(fn, p, st);
+    return r == DSA_OK ? ok() : r;
+}
+
+dsa_status_t dsa_indexer_kl_backward(const void* q_I, const void* k_I, const float* w,
+                                     const float* G, int64_t L, int H_I, int d_I, float* dq_I,
+                                     float* dk_I, float* dw, dsa_stream_t stream) {
+    static const char fn[] = "dsa_indexer_kl_backward";
+    CHECK_PTR(q_I);
+    CHECK_PTR(k_I);
+    CHECK_PTR(w);
+    CHECK_PTR(G);
+    CHECK_PTR(dq_I);
+    CHECK_PTR(dk_I);
+    CHECK_PTR(dw);
+    if (L < 1 || L * L >= (int64_t(1) << 31))
+        return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld (L * L must be < 2^31)", fn, (long long)L);
+    if (H_I < 1 || H_I > 256) return fail(DSA_ERR_INVALID_ARG, "%s: H_I = %d (1..256)", fn, H_I);
+    if (d_I != 64 && d_I != 128)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: d_I = %d (64 or 128)", fn, d_I);
+    dsa::kl::Params p{};
+    p.qI = static_cast<const uint8_t*>(q_I);
+    p.kI = static_cast<const uint8_t*>(k_I);
+    p.w = w;
+    p.L = L;
+    p.HI = H_I;
+    p.ntiles = (int)((L + dsa::kl::kTile - 1) / dsa::kl::kTile);
+    p.Gin = G;
+    p.dq = dq_I;
+    p.dk = dk_I;
+    p.dw = dw;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const dsa_status_t r =
+        d_I == 128 ? launch_kl_backward<128>(fn, p, st) : launch_kl_backward<64>(fn, p, st);
+    return r == DSA_OK ? ok() : r;
+}
+
+}  // extern "C"
