@@ -62,6 +62,10 @@ def parse():
                     help="instead of timing: run the prefill indexer once and report how many "
                          "distinct keys the index rows of G consecutive queries select together "
                          "(the traffic an adjacent-query dedup would read)")
+    ap.add_argument("--kl", type=int, default=0, metavar="L",
+                    help="instead of the inference step: time the indexer warm-up KL loss "
+                         "(forward: loss and dL/dI; backward: dq_I, dk_I, dw) at sequence "
+                         "length L with the prefill workload's head shapes")
     return ap.parse_args()
 
 
@@ -546,6 +550,93 @@ def union_stats(args) -> dict:
                 p90=float(np.percentile(fr, 90)), k=cfg.k, data="synthetic")
 
 
+def kl_flops(L, H_I, d_I, Hq, d):
+    """Algorithmic tensor work of the warm-up loss per causal (t, s) pair:
+    forward = indexer scores (FP8, 2 H_I d_I) + two passes over the attention
+    scores (bf16, 2 x 2 Hq d); backward = the indexer scores again in each of
+    its two kernels (FP8, 2 x 2 H_I d_I) + the dS products with k_I and q_I
+    (bf16, 2 x 2 H_I d_I)."""
+    pairs = L * (L + 1) / 2.0
+    return dict(fwd_fp8=pairs * 2 * H_I * d_I, fwd_bf16=pairs * 2 * 2 * Hq * d,
+                bwd_fp8=pairs * 2 * 2 * H_I * d_I, bwd_bf16=pairs * 2 * 2 * H_I * d_I)
+
+
+def kl_bench(args) -> dict:
+    """Times dsa_indexer_kl_forward and dsa_indexer_kl_backward with CUDA events
+    (L2 flushed before each step), reports tokens/s of forward + backward and
+    the tensor roofline of each call: the time its FP8 and bf16 work would
+    take at the measured peaks, divided by the measured time."""
+    import torch
+    import sparse_long_context_02_b200 as dsa
+    L = args.kl
+    base = gen.CONFIGS[3]
+    cfg = gen.custom(L=L, H_I=base.H_I, d_I=base.d_I, k=8, Hq=base.Hq, Hkv=base.Hkv, d=base.d,
+                     seed=51)
+    host = gen.prefill_inputs(cfg)
+    q, kI, w = (torch.from_numpy(host[n]).cuda() for n in ("q_I", "k_I", "w"))
+    Q, K = (torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).cuda() for n in ("Q", "K"))
+    scale_I = 1.0 / 2048
+    kl = torch.empty(L, dtype=torch.float32, device="cuda")
+    G = torch.empty((L, L), dtype=torch.float32, device="cuda")
+    ws = torch.empty(dsa.indexer_kl_workspace_size(L, cfg.Hq), dtype=torch.uint8, device="cuda")
+    dq = torch.empty((L, cfg.H_I, cfg.d_I), dtype=torch.float32, device="cuda")
+    dk = torch.empty((L, cfg.d_I), dtype=torch.float32, device="cuda")
+    dw = torch.empty((L, cfg.H_I), dtype=torch.float32, device="cuda")
+    wsb = torch.empty(dsa.lib().dsa_indexer_kl_backward_workspace_size(L, cfg.H_I, cfg.d_I),
+                      dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        dsa.indexer_kl_forward(q, kI, w, Q, K, cfg.scale, scale_I, kl=kl, G=G, workspace=ws)
+        if ev:
+            ev[1].record()
+        dsa.indexer_kl_backward(q, kI, w, G, dq_I=dq, dk_I=dk, dw=dw, workspace=wsb)
+        if ev:
+            ev[2].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = Clocks(torch.cuda.current_device())
+    clocks.start()
+    tf, tb = [], []
+    for _ in range(args.steps):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        step(ev)
+        torch.cuda.synchronize()
+        tf.append(ev[0].elapsed_time(ev[1]))
+        tb.append(ev[1].elapsed_time(ev[2]))
+    ck = clocks.stop()
+    if dsa.device_error() != dsa.DEVERR_NONE:
+        raise RuntimeError("device error during the KL loss")
+    pk = peaks()
+    fp8_peak = 2 * pk["bf16_sus"]  # TFLOP/s
+    bf16_peak = pk["bf16_sus"]
+    fl = kl_flops(L, cfg.H_I, cfg.d_I, cfg.Hq, cfg.d)
+    ms_f, ms_b = float(np.mean(tf)), float(np.mean(tb))
+
+    def roof(ms, f8, b16):
+        ideal_ms = (f8 / (fp8_peak * 1e12) + b16 / (bf16_peak * 1e12)) * 1e3
+        return dict(bound="tensor", ms=ms, flops=f8 + b16,
+                    achieved=(f8 + b16) / (ms * 1e-3) / 1e12, unit="TFLOP/s",
+                    ideal_ms=ideal_ms, frac=ideal_ms / ms)
+
+    return dict(metric="indexer warm-up KL loss, forward + backward tokens/s",
+                value=L / ((ms_f + ms_b) * 1e-3), unit="tokens/s", higher_is_better=True,
+                steps=args.steps, warmup=args.warmup, dtype="fp8-e4m3/bf16", data="synthetic",
+                config=dict(workload="indexer KL loss L=%d" % L, L=L, H_I=cfg.H_I, d_I=cfg.d_I,
+                            Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, scale_I=scale_I,
+                            l2="flushed before each step (256 MiB write, outside the events)"),
+                forward=roof(ms_f, fl["fwd_fp8"], fl["fwd_bf16"]),
+                backward=roof(ms_b, fl["bwd_fp8"], fl["bwd_bf16"]),
+                peaks=dict(fp8_tflops=fp8_peak, bf16_tflops=bf16_peak,
+                           source=pk["src"] + " (bf16 sustained; fp8 = 2 x bf16)"),
+                clocks=ck, mean_kl=float(kl.mean().item()))
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -559,6 +650,10 @@ def main():
     if args.union_stats:
         if rank == 0:
             print(json.dumps(union_stats(args)), flush=True)
+        return
+    if args.kl:
+        if rank == 0:
+            print(json.dumps(kl_bench(args)), flush=True)
         return
 
     import datetime

@@ -302,12 +302,18 @@ DSA_API dsa_status_t dsa_indexer_kl_forward(const void* q_I, const void* k_I, co
  *   G     [L][L]         fp32  (only s <= t is read)
  *   dq_I  [L][H_I][d_I]  fp32  OUT,  dk_I [L][d_I] fp32 OUT,  dw [L][H_I] fp32 OUT
  * G [S > 0] w is rounded to bf16 for the two products with k_I and q_I (fp32
- * accumulation); dw is fp32 throughout.  Supported: d_I in {64, 128},
- * 1 <= H_I <= 256, L * L < 2^31.
+ * accumulation); dw is fp32 throughout.  dk_I is summed over groups of heads
+ * through the caller's workspace (dsa_indexer_kl_backward_workspace_size
+ * bytes, 256-byte aligned), in a fixed order: results are bit-identical run
+ * to run.  Supported: d_I in {64, 128}, 1 <= H_I <= 256, L * L < 2^31.
+ * Errors: DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE.
  */
+DSA_API size_t dsa_indexer_kl_backward_workspace_size(int64_t L, int H_I, int d_I);
+
 DSA_API dsa_status_t dsa_indexer_kl_backward(const void* q_I, const void* k_I, const float* w,
                                      const float* G, int64_t L, int H_I, int d_I, float* dq_I,
-                                     float* dk_I, float* dw, dsa_stream_t stream);
+                                     float* dk_I, float* dw, void* workspace,
+                                     size_t workspace_bytes, dsa_stream_t stream);
 
 /*
  * dsa_device_error - synchronizes `stream`, then reads and clears the

@@ -75,7 +75,10 @@ def lib() -> ctypes.CDLL:
         L.dsa_indexer_kl_forward.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, f32,
                                              f32, vp, vp, vp, sz, vp]
         L.dsa_indexer_kl_backward.restype = i32
-        L.dsa_indexer_kl_backward.argtypes = [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp]
+        L.dsa_indexer_kl_backward_workspace_size.restype = sz
+        L.dsa_indexer_kl_backward_workspace_size.argtypes = [i64, i32, i32]
+        L.dsa_indexer_kl_backward.argtypes = [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz,
+                                              vp]
         L.dsa_device_error.restype = i32
         L.dsa_device_error.argtypes = [ctypes.POINTER(i32), vp]
         _lib = L
@@ -300,11 +303,15 @@ def indexer_kl_forward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, Q:
 
 def indexer_kl_backward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, G: torch.Tensor,
                         dq_I: Optional[torch.Tensor] = None, dk_I: Optional[torch.Tensor] = None,
-                        dw: Optional[torch.Tensor] = None, stream=None):
+                        dw: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None):
     """Gradients of sum_t kl[t] with respect to q_I, k_I and w, from G.
     Returns (dq_I [L][H_I][d_I], dk_I [L][d_I], dw [L][H_I]), float32."""
     L, H_I, d_I = q_I.shape
     dev = q_I.device
+    if workspace is None:
+        workspace = torch.empty(lib().dsa_indexer_kl_backward_workspace_size(L, H_I, d_I),
+                                dtype=torch.uint8, device=dev)
     if dq_I is None:
         dq_I = torch.empty((L, H_I, d_I), dtype=torch.float32, device=dev)
     if dk_I is None:
@@ -313,6 +320,7 @@ def indexer_kl_backward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, G
         dw = torch.empty((L, H_I), dtype=torch.float32, device=dev)
     _check(lib().dsa_indexer_kl_backward(
         _dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), _dev(G, "G", 4), L, H_I, d_I,
-        _dev(dq_I, "dq_I", 4), _dev(dk_I, "dk_I", 4), _dev(dw, "dw", 4), _stream(stream)),
-        "dsa_indexer_kl_backward")
+        _dev(dq_I, "dq_I", 4), _dev(dk_I, "dk_I", 4), _dev(dw, "dw", 4),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "dsa_indexer_kl_backward")
     return dq_I, dk_I, dw

@@ -687,20 +687,35 @@ template <int DI>
 dsa_status_t launch_kl_backward(const char* fn, const dsa::kl::Params& p, cudaStream_t st) {
     using namespace dsa::kl;
     const int smem_dq = 2 * F8Tile<DI>::BYTES;
-    const int smem_dk = 2 * F8Tile<DI>::BYTES + p.HI * kWStride * 4;
+    const int smem_dk = 2 * F8Tile<DI>::BYTES + (p.HI / p.nsplit) * kWStride * 4;
     CUDA_TRY(cudaFuncSetAttribute(dq_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem_dq));
     CUDA_TRY(cudaFuncSetAttribute(dk_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem_dk));
-    dq_kernel<DI><<<dim3(p.ntiles, p.HI), kThreads, smem_dq, st>>>(p);
-    dk_kernel<DI><<<p.ntiles, kThreads, smem_dk, st>>>(p);
+    dq_kernel<DI><<<dim3(p.HI, p.ntiles), kThreads, smem_dq, st>>>(p);
+    dk_kernel<DI><<<dim3(p.nsplit, p.ntiles), kThreads, smem_dk, st>>>(p);
+    if (p.nsplit > 1)
+        dk_reduce_kernel<<<(unsigned)((p.L * DI / 4 + 255) / 256), 256, 0, st>>>(p, DI);
     CUDA_TRY(cudaGetLastError());
     return DSA_OK;
+}
+
+// Head groups of dk_kernel: the largest divisor of H_I that is at most 8.
+int kl_dk_splits(int H_I) {
+    for (int n = 8; n > 1; --n)
+        if (H_I % n == 0) return n;
+    return 1;
 }
 
 }  // namespace
 
 extern "C" {
+
+size_t dsa_indexer_kl_backward_workspace_size(int64_t L, int H_I, int d_I) {
+    if (L < 1 || H_I < 1 || d_I < 1) return 0;
+    const int n = kl_dk_splits(H_I);
+    return n > 1 ? align256((size_t)n * L * d_I * 4) : 256;
+}
 
 size_t dsa_indexer_kl_workspace_size(int64_t L, int Hq) {
     if (L < 1 || Hq < 1) return 0;
@@ -761,7 +776,8 @@ dsa_status_t dsa_indexer_kl_forward(const void* q_I, const void* k_I, const floa
 
 dsa_status_t dsa_indexer_kl_backward(const void* q_I, const void* k_I, const float* w,
                                      const float* G, int64_t L, int H_I, int d_I, float* dq_I,
-                                     float* dk_I, float* dw, dsa_stream_t stream) {
+                                     float* dk_I, float* dw, void* workspace,
+                                     size_t workspace_bytes, dsa_stream_t stream) {
     static const char fn[] = "dsa_indexer_kl_backward";
     CHECK_PTR(q_I);
     CHECK_PTR(k_I);
@@ -775,7 +791,16 @@ dsa_status_t dsa_indexer_kl_backward(const void* q_I, const void* k_I, const flo
     if (H_I < 1 || H_I > 256) return fail(DSA_ERR_INVALID_ARG, "%s: H_I = %d (1..256)", fn, H_I);
     if (d_I != 64 && d_I != 128)
         return fail(DSA_ERR_UNSUPPORTED, "%s: d_I = %d (64 or 128)", fn, d_I);
+    CHECK_PTR(workspace);
+    const size_t need = dsa_indexer_kl_backward_workspace_size(L, H_I, d_I);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace must be 256-byte aligned", fn);
+    if (workspace_bytes < need)
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace of %zu bytes, %zu needed", fn,
+                    workspace_bytes, need);
     dsa::kl::Params p{};
+    p.nsplit = kl_dk_splits(H_I);
+    p.dk_part = static_cast<float*>(workspace);
     p.qI = static_cast<const uint8_t*>(q_I);
     p.kI = static_cast<const uint8_t*>(k_I);
     p.w = w;

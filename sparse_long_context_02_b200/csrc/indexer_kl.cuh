@@ -20,7 +20,9 @@
 //   target_kernel      p, the row KL partials and G, written over I in place
 //   kl_reduce_kernel   kl[t] from the partials in a fixed order
 //   dq_kernel          dq_I and dw for one indexer head and 64 query rows
-//   dk_kernel          dk_I for 64 keys, over all later query rows and heads
+//   dk_kernel          dk_I for 64 keys, over all later query rows and a group
+//                      of heads (one partial per group)
+//   dk_reduce_kernel   dk_I = sum of the groups' partials, in a fixed order
 // The score products run on the tensor cores (bf16 m16n8k16 for the
 // attention, e4m3 m16n8k32 for the indexer); dS is rounded to bf16 for the
 // dq/dk products, as a flash-attention backward does.  Every result is
@@ -62,6 +64,8 @@ struct Params {
     float* dq;                // [L][HI][DI]
     float* dk;                // [L][DI]
     float* dw;                // [L][HI]
+    int nsplit;               // head groups of dk_kernel (a divisor of HI)
+    float* dk_part;           // [nsplit][L][DI] (nsplit > 1)
 };
 
 using attn::ex2;
@@ -473,11 +477,12 @@ __device__ __forceinline__ void ds_times_rows(float (&acc)[DI / 8][4], const flo
     }
 }
 
-// dq_I and dw of indexer head j for 64 query rows.  Grid (ntiles, HI).
+// dq_I and dw of indexer head j for 64 query rows.  Grid (HI, ntiles): the
+// heads of one query tile run side by side and share its G band in L2.
 template <int DI>
 __global__ void __launch_bounds__(kThreads) dq_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int qt = p.ntiles - 1 - blockIdx.x, j = blockIdx.y;
+    const int qt = p.ntiles - 1 - blockIdx.y, j = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
     const int64_t t_a = (int64_t)qt * kTile + warp * 16 + r, t_b = t_a + 8;
     const int64_t ra = t_a < p.L ? t_a : p.L - 1, rb = t_b < p.L ? t_b : p.L - 1;
@@ -550,19 +555,20 @@ __global__ void __launch_bounds__(kThreads) dq_kernel(const Params p) {
 }
 
 // dk_I for 64 keys: over every query tile at or after the keys' tile and
-// every indexer head.  Grid (ntiles); the longest key tiles (the first)
-// first.  Shared: a two-slot ring of q_I tiles, then w^T of the query tile
+// the heads of one group.  Grid (nsplit, ntiles): the groups of one key tile
+// run side by side; the longest key tiles (the first) first.  Shared: a two-slot ring of q_I tiles, then w^T of the query tile
 // (rows of kWStride floats: the transposing stores avoid bank conflicts).
 constexpr int kWStride = kTile + 1;
 
 template <int DI>
 __global__ void __launch_bounds__(kThreads) dk_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int kt = blockIdx.x;
+    const int split = blockIdx.x, kt = blockIdx.y;
+    const int hps = p.HI / p.nsplit, j0 = split * hps;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
     const int64_t s_a = (int64_t)kt * kTile + warp * 16 + r, s_b = s_a + 8;
     const int64_t ra = s_a < p.L ? s_a : p.L - 1, rb = s_b < p.L ? s_b : p.L - 1;
-    float* wT = reinterpret_cast<float*>(smem + 2 * F8Tile<DI>::BYTES);  // [HI][kWStride]
+    float* wT = reinterpret_cast<float*>(smem + 2 * F8Tile<DI>::BYTES);  // [hps][kWStride]
 
     uint32_t ka[DI / 32][4];
     load_a_e4m3<DI>(ka, p.kI + ra * DI, p.kI + rb * DI);
@@ -590,15 +596,15 @@ __global__ void __launch_bounds__(kThreads) dk_kernel(const Params p) {
                 gv[nt][2 + e] = tv && s_b <= t && s_b < p.L ? p.Gin[t * p.L + s_b] : 0.f;
             }
         __syncthreads();  // the previous tile's w^T and q slots are no longer read
-        for (int i = threadIdx.x; i < kTile * p.HI; i += kThreads) {
-            const int tt = i / p.HI, jj = i % p.HI;
-            wT[jj * kWStride + tt] = tt < qn ? p.w[(t0 + tt) * p.HI + jj] : 0.f;
+        for (int i = threadIdx.x; i < kTile * hps; i += kThreads) {
+            const int tt = i / hps, jj = i % hps;
+            wT[jj * kWStride + tt] = tt < qn ? p.w[(t0 + tt) * p.HI + j0 + jj] : 0.f;
         }
-        ld.load(p.qI + t0 * qstride, qstride, qn);
+        ld.load(p.qI + t0 * qstride + j0 * DI, qstride, qn);
         ld.store(smem + slot * F8Tile<DI>::BYTES);
         __syncthreads();
-        for (int j = 0; j < p.HI; ++j) {
-            if (j + 1 < p.HI) ld.load(p.qI + t0 * qstride + (j + 1) * DI, qstride, qn);
+        for (int j = 0; j < hps; ++j) {
+            if (j + 1 < hps) ld.load(p.qI + t0 * qstride + (j0 + j + 1) * DI, qstride, qn);
             const uint32_t base = smem_u32(smem + slot * F8Tile<DI>::BYTES);
             float S[8][4];
             qk_e4m3<DI>(S, ka, base);
@@ -611,25 +617,43 @@ __global__ void __launch_bounds__(kThreads) dk_kernel(const Params p) {
                     S[nt][2 + e] = S[nt][2 + e] > 0.f ? gv[nt][2 + e] * wv : 0.f;
                 }
             ds_times_rows<DI>(acc, S, base);
-            if (j + 1 < p.HI) {
+            if (j + 1 < hps) {
                 ld.store(smem + (slot ^ 1) * F8Tile<DI>::BYTES);
                 __syncthreads();
                 slot ^= 1;
             }
         }
     }
+    float* dk = p.nsplit > 1 ? p.dk_part + (int64_t)split * p.L * DI : p.dk;
     if (s_a < p.L) {
-        float* out = p.dk + s_a * DI;
+        float* out = dk + s_a * DI;
 #pragma unroll
         for (int n = 0; n < DI / 8; ++n)
             *reinterpret_cast<float2*>(out + n * 8 + 2 * c) = make_float2(acc[n][0], acc[n][1]);
     }
     if (s_b < p.L) {
-        float* out = p.dk + s_b * DI;
+        float* out = dk + s_b * DI;
 #pragma unroll
         for (int n = 0; n < DI / 8; ++n)
             *reinterpret_cast<float2*>(out + n * 8 + 2 * c) = make_float2(acc[n][2], acc[n][3]);
     }
+}
+
+// dk_I[i] = sum over the head groups' partials, in group order (float4).
+__global__ void dk_reduce_kernel(const Params p, int DI) {
+    const int64_t n4 = p.L * DI / 4;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    const float4* part = reinterpret_cast<const float4*>(p.dk_part);
+    float4 a = part[i];
+    for (int sp = 1; sp < p.nsplit; ++sp) {
+        const float4 b = part[sp * n4 + i];
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+    }
+    reinterpret_cast<float4*>(p.dk)[i] = a;
 }
 
 }  // namespace kl

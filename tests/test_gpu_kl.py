@@ -110,3 +110,9 @@ def test_kl_rejects_bad_arguments():
     with pytest.raises(dsa.DSAError):  # workspace too small
         dsa.indexer_kl_forward(q, kI, w, Q, K, cfg.scale, 1.0,
                                workspace=torch.empty(256, dtype=torch.uint8, device="cuda"))
+    cfg2, inp2 = _inputs(CASES[0])
+    q2, k2, w2 = dev(inp2["q_I"]), dev(inp2["k_I"]), dev(inp2["w"])
+    G2 = torch.zeros((cfg2.L, cfg2.L), dtype=torch.float32, device="cuda")
+    with pytest.raises(dsa.DSAError):  # backward workspace too small (8 head groups here)
+        dsa.indexer_kl_backward(q2, k2, w2, G2,
+                                workspace=torch.empty(256, dtype=torch.uint8, device="cuda"))
