@@ -18,6 +18,7 @@
 #include "index_topk.cuh"
 #include "sparse_attn.cuh"
 #include "indexer_kl.cuh"
+#include "indexer_kl_tc.cuh"
 
 namespace {
 
@@ -692,7 +693,16 @@ dsa_status_t launch_kl_backward(const char* fn, const dsa::kl::Params& p, cudaSt
                                   smem_dq));
     CUDA_TRY(cudaFuncSetAttribute(dk_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem_dk));
-    dq_kernel<DI><<<dim3(p.HI, p.ntiles), kThreads, smem_dq, st>>>(p);
+    if (DI == dsa::kltc::kDI) {  // tcgen05: S in e4m3, dq in bf16, both in TMEM
+        CUDA_TRY(cudaFuncSetAttribute(dsa::kltc::dq_tc_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      dsa::kltc::kSmemBytes));
+        dsa::kltc::dq_tc_kernel<<<dim3(p.HI, (unsigned)((p.L + dsa::kltc::kRows - 1) /
+                                                         dsa::kltc::kRows)),
+                                  dsa::kltc::kThreads, dsa::kltc::kSmemBytes, st>>>(p);
+    } else {
+        dq_kernel<DI><<<dim3(p.HI, p.ntiles), kThreads, smem_dq, st>>>(p);
+    }
     dk_kernel<DI><<<dim3(p.nsplit, p.ntiles), kThreads, smem_dk, st>>>(p);
     if (p.nsplit > 1)
         dk_reduce_kernel<<<(unsigned)((p.L * DI / 4 + 255) / 256), 256, 0, st>>>(p, DI);

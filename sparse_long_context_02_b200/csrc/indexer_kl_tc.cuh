@@ -1,0 +1,386 @@
+// Indexer warm-up loss, backward into the query side on the 5th-generation
+// tensor cores: dq_I and dw for one indexer head and 128 query rows.
+//
+// Formulas (Kwai Keye-VL-2.0 technical-report summary, section 1, dense
+// warm-up; the reading is stated in indexer_kl.cuh):
+//   S[t,s]     = q_I[t,j] . k_I[s]                       (exact in fp32)
+//   dS[t,s]    = G[t,s] w[t,j] [S[t,s] > 0]   (s <= t)
+//   dq_I[t,j]  = sum_s dS[t,s] k_I[s],  dw[t,j] = sum_s G[t,s] relu(S[t,s])
+//
+// Per CTA and 128-key tile:
+//   1. eight worker warps copy the key rows from global memory into two
+//      shared tiles: e4m3 K-major (128-byte swizzle, the operand of S) and
+//      bf16 MN-major (128-byte swizzle, the operand of the dq product), two
+//      tiles ahead (three stages);
+//   2. one thread issues S = q . k^T (tcgen05 kind::f8f6f4, M = N = 128,
+//      K = 128) into a double-buffered TMEM accumulator;
+//   3. the workers read S rows from TMEM (thread = query row, two warps per
+//      32-row lane group, one half of the keys each), build dS in bf16 into
+//      a K-major swizzled tile and accumulate dw in fp32;
+//   4. the same thread issues dq += dS . k (kind::f16, bf16, B MN-major) into
+//      a third TMEM region, which the workers read out at the end.
+// The workers build dS of tile i before they wait for the dq product of
+// tile i - 1 (to reuse its key stage for tile i + 2), so that wait finds it
+// done; the tensor core runs S of tile i + 1 and dq of tile i meanwhile.
+// Every wait is bounded (2 s); a wait that gives up sets an abort flag, after which the
+// CTA stops issuing, waits (bounded) for its own MMAs, frees TMEM and
+// returns with DSA_DEVERR_TIMEOUT recorded.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+#include "indexer_kl.cuh"
+
+namespace dsa {
+namespace kltc {
+
+constexpr int kRows = 128;                // query rows per CTA (TMEM lanes)
+constexpr int kKeys = 128;                // keys per tile
+constexpr int kDI = 128;                  // indexer head dim (one 128-byte e4m3 row)
+constexpr int kWorkers = 8;               // worker warps
+constexpr int kMmaWarp = kWorkers;        // the warp that allocates TMEM and issues MMAs
+constexpr int kThreads = (kWorkers + 1) * 32;
+constexpr int kTmemCols = 512;            // S[2] at 0 / 128, dq at 256
+
+// Shared layout, from a 1024-byte aligned base.
+constexpr int kQ = 0;                          // e4m3 [128 rows][128 B], K-major SW128
+constexpr int kK8 = kQ + kRows * kDI;          // e4m3 k tiles [3]
+constexpr int kStages = 3;                     // key tile stages
+constexpr int kKB = kK8 + kStages * kKeys * kDI;  // bf16 k tiles [3], MN-major SW128
+constexpr int kKB_BYTES = kKeys * kDI * 2;
+constexpr int kDS = kKB + kStages * kKB_BYTES;    // bf16 dS tiles [2], K-major SW128 (two 64-key halves)
+constexpr int kDS_BYTES = kRows * kKeys * 2;
+constexpr int kMisc = kDS + 2 * kDS_BYTES;
+
+struct Misc {
+    uint64_t kready[kStages];  // workers: e4m3 + bf16 key tile (and the query tile) written
+    uint64_t sfull[2];         // MMA: S of the tile complete
+    uint64_t dsready[2];       // workers: S read, dS written
+    uint64_t kfree[kStages];   // MMA: dq product of the tile complete (its key stage and dS buffer free)
+    uint64_t done;        // MMA: every MMA complete
+    uint32_t tmem_base;
+    volatile int abort_flag;
+    float dw[kRows];      // second half's partial dw per row
+};
+constexpr int kSmemBytes = kMisc + (int)sizeof(Misc) + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory per block");
+
+// Instruction descriptors: M = N = 128, fp32 accumulator.
+//   S:  kind::f8f6f4, A and B e4m3, both K-major.
+//   dq: kind::f16, A and B bf16, A K-major, B MN-major.
+constexpr uint32_t kIdescS = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(kKeys >> 3) << 17) |
+                             ((uint32_t)(kRows >> 4) << 24);
+constexpr uint32_t kIdescDQ = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                              ((uint32_t)(kDI >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Shared-memory descriptor with 128-byte swizzle, given the leading and the
+// stride byte offsets (version 1).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= 1ull << 46;
+    d |= 2ull << 61;  // SWIZZLE_128B
+    return d;
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 bytes from global memory in one request (a whole sector); the address
+// is 32-byte aligned.
+__device__ __forceinline__ void ld_global_v8(const void* ptr, uint32_t (&v)[8]) {
+    asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                   "=r"(v[6]), "=r"(v[7])
+                 : "l"(ptr));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Byte offset of 16-byte chunk `c` of row `r` in a K-major tile of 128-byte
+// rows with the 128-byte swizzle (8-row groups of 1024 bytes).
+__device__ __forceinline__ uint32_t kmajor_off(int r, int c) {
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// Writes 64 e4m3 bytes (row `r`, bytes [64 h, 64 h + 64)) into a K-major
+// e4m3 tile, and, if kb != 0, their bf16 values into an MN-major tile whose
+// K index is the row: 8-row K groups of 2048 bytes, two 64-element MN blocks
+// of 1024 bytes each, 128-byte rows swizzled.
+__device__ __forceinline__ void put_row_half(uint32_t k8, uint32_t kb, int r, int h,
+                                             const uint4 (&v)[4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        st_shared_v4(k8 + kmajor_off(r, 4 * h + i), v[i]);
+        if (kb) {
+            const uint32_t atom = kb + (uint32_t)((r >> 3) * 2048 + h * 1024 + (r & 7) * 128);
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+            uint32_t o[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint2 b = kl::e4m3x4_to_bf16x4(w[q]);
+                o[2 * q] = b.x;
+                o[2 * q + 1] = b.y;
+            }
+            st_shared_v4(atom + ((((2 * i) ^ (r & 7))) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+            st_shared_v4(atom + ((((2 * i + 1) ^ (r & 7))) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+        }
+    }
+}
+
+// Loads 64 e4m3 bytes of a row (zeros if the row is out of range), in
+// 32-byte requests when the row is 32-byte aligned (v8), else 16-byte ones.
+__device__ __forceinline__ void get_row_half(const uint8_t* row, bool valid, int h, bool v8,
+                                             uint4 (&v)[4]) {
+    if (v8) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            uint32_t x[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (valid) ld_global_v8(row + 64 * h + 32 * i, x);
+            v[2 * i] = make_uint4(x[0], x[1], x[2], x[3]);
+            v[2 * i + 1] = make_uint4(x[4], x[5], x[6], x[7]);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            v[i] = valid ? *reinterpret_cast<const uint4*>(row + 64 * h + 16 * i)
+                         : make_uint4(0, 0, 0, 0);
+    }
+}
+
+// Grid (HI, ceil(L / 128)): the heads of one query tile run side by side;
+// the longest query tiles first.
+__global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Misc* misc = reinterpret_cast<Misc*>(smem + kMisc);
+    const uint32_t sb = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = blockIdx.x;
+    const int ntq = (int)((p.L + kRows - 1) / kRows);
+    const int qt = ntq - 1 - (int)blockIdx.y;
+    const int64_t t0 = (int64_t)qt * kRows;
+    const int nkt = qt + 1;  // key tiles 0 .. qt
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < kStages; ++b) {
+            mbar_init(smem_u32(&misc->kready[b]), kWorkers);
+            mbar_init(smem_u32(&misc->kfree[b]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&misc->sfull[b]), 1);
+            mbar_init(smem_u32(&misc->dsready[b]), kWorkers);
+        }
+        mbar_init(smem_u32(&misc->done), 1);
+        misc->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(&misc->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+
+    if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint64_t adesc_q = sdesc_sw128(sb + kQ, 16, 1024);
+            auto dq_tile = [&](int kt) {
+                const int b = kt & 1, st = kt % kStages;
+                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->dsready[b]), (kt >> 1) & 1))
+                    misc->abort_flag = 1;
+                if (misc->abort_flag) return;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kKeys / 16; ++kk) {
+                    const uint64_t a = sdesc_sw128(
+                        sb + kDS + b * kDS_BYTES + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sb + kKB + st * kKB_BYTES + kk * 4096, 1024, 2048);
+                    umma_f16(tmem + 256, a, bd, kIdescDQ, (kt > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(smem_u32(&misc->kfree[st]));
+            };
+            for (int kt = 0; kt < nkt; ++kt) {
+                const int b = kt & 1, st = kt % kStages;
+                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->kready[st]), (kt / kStages) & 1))
+                    misc->abort_flag = 1;
+                if (misc->abort_flag) break;
+                tc_fence_after();
+                const uint64_t bdesc_k = sdesc_sw128(sb + kK8 + st * (kKeys * kDI), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kDI / 32; ++kk)
+                    umma_f8f6f4(tmem + b * 128, adesc_q + (uint64_t)(2 * kk),
+                                bdesc_k + (uint64_t)(2 * kk), kIdescS, kk > 0 ? 1u : 0u);
+                umma_commit(smem_u32(&misc->sfull[b]));
+                if (kt >= 1) dq_tile(kt - 1);
+            }
+            if (!misc->abort_flag) dq_tile(nkt - 1);
+            umma_commit(smem_u32(&misc->done));
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ workers
+        const int h = warp >> 2;                       // key half of this warp
+        const int m = (warp & 3) * 32 + lane;          // TMEM lane = query row
+        const int64_t t = t0 + m;
+        const bool trow = t < p.L;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const float wj = trow ? p.w[t * p.HI + j] : 0.f;
+        // 32-byte requests where rows are 32-byte aligned
+        const bool g_vec = (p.L & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Gin) & 31) == 0;
+        const bool q_v8 = (reinterpret_cast<uintptr_t>(p.qI) & 31) == 0;
+        const bool k_v8 = (reinterpret_cast<uintptr_t>(p.kI) & 31) == 0;
+
+        // the query tile of head j, written with key tile 0
+        {
+            uint4 v[4];
+            get_row_half(p.qI + ((trow ? t : 0) * p.HI + j) * kDI, trow, h, q_v8, v);
+            put_row_half(sb + kQ, 0, m, h, v);
+        }
+        auto load_k = [&](int kt, uint4 (&v)[4]) {
+            const int64_t srow = (int64_t)kt * kKeys + m;  // this thread's key row
+            get_row_half(p.kI + (srow < p.L ? srow : 0) * kDI, srow < p.L, h, k_v8, v);
+        };
+        auto put_k = [&](int kt, const uint4 (&v)[4]) {
+            const int st = kt % kStages;
+            put_row_half(sb + kK8 + st * (kKeys * kDI), sb + kKB + st * kKB_BYTES, m, h, v);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&misc->kready[st]));
+        };
+        {
+            uint4 v[4];
+            load_k(0, v);
+            put_k(0, v);
+            if (nkt > 1) {
+                load_k(1, v);
+                put_k(1, v);
+            }
+        }
+
+        float dw_acc = 0.f;
+        for (int kt = 0; kt < nkt; ++kt) {
+            const int b = kt & 1;
+            // the key rows of tile kt + 2 and this tile's G row segment, in flight together
+            uint4 kv[4];
+            if (kt + 2 < nkt) load_k(kt + 2, kv);
+            const int64_t s0 = (int64_t)kt * kKeys + 64 * h;
+            float g[64];
+            if (trow && g_vec) {  // 32-byte requests, one whole sector each
+                const float* gp = p.Gin + t * p.L + s0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    uint32_t x[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                    if (s0 + 8 * i < p.L) ld_global_v8(gp + 8 * i, x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) g[8 * i + e] = __uint_as_float(x[e]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) g[i] = trow && s0 + i <= t ? p.Gin[t * p.L + s0 + i] : 0.f;
+            }
+            if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (kt >> 1) & 1))
+                misc->abort_flag = 1;
+            if (!misc->abort_flag) {
+                tc_fence_after();
+                float sv[64];
+                {
+                    float a[32], c[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + b * 128 + 64 * h, a);
+                    tmem_ld_32x32b_x32(tmem + lane_base + b * 128 + 64 * h + 32, c);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        sv[i] = a[i];
+                        sv[32 + i] = c[i];
+                    }
+                }
+                // dS (bf16) into the K-major tile: row m, keys [64 h, 64 h + 64); the
+                // buffer's previous tile (kt - 2) was waited for one iteration ago
+                const uint32_t ds = sb + kDS + b * kDS_BYTES + h * (kRows * 128);
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    uint32_t o[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float d2[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int i = c8 * 8 + 2 * q + e;
+                            const bool vis = s0 + i <= t;
+                            const float gv = vis ? g[i] : 0.f;
+                            dw_acc = fmaf(gv, fmaxf(sv[i], 0.f), dw_acc);
+                            d2[e] = sv[i] > 0.f ? gv * wj : 0.f;
+                        }
+                        o[q] = kl::pack_bf16(d2[0], d2[1]);
+                    }
+                    st_shared_v4(ds + kmajor_off(m, c8), make_uint4(o[0], o[1], o[2], o[3]));
+                }
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&misc->dsready[b]));
+            }
+            // The dq product of tile kt - 1 must be done before the next
+            // iteration writes its dS buffer and before tile kt + 2 takes its
+            // key stage.
+            if (kt >= 1 && kt + 1 < nkt && !misc->abort_flag &&
+                !mbar_wait(smem_u32(&misc->kfree[(kt - 1) % kStages]), ((kt - 1) / kStages) & 1))
+                misc->abort_flag = 1;
+            if (kt + 2 < nkt && !misc->abort_flag) put_k(kt + 2, kv);
+        }
+        // dq and dw
+        if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
+        tc_fence_after();
+        if (!misc->abort_flag) {
+            float a[32], c[32];
+            tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h, a);
+            tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h + 32, c);
+            if (trow) {
+                float* out = p.dq + (t * p.HI + j) * kDI + 64 * h;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    reinterpret_cast<float4*>(out)[i] =
+                        make_float4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    reinterpret_cast<float4*>(out + 32)[i] =
+                        make_float4(c[4 * i], c[4 * i + 1], c[4 * i + 2], c[4 * i + 3]);
+            }
+        }
+        if (h == 1) misc->dw[m] = dw_acc;
+        named_bar_sync(1, kWorkers * 32);
+        if (h == 0 && trow && !misc->abort_flag) p.dw[t * p.HI + j] = dw_acc + misc->dw[m];
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace kltc
+}  // namespace dsa

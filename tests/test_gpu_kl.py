@@ -39,6 +39,8 @@ CASES = [
     dict(L=700, H_I=64, d_I=128, Hq=32, Hkv=4, d=128, scale_I=1.0 / 2048, seed=41),
     # small heads
     dict(L=1000, H_I=4, d_I=64, Hq=8, Hkv=2, d=64, scale_I=1.0 / 128, seed=42),
+    # L % 8 == 0 (32-byte G row loads in the tensor-core dq kernel), ragged 128-row tail
+    dict(L=1032, H_I=64, d_I=128, Hq=32, Hkv=4, d=128, scale_I=1.0 / 2048, seed=45),
     # exactly one tile, and one row
     dict(L=64, H_I=64, d_I=128, Hq=32, Hkv=4, d=128, scale_I=1.0 / 2048, seed=43),
     dict(L=1, H_I=4, d_I=64, Hq=8, Hkv=2, d=64, scale_I=1.0 / 128, seed=44),
