@@ -703,7 +703,16 @@ dsa_status_t launch_kl_backward(const char* fn, const dsa::kl::Params& p, cudaSt
     } else {
         dq_kernel<DI><<<dim3(p.HI, p.ntiles), kThreads, smem_dq, st>>>(p);
     }
-    dk_kernel<DI><<<dim3(p.nsplit, p.ntiles), kThreads, smem_dk, st>>>(p);
+    if (DI == dsa::kltc::kDI && p.HI / p.nsplit <= dsa::kltc::kMaxHps) {
+        CUDA_TRY(cudaFuncSetAttribute(dsa::kltc::dk_tc_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      dsa::kltc::kDkSmemBytes));
+        dsa::kltc::dk_tc_kernel<<<dim3(p.nsplit, (unsigned)((p.L + dsa::kltc::kRows - 1) /
+                                                            dsa::kltc::kRows)),
+                                  dsa::kltc::kThreads, dsa::kltc::kDkSmemBytes, st>>>(p);
+    } else {
+        dk_kernel<DI><<<dim3(p.nsplit, p.ntiles), kThreads, smem_dk, st>>>(p);
+    }
     if (p.nsplit > 1)
         dk_reduce_kernel<<<(unsigned)((p.L * DI / 4 + 255) / 256), 256, 0, st>>>(p, DI);
     CUDA_TRY(cudaGetLastError());

@@ -124,14 +124,16 @@ __device__ __forceinline__ uint32_t kmajor_off(int r, int c) {
 }
 
 // Writes 64 e4m3 bytes (row `r`, bytes [64 h, 64 h + 64)) into a K-major
-// e4m3 tile, and, if kb != 0, their bf16 values into an MN-major tile whose
-// K index is the row: 8-row K groups of 2048 bytes, two 64-element MN blocks
-// of 1024 bytes each, 128-byte rows swizzled.
+// e4m3 tile (with_e4m3), and, if kb != 0, their bf16 values into a tile of
+// 8-row groups of 2048 bytes, each two 1024-byte atoms of 64 elements per
+// row (128-byte rows, 128-byte swizzle).  That bf16 tile is an MN-major
+// operand whose K index is the row (LBO 1024, SBO 2048) and also a K-major
+// operand whose M/N index is the row (SBO 2048, K steps inside the atom).
 __device__ __forceinline__ void put_row_half(uint32_t k8, uint32_t kb, int r, int h,
-                                             const uint4 (&v)[4]) {
+                                             const uint4 (&v)[4], bool with_e4m3 = true) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        st_shared_v4(k8 + kmajor_off(r, 4 * h + i), v[i]);
+        if (with_e4m3) st_shared_v4(k8 + kmajor_off(r, 4 * h + i), v[i]);
         if (kb) {
             const uint32_t atom = kb + (uint32_t)((r >> 3) * 2048 + h * 1024 + (r & 7) * 128);
             const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
@@ -373,6 +375,240 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) 
         if (h == 1) misc->dw[m] = dw_acc;
         named_bar_sync(1, kWorkers * 32);
         if (h == 0 && trow && !misc->abort_flag) p.dw[t * p.HI + j] = dw_acc + misc->dw[m];
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- dk
+
+// dk_I for 128 keys over the query tiles at or after theirs and a group of
+// heads, keys on the TMEM lanes:
+//   S^T[s,t]  = k_I[s] . q_I[t,j]            (tcgen05 kind::f16, bf16)
+//   dS^T[s,t] = G[t,s] w[t,j] [S > 0]       (t >= s)
+//   dk[s]    += sum_t dS^T[s,t] q_I[t,j]     (kind::f16, B MN-major)
+// G^T of a query tile is read once (32 consecutive keys per token and
+// request) and serves every head of the group; w of the tile is staged in
+// shared memory.  Each query tile and head is one unit; the units' q tiles
+// go through three stages, as the key tiles of dq_tc_kernel.
+constexpr int kMaxHps = 32;                        // heads per group
+constexpr int kDkKB = 0;                           // bf16 k tile (A of S^T)
+constexpr int kDkQB = kDkKB + kKB_BYTES;           // bf16 q tiles [3]
+constexpr int kDkDS = kDkQB + kStages * kKB_BYTES; // bf16 dS^T tiles [2]
+constexpr int kDkW = kDkDS + 2 * kDS_BYTES;        // w^T of the query tile [2][hps][128]
+constexpr int kDkMisc = kDkW + 2 * kMaxHps * kRows * 4;
+constexpr int kDkSmemBytes = kDkMisc + (int)sizeof(Misc) + 1024;
+static_assert(kDkSmemBytes <= 232448, "shared memory per block");
+
+constexpr uint32_t kIdescSt = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kRows >> 3) << 17) |
+                              ((uint32_t)(kRows >> 4) << 24);
+
+// Grid (nsplit, ceil(L / 128)): the groups of one key tile side by side; the
+// longest key tiles (the first) first.
+__global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Misc* misc = reinterpret_cast<Misc*>(smem + kDkMisc);
+    const uint32_t sb = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int split = blockIdx.x;
+    const int hps = p.HI / p.nsplit, j0 = split * hps;
+    const int ntq = (int)((p.L + kRows - 1) / kRows);
+    const int kt = (int)blockIdx.y;
+    const int64_t s_base = (int64_t)kt * kRows;
+    const int nunits = (ntq - kt) * hps;  // (query tile, head) pairs
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < kStages; ++b) {
+            mbar_init(smem_u32(&misc->kready[b]), kWorkers);
+            mbar_init(smem_u32(&misc->kfree[b]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&misc->sfull[b]), 1);
+            mbar_init(smem_u32(&misc->dsready[b]), kWorkers);
+        }
+        mbar_init(smem_u32(&misc->done), 1);
+        misc->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(&misc->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+
+    if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            auto dk_unit = [&](int u) {
+                const int b = u & 1, st = u % kStages;
+                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->dsready[b]), (u >> 1) & 1))
+                    misc->abort_flag = 1;
+                if (misc->abort_flag) return;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kRows / 16; ++kk) {
+                    const uint64_t a = sdesc_sw128(
+                        sb + kDkDS + b * kDS_BYTES + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sb + kDkQB + st * kKB_BYTES + kk * 4096, 1024, 2048);
+                    umma_f16(tmem + 256, a, bd, kIdescDQ, (u > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(smem_u32(&misc->kfree[st]));
+            };
+            for (int u = 0; u < nunits; ++u) {
+                const int b = u & 1, st = u % kStages;
+                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->kready[st]), (u / kStages) & 1))
+                    misc->abort_flag = 1;
+                if (misc->abort_flag) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kDI / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 32;
+                    umma_f16(tmem + b * 128, sdesc_sw128(sb + kDkKB + off, 16, 2048),
+                             sdesc_sw128(sb + kDkQB + st * kKB_BYTES + off, 16, 2048), kIdescSt,
+                             kk > 0 ? 1u : 0u);
+                }
+                umma_commit(smem_u32(&misc->sfull[b]));
+                if (u >= 1) dk_unit(u - 1);
+            }
+            if (!misc->abort_flag && nunits > 0) dk_unit(nunits - 1);
+            umma_commit(smem_u32(&misc->done));
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ workers
+        const int h = warp >> 2;                  // token half of this warp
+        const int m = (warp & 3) * 32 + lane;     // TMEM lane = key row
+        const int64_t s = s_base + m;
+        const bool srow = s < p.L;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const bool q_v8 = (reinterpret_cast<uintptr_t>(p.qI) & 31) == 0;
+        const bool k_v8 = (reinterpret_cast<uintptr_t>(p.kI) & 31) == 0;
+        const int64_t qstride = (int64_t)p.HI * kDI;
+        float* wS = reinterpret_cast<float*>(smem + kDkW);
+
+        // the key tile in bf16, written with unit 0
+        {
+            uint4 v[4];
+            get_row_half(p.kI + (srow ? s : 0) * kDI, srow, h, k_v8, v);
+            put_row_half(0, sb + kDkKB, m, h, v, false);
+        }
+        auto load_q = [&](int u, uint4 (&v)[4]) {
+            const int64_t t = s_base + (int64_t)(u / hps) * kRows + m;  // this thread's token row
+            const int jj = j0 + u % hps;
+            get_row_half(p.qI + (t < p.L ? t : 0) * qstride + jj * kDI, t < p.L, h, q_v8, v);
+        };
+        auto put_q = [&](int u, const uint4 (&v)[4]) {
+            const int st = u % kStages;
+            put_row_half(0, sb + kDkQB + st * kKB_BYTES, m, h, v, false);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&misc->kready[st]));
+        };
+        {
+            uint4 v[4];
+            if (nunits > 0) {
+                load_q(0, v);
+                put_q(0, v);
+            }
+            if (nunits > 1) {
+                load_q(1, v);
+                put_q(1, v);
+            }
+        }
+
+        float gT[64];
+        for (int u = 0; u < nunits; ++u) {
+            const int b = u & 1, jj = u % hps, qi = u / hps;
+            const int64_t tq = s_base + (int64_t)qi * kRows;  // first token of the query tile
+            uint4 qv[4];
+            if (u + 2 < nunits) load_q(u + 2, qv);
+            if (jj == 0) {
+                // G^T of this query tile (token half h), and its w^T
+                const int64_t t0h = tq + 64 * h;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const int64_t t = t0h + i;
+                    gT[i] = srow && t < p.L && t >= s ? p.Gin[t * p.L + s] : 0.f;
+                }
+                float* wb = wS + (qi & 1) * (kMaxHps * kRows);
+                for (int i = threadIdx.x; i < hps * kRows; i += kWorkers * 32) {
+                    const int hh = i / kRows, tt = i % kRows;
+                    wb[hh * kRows + tt] = tq + tt < p.L ? p.w[(tq + tt) * p.HI + j0 + hh] : 0.f;
+                }
+                named_bar_sync(1, kWorkers * 32);
+            }
+            if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (u >> 1) & 1))
+                misc->abort_flag = 1;
+            if (!misc->abort_flag) {
+                tc_fence_after();
+                float sv[64];
+                {
+                    float a[32], c[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + b * 128 + 64 * h, a);
+                    tmem_ld_32x32b_x32(tmem + lane_base + b * 128 + 64 * h + 32, c);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        sv[i] = a[i];
+                        sv[32 + i] = c[i];
+                    }
+                }
+                const float4* wr =
+                    reinterpret_cast<const float4*>(wS + (qi & 1) * (kMaxHps * kRows) + jj * kRows + 64 * h);
+                const uint32_t ds = sb + kDkDS + b * kDS_BYTES + h * (kRows * 128);
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const float4 w0 = wr[2 * c8], w1 = wr[2 * c8 + 1];
+                    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float d2[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int i = c8 * 8 + 2 * q + e;
+                            d2[e] = sv[i] > 0.f ? gT[i] * wv[2 * q + e] : 0.f;
+                        }
+                        o[q] = kl::pack_bf16(d2[0], d2[1]);
+                    }
+                    st_shared_v4(ds + kmajor_off(m, c8), make_uint4(o[0], o[1], o[2], o[3]));
+                }
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&misc->dsready[b]));
+            }
+            if (u >= 1 && u + 1 < nunits && !misc->abort_flag &&
+                !mbar_wait(smem_u32(&misc->kfree[(u - 1) % kStages]), ((u - 1) / kStages) & 1))
+                misc->abort_flag = 1;
+            if (u + 2 < nunits && !misc->abort_flag) put_q(u + 2, qv);
+        }
+        if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
+        tc_fence_after();
+        if (!misc->abort_flag) {  // (the TMEM loads are warp-collective: every lane)
+            float a[32], c[32];
+            tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h, a);
+            tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h + 32, c);
+            if (srow) {
+                float* dk = p.nsplit > 1 ? p.dk_part + (int64_t)split * p.L * kDI : p.dk;
+                float* out = dk + s * kDI + 64 * h;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    reinterpret_cast<float4*>(out)[i] =
+                        make_float4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    reinterpret_cast<float4*>(out + 32)[i] =
+                        make_float4(c[4 * i], c[4 * i + 1], c[4 * i + 2], c[4 * i + 3]);
+            }
+        }
     }
     tc_fence_before();
     __syncthreads();
