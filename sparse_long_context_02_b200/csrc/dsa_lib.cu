@@ -668,17 +668,32 @@ struct KlWorkspace {
 };
 
 template <int D>
-dsa_status_t launch_kl_forward(const char* fn, const dsa::kl::Params& p, cudaStream_t st) {
+dsa_status_t launch_kl_forward(const char* fn, dsa::kl::Params p, cudaStream_t st) {
     using namespace dsa::kl;
-    const int smem_lse = 2 * BfTile<D>::BYTES;
-    const int smem_tgt = (p.Hkv + 2) * BfTile<D>::BYTES;
-    CUDA_TRY(cudaFuncSetAttribute(head_lse_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  smem_lse));
-    CUDA_TRY(cudaFuncSetAttribute(target_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  smem_tgt));
     row_lse_kernel<<<(unsigned)((p.L + 7) / 8), 256, 0, st>>>(p);
-    head_lse_kernel<D><<<dim3(p.ntiles, p.Hq), kThreads, smem_lse, st>>>(p);
-    target_kernel<D><<<dim3(p.ntiles, p.ntiles), kThreads, smem_tgt, st>>>(p);
+    if (D == dsa::kltc::kD && p.Hkv <= 4) {  // tcgen05: 128 x 128 tiles of S in TMEM
+        namespace tc = dsa::kltc;
+        const unsigned ntq = (unsigned)((p.L + tc::kRows - 1) / tc::kRows);
+        p.kl_tile_log2 = 7;
+        CUDA_TRY(cudaFuncSetAttribute(tc::head_lse_tc_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      tc::kLseSmemBytes));
+        CUDA_TRY(cudaFuncSetAttribute(tc::target_tc_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      tc::kTgtSmemBytes));
+        tc::head_lse_tc_kernel<<<dim3(p.Hq, ntq), tc::kThreads, tc::kLseSmemBytes, st>>>(p);
+        tc::target_tc_kernel<<<dim3(ntq, ntq), tc::kThreads, tc::kTgtSmemBytes, st>>>(p);
+    } else {
+        p.kl_tile_log2 = 6;
+        const int smem_lse = 2 * BfTile<D>::BYTES;
+        const int smem_tgt = (p.Hkv + 2) * BfTile<D>::BYTES;
+        CUDA_TRY(cudaFuncSetAttribute(head_lse_kernel<D>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem_lse));
+        CUDA_TRY(cudaFuncSetAttribute(target_kernel<D>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem_tgt));
+        head_lse_kernel<D><<<dim3(p.ntiles, p.Hq), kThreads, smem_lse, st>>>(p);
+        target_kernel<D><<<dim3(p.ntiles, p.ntiles), kThreads, smem_tgt, st>>>(p);
+    }
     kl_reduce_kernel<<<(unsigned)((p.L + 255) / 256), 256, 0, st>>>(p);
     CUDA_TRY(cudaGetLastError());
     return DSA_OK;

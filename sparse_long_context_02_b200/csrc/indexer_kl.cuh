@@ -59,7 +59,8 @@ struct Params {
     const float* Gin;         // [L][L]: G for the backward kernels
     float* lse_h;             // [L][Hq] log2-domain lse of each attention row
     float* lse_I;             // [L]     natural-log lse of scale_I * I[t, 0..t]
-    float* kl_part;           // [L][ntiles]
+    float* kl_part;           // [L][ntiles]: row partials of kl, one per key tile
+    int kl_tile_log2;         // key tile of the partials: 64 or 128 keys
     float* kl;                // [L]
     float* dq;                // [L][HI][DI]
     float* dk;                // [L][DI]
@@ -371,7 +372,7 @@ __global__ void kl_reduce_kernel(const Params p) {
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= p.L) return;
     float s = 0.f;
-    const int n = (int)(t / kTile) + 1;
+    const int n = (int)(t >> p.kl_tile_log2) + 1;
     for (int i = 0; i < n; ++i) s += p.kl_part[t * p.ntiles + i];
     p.kl[t] = s;
 }

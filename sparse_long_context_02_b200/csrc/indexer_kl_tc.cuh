@@ -63,7 +63,8 @@ struct Misc {
     uint64_t done;        // MMA: every MMA complete
     uint32_t tmem_base;
     volatile int abort_flag;
-    float dw[kRows];      // second half's partial dw per row
+    float dw[kRows];      // second half's partial per row (dw, kl, running max)
+    float xl[kRows];      // second half's running sum per row (head_lse_tc_kernel)
 };
 constexpr int kSmemBytes = kMisc + (int)sizeof(Misc) + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory per block");
@@ -123,50 +124,99 @@ __device__ __forceinline__ uint32_t kmajor_off(int r, int c) {
     return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
-// Writes 64 e4m3 bytes (row `r`, bytes [64 h, 64 h + 64)) into a K-major
-// e4m3 tile (with_e4m3), and, if kb != 0, their bf16 values into a tile of
-// 8-row groups of 2048 bytes, each two 1024-byte atoms of 64 elements per
-// row (128-byte rows, 128-byte swizzle).  That bf16 tile is an MN-major
-// operand whose K index is the row (LBO 1024, SBO 2048) and also a K-major
-// operand whose M/N index is the row (SBO 2048, K steps inside the atom).
-__device__ __forceinline__ void put_row_half(uint32_t k8, uint32_t kb, int r, int h,
-                                             const uint4 (&v)[4], bool with_e4m3 = true) {
+
+// ------------------------------------------------------------ cooperative tile loads
+// The 256 worker threads fill a 128-row operand tile in 32-byte pieces
+// assigned so that one warp request covers whole rows (8 cache lines rather
+// than one line per thread): the tile goes to shared memory for the tensor
+// core, so which thread moves which piece does not matter.
+constexpr int kWorkerThreads = kWorkers * 32;
+
+struct F8Pieces {  // e4m3 tile of 128 rows x 128 bytes: 2 pieces per thread
+    uint32_t x[2][8];
+};
+struct BfPieces {  // bf16 tile of 128 rows x 128 elements: 4 pieces per thread
+    uint32_t x[4][8];
+};
+
+__device__ __forceinline__ void ld_piece(const uint8_t* src, bool v8, uint32_t (&x)[8]) {
+    if (v8) {
+        ld_global_v8(src, x);
+    } else {
+        const uint4 a = *reinterpret_cast<const uint4*>(src);
+        const uint4 b = *reinterpret_cast<const uint4*>(src + 16);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+}
+
+// Rows r at row0 + r * stride bytes; rows >= nvalid are zeros.
+__device__ __forceinline__ void load_f8_tile(F8Pieces& P, const uint8_t* row0, int64_t nvalid,
+                                             int64_t stride, bool v8, int tid) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if (with_e4m3) st_shared_v4(k8 + kmajor_off(r, 4 * h + i), v[i]);
-        if (kb) {
-            const uint32_t atom = kb + (uint32_t)((r >> 3) * 2048 + h * 1024 + (r & 7) * 128);
-            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-            uint32_t o[8];
+    for (int i = 0; i < 2; ++i) {
+        const int pc = i * kWorkerThreads + tid, r = pc >> 2, c4 = pc & 3;
+        if (r < nvalid) {
+            ld_piece(row0 + r * stride + 32 * c4, v8, P.x[i]);
+        } else {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint2 b = kl::e4m3x4_to_bf16x4(w[q]);
-                o[2 * q] = b.x;
-                o[2 * q + 1] = b.y;
-            }
-            st_shared_v4(atom + ((((2 * i) ^ (r & 7))) << 4), make_uint4(o[0], o[1], o[2], o[3]));
-            st_shared_v4(atom + ((((2 * i + 1) ^ (r & 7))) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+            for (int e = 0; e < 8; ++e) P.x[i][e] = 0u;
         }
     }
 }
 
-// Loads 64 e4m3 bytes of a row (zeros if the row is out of range), in
-// 32-byte requests when the row is 32-byte aligned (v8), else 16-byte ones.
-__device__ __forceinline__ void get_row_half(const uint8_t* row, bool valid, int h, bool v8,
-                                             uint4 (&v)[4]) {
-    if (v8) {
+// Stores the pieces into a K-major e4m3 tile (with_e4m3) and, if kb != 0,
+// their bf16 values into the 2048-byte-group tile described above.
+__device__ __forceinline__ void put_f8_tile(const F8Pieces& P, uint32_t k8, bool with_e4m3,
+                                            uint32_t kb, int tid) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            uint32_t x[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (valid) ld_global_v8(row + 64 * h + 32 * i, x);
-            v[2 * i] = make_uint4(x[0], x[1], x[2], x[3]);
-            v[2 * i + 1] = make_uint4(x[4], x[5], x[6], x[7]);
+    for (int i = 0; i < 2; ++i) {
+        const int pc = i * kWorkerThreads + tid, r = pc >> 2, c4 = pc & 3;
+        const uint32_t(&x)[8] = P.x[i];
+        if (with_e4m3) {
+            st_shared_v4(k8 + kmajor_off(r, 2 * c4), make_uint4(x[0], x[1], x[2], x[3]));
+            st_shared_v4(k8 + kmajor_off(r, 2 * c4 + 1), make_uint4(x[4], x[5], x[6], x[7]));
         }
-    } else {
+        if (kb) {
+            uint32_t o[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            v[i] = valid ? *reinterpret_cast<const uint4*>(row + 64 * h + 16 * i)
-                         : make_uint4(0, 0, 0, 0);
+            for (int q = 0; q < 8; ++q) {
+                const uint2 b = kl::e4m3x4_to_bf16x4(x[q]);
+                o[2 * q] = b.x;
+                o[2 * q + 1] = b.y;
+            }
+            const uint32_t atom = kb + (uint32_t)((r >> 3) * 2048 + (c4 >> 1) * 1024 + (r & 7) * 128);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+                st_shared_v4(atom + ((((c4 & 1) * 4 + qq) ^ (r & 7)) << 4),
+                             make_uint4(o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]));
+        }
+    }
+}
+
+// bf16 rows r at row0 + r * stride elements; rows >= nvalid are zeros.
+__device__ __forceinline__ void load_bf_tile(BfPieces& P, const __nv_bfloat16* row0, int64_t nvalid,
+                                             int64_t stride, bool v8, int tid) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int pc = i * kWorkerThreads + tid, r = pc >> 3, c8 = pc & 7;
+        if (r < nvalid) {
+            ld_piece(reinterpret_cast<const uint8_t*>(row0 + r * stride) + 32 * c8, v8, P.x[i]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) P.x[i][e] = 0u;
+        }
+    }
+}
+
+__device__ __forceinline__ void put_bf_tile(const BfPieces& P, uint32_t tile, int tid) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int pc = i * kWorkerThreads + tid, r = pc >> 3, c8 = pc & 7;
+        const uint32_t(&x)[8] = P.x[i];
+        const uint32_t atom = tile + (uint32_t)((r >> 3) * 2048 + (c8 >> 2) * 1024 + (r & 7) * 128);
+        st_shared_v4(atom + ((((c8 & 3) * 2) ^ (r & 7)) << 4), make_uint4(x[0], x[1], x[2], x[3]));
+        st_shared_v4(atom + ((((c8 & 3) * 2 + 1) ^ (r & 7)) << 4), make_uint4(x[4], x[5], x[6], x[7]));
     }
 }
 
@@ -256,30 +306,31 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) 
         const bool q_v8 = (reinterpret_cast<uintptr_t>(p.qI) & 31) == 0;
         const bool k_v8 = (reinterpret_cast<uintptr_t>(p.kI) & 31) == 0;
 
+        const int tid = threadIdx.x;
         // the query tile of head j, written with key tile 0
         {
-            uint4 v[4];
-            get_row_half(p.qI + ((trow ? t : 0) * p.HI + j) * kDI, trow, h, q_v8, v);
-            put_row_half(sb + kQ, 0, m, h, v);
+            F8Pieces P;
+            load_f8_tile(P, p.qI + (t0 * p.HI + j) * kDI, p.L - t0, (int64_t)p.HI * kDI, q_v8, tid);
+            put_f8_tile(P, sb + kQ, true, 0, tid);
         }
-        auto load_k = [&](int kt, uint4 (&v)[4]) {
-            const int64_t srow = (int64_t)kt * kKeys + m;  // this thread's key row
-            get_row_half(p.kI + (srow < p.L ? srow : 0) * kDI, srow < p.L, h, k_v8, v);
+        auto load_k = [&](int kt, F8Pieces& P) {
+            const int64_t s0k = (int64_t)kt * kKeys;
+            load_f8_tile(P, p.kI + s0k * kDI, p.L - s0k, kDI, k_v8, tid);
         };
-        auto put_k = [&](int kt, const uint4 (&v)[4]) {
+        auto put_k = [&](int kt, const F8Pieces& P) {
             const int st = kt % kStages;
-            put_row_half(sb + kK8 + st * (kKeys * kDI), sb + kKB + st * kKB_BYTES, m, h, v);
+            put_f8_tile(P, sb + kK8 + st * (kKeys * kDI), true, sb + kKB + st * kKB_BYTES, tid);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&misc->kready[st]));
         };
         {
-            uint4 v[4];
-            load_k(0, v);
-            put_k(0, v);
+            F8Pieces P;
+            load_k(0, P);
+            put_k(0, P);
             if (nkt > 1) {
-                load_k(1, v);
-                put_k(1, v);
+                load_k(1, P);
+                put_k(1, P);
             }
         }
 
@@ -287,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) 
         for (int kt = 0; kt < nkt; ++kt) {
             const int b = kt & 1;
             // the key rows of tile kt + 2 and this tile's G row segment, in flight together
-            uint4 kv[4];
+            F8Pieces kv;
             if (kt + 2 < nkt) load_k(kt + 2, kv);
             const int64_t s0 = (int64_t)kt * kKeys + 64 * h;
             float g[64];
@@ -306,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) 
             }
             if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (kt >> 1) & 1))
                 misc->abort_flag = 1;
-            if (!misc->abort_flag) {
+            if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
                 tc_fence_after();
                 float sv[64];
                 {
@@ -356,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) 
         // dq and dw
         if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
         tc_fence_after();
-        if (!misc->abort_flag) {
+        if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // the TMEM loads are warp-collective
             float a[32], c[32];
             tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h, a);
             tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h + 32, c);
@@ -494,33 +545,33 @@ __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) 
         const int64_t qstride = (int64_t)p.HI * kDI;
         float* wS = reinterpret_cast<float*>(smem + kDkW);
 
+        const int tid = threadIdx.x;
         // the key tile in bf16, written with unit 0
         {
-            uint4 v[4];
-            get_row_half(p.kI + (srow ? s : 0) * kDI, srow, h, k_v8, v);
-            put_row_half(0, sb + kDkKB, m, h, v, false);
+            F8Pieces P;
+            load_f8_tile(P, p.kI + s_base * kDI, p.L - s_base, kDI, k_v8, tid);
+            put_f8_tile(P, 0, false, sb + kDkKB, tid);
         }
-        auto load_q = [&](int u, uint4 (&v)[4]) {
-            const int64_t t = s_base + (int64_t)(u / hps) * kRows + m;  // this thread's token row
-            const int jj = j0 + u % hps;
-            get_row_half(p.qI + (t < p.L ? t : 0) * qstride + jj * kDI, t < p.L, h, q_v8, v);
+        auto load_q = [&](int u, F8Pieces& P) {
+            const int64_t tq0 = s_base + (int64_t)(u / hps) * kRows;  // first token of the unit
+            load_f8_tile(P, p.qI + tq0 * qstride + (j0 + u % hps) * kDI, p.L - tq0, qstride, q_v8, tid);
         };
-        auto put_q = [&](int u, const uint4 (&v)[4]) {
+        auto put_q = [&](int u, const F8Pieces& P) {
             const int st = u % kStages;
-            put_row_half(0, sb + kDkQB + st * kKB_BYTES, m, h, v, false);
+            put_f8_tile(P, 0, false, sb + kDkQB + st * kKB_BYTES, tid);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&misc->kready[st]));
         };
         {
-            uint4 v[4];
+            F8Pieces P;
             if (nunits > 0) {
-                load_q(0, v);
-                put_q(0, v);
+                load_q(0, P);
+                put_q(0, P);
             }
             if (nunits > 1) {
-                load_q(1, v);
-                put_q(1, v);
+                load_q(1, P);
+                put_q(1, P);
             }
         }
 
@@ -528,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) 
         for (int u = 0; u < nunits; ++u) {
             const int b = u & 1, jj = u % hps, qi = u / hps;
             const int64_t tq = s_base + (int64_t)qi * kRows;  // first token of the query tile
-            uint4 qv[4];
+            F8Pieces qv;
             if (u + 2 < nunits) load_q(u + 2, qv);
             if (jj == 0) {
                 // G^T of this query tile (token half h), and its w^T
@@ -547,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) 
             }
             if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (u >> 1) & 1))
                 misc->abort_flag = 1;
-            if (!misc->abort_flag) {
+            if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
                 tc_fence_after();
                 float sv[64];
                 {
@@ -592,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) 
         }
         if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
         tc_fence_after();
-        if (!misc->abort_flag) {  // (the TMEM loads are warp-collective: every lane)
+        if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // the TMEM loads are warp-collective
             float a[32], c[32];
             tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h, a);
             tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h + 32, c);
@@ -615,6 +666,375 @@ __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) 
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- forward
+
+// S (128 x 128) = A . B^T over D = 128 from two bf16 tiles of that layout.
+__device__ __forceinline__ void mma_bf16_tile(uint32_t d_tmem, uint32_t a_tile, uint32_t b_tile) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 32;
+        umma_f16(d_tmem, sdesc_sw128(a_tile + off, 16, 2048), sdesc_sw128(b_tile + off, 16, 2048),
+                 kIdescSt, kk > 0 ? 1u : 0u);
+    }
+}
+
+// 64 columns of a TMEM accumulator row (two 32-column loads).
+__device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&v)[64]) {
+    float a[32], c[32];
+    tmem_ld_32x32b_x32(taddr, a);
+    tmem_ld_32x32b_x32(taddr + 32, c);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        v[i] = a[i];
+        v[32 + i] = c[i];
+    }
+}
+
+constexpr int kFwdQ = 0;                            // bf16 tile of the fixed operand
+constexpr int kFwdS = kFwdQ + kKB_BYTES;            // bf16 streamed tiles [3]
+constexpr int kFwdMisc = kFwdS + kStages * kKB_BYTES;
+constexpr int kLseSmemBytes = kFwdMisc + (int)sizeof(Misc) + 1024;
+constexpr int kD = 128;                             // attention head dim of these kernels
+
+// lse_h[t][h] (log2 domain) of scale * Q[t,h] . K[s,g] over s <= t, for 128
+// query rows and one head: S tiles of 128 keys in double-buffered TMEM; each
+// worker keeps an online max and sum over its half of the keys.  Grid (Hq,
+// ceil(L / 128)): the heads of a query tile side by side, longest first.
+__global__ void __launch_bounds__(kThreads, 1) head_lse_tc_kernel(const kl::Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Misc* misc = reinterpret_cast<Misc*>(smem + kFwdMisc);
+    const uint32_t sb = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hq = blockIdx.x, g = hq / (p.Hq / p.Hkv);
+    const int ntq = (int)((p.L + kRows - 1) / kRows);
+    const int qt = ntq - 1 - (int)blockIdx.y;
+    const int64_t t0 = (int64_t)qt * kRows;
+    const int nkt = qt + 1;
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < kStages; ++b) {
+            mbar_init(smem_u32(&misc->kready[b]), kWorkers);
+            mbar_init(smem_u32(&misc->kfree[b]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&misc->sfull[b]), 1);
+            mbar_init(smem_u32(&misc->dsready[b]), kWorkers);  // here: S buffer read
+        }
+        mbar_init(smem_u32(&misc->done), 1);
+        misc->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(&misc->tmem_base), 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+
+    if (warp == kMmaWarp) {
+        if (lane == 0) {
+            for (int kt = 0; kt < nkt; ++kt) {
+                const int b = kt & 1, st = kt % kStages;
+                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->kready[st]), (kt / kStages) & 1))
+                    misc->abort_flag = 1;
+                if (!misc->abort_flag && kt >= 2 &&
+                    !mbar_wait(smem_u32(&misc->dsready[b]), ((kt - 2) >> 1) & 1))
+                    misc->abort_flag = 1;
+                if (misc->abort_flag) break;
+                tc_fence_after();
+                mma_bf16_tile(tmem + b * 128, sb + kFwdQ, sb + kFwdS + st * kKB_BYTES);
+                umma_commit(smem_u32(&misc->sfull[b]));
+                umma_commit(smem_u32(&misc->kfree[st]));
+            }
+            umma_commit(smem_u32(&misc->done));
+        }
+        __syncwarp();
+    } else {
+        const int h = warp >> 2;
+        const int m = (warp & 3) * 32 + lane;
+        const int64_t t = t0 + m;
+        const bool trow = t < p.L;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const bool q_v8 = (reinterpret_cast<uintptr_t>(p.Q) & 31) == 0;
+        const bool k_v8 = (reinterpret_cast<uintptr_t>(p.K) & 31) == 0;
+        const int64_t kstride = (int64_t)p.Hkv * kD;
+        const int tid = threadIdx.x;
+        {
+            BfPieces P;
+            load_bf_tile(P, p.Q + (t0 * p.Hq + hq) * kD, p.L - t0, (int64_t)p.Hq * kD, q_v8, tid);
+            put_bf_tile(P, sb + kFwdQ, tid);
+        }
+        auto load_k = [&](int kt, BfPieces& P) {
+            const int64_t s0k = (int64_t)kt * kKeys;
+            load_bf_tile(P, p.K + s0k * kstride + g * kD, p.L - s0k, kstride, k_v8, tid);
+        };
+        auto put_k = [&](int kt, const BfPieces& P) {
+            const int st = kt % kStages;
+            put_bf_tile(P, sb + kFwdS + st * kKB_BYTES, tid);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&misc->kready[st]));
+        };
+        {
+            BfPieces P;
+            load_k(0, P);
+            put_k(0, P);
+            if (nkt > 1) {
+                load_k(1, P);
+                put_k(1, P);
+            }
+        }
+        float mrun = -INFINITY, lrun = 0.f;
+        for (int kt = 0; kt < nkt; ++kt) {
+            const int b = kt & 1;
+            BfPieces kv;
+            if (kt + 2 < nkt) load_k(kt + 2, kv);
+            if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (kt >> 1) & 1))
+                misc->abort_flag = 1;
+            if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
+                tc_fence_after();
+                float x[64];
+                tmem_row64(tmem + lane_base + b * 128 + 64 * h, x);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&misc->dsready[b]));
+                const int64_t s0 = (int64_t)kt * kKeys + 64 * h;
+                float mx = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    x[i] = s0 + i <= t ? x[i] * p.scale_log2 : -INFINITY;
+                    mx = fmaxf(mx, x[i]);
+                }
+                const float mn = fmaxf(mrun, mx);
+                const float mu = mn == -INFINITY ? 0.f : mn;
+                float sum = 0.f;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) sum += kl::ex2(x[i] - mu);
+                lrun = lrun * kl::ex2(mrun - mu) + sum;
+                mrun = mn;
+            }
+            if (kt >= 1 && kt + 1 < nkt && !misc->abort_flag &&
+                !mbar_wait(smem_u32(&misc->kfree[(kt - 1) % kStages]), ((kt - 1) / kStages) & 1))
+                misc->abort_flag = 1;
+            if (kt + 2 < nkt && !misc->abort_flag) put_k(kt + 2, kv);
+        }
+        // combine the two halves of each row (the second half's max may be
+        // -inf: it can hold no visible key)
+        if (h == 1) {
+            misc->dw[m] = mrun;
+            misc->xl[m] = lrun;
+        }
+        named_bar_sync(1, kWorkers * 32);
+        if (h == 0) {
+            const float mo = misc->dw[m], lo = misc->xl[m];
+            const float mt = fmaxf(mrun, mo);
+            const float mu = mt == -INFINITY ? 0.f : mt;
+            const float l = lrun * kl::ex2(mrun - mu) + lo * kl::ex2(mo - mu);
+            if (trow && !misc->abort_flag) p.lse_h[t * p.Hq + hq] = mt + kl::lg2(l);
+        }
+        if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+constexpr int kTgtK = 0;                                 // bf16 key tiles of every group [Hkv <= 4]
+constexpr int kTgtQ = kTgtK + 4 * kKB_BYTES;             // bf16 query tiles [3]
+constexpr int kTgtMisc = kTgtQ + kStages * kKB_BYTES;
+constexpr int kTgtSmemBytes = kTgtMisc + (int)sizeof(Misc) + 1024;
+static_assert(kTgtSmemBytes <= 232448, "shared memory per block");
+
+// One (query tile, key tile) of 128 x 128: p summed over every query head
+// (S of each head in double-buffered TMEM, its query tile streamed through
+// three stages, the Hkv key tiles resident), then the KL row partials and G
+// written over I.  Tiles above the diagonal only write G = 0.  Grid (ntq
+// key tiles, ntq query tiles).  Needs Hkv <= 4.
+__global__ void __launch_bounds__(kThreads, 1) target_tc_kernel(const kl::Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kt = blockIdx.x, qt = blockIdx.y;
+    const int64_t t0 = (int64_t)qt * kRows, s0 = (int64_t)kt * kKeys;
+    if (kt > qt) {
+        for (int i = threadIdx.x; i < kRows * kKeys; i += kThreads) {
+            const int64_t t = t0 + i / kKeys, s = s0 + i % kKeys;
+            if (t < p.L && s < p.L) p.G[t * p.L + s] = 0.f;
+        }
+        return;
+    }
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Misc* misc = reinterpret_cast<Misc*>(smem + kTgtMisc);
+    const uint32_t sb = smem_u32(smem);
+    const int G = p.Hq / p.Hkv;
+    const int nunits = p.Hq;
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < kStages; ++b) {
+            mbar_init(smem_u32(&misc->kready[b]), kWorkers);
+            mbar_init(smem_u32(&misc->kfree[b]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&misc->sfull[b]), 1);
+            mbar_init(smem_u32(&misc->dsready[b]), kWorkers);  // here: S buffer read
+        }
+        mbar_init(smem_u32(&misc->done), 1);
+        misc->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(&misc->tmem_base), 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+
+    if (warp == kMmaWarp) {
+        if (lane == 0) {
+            for (int u = 0; u < nunits; ++u) {
+                const int b = u & 1, st = u % kStages;
+                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->kready[st]), (u / kStages) & 1))
+                    misc->abort_flag = 1;
+                if (!misc->abort_flag && u >= 2 &&
+                    !mbar_wait(smem_u32(&misc->dsready[b]), ((u - 2) >> 1) & 1))
+                    misc->abort_flag = 1;
+                if (misc->abort_flag) break;
+                tc_fence_after();
+                mma_bf16_tile(tmem + b * 128, sb + kTgtQ + st * kKB_BYTES,
+                              sb + kTgtK + (u / G) * kKB_BYTES);
+                umma_commit(smem_u32(&misc->sfull[b]));
+                umma_commit(smem_u32(&misc->kfree[st]));
+            }
+            umma_commit(smem_u32(&misc->done));
+        }
+        __syncwarp();
+    } else {
+        const int h = warp >> 2;
+        const int m = (warp & 3) * 32 + lane;
+        const int64_t t = t0 + m;
+        const bool trow = t < p.L;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const bool q_v8 = (reinterpret_cast<uintptr_t>(p.Q) & 31) == 0;
+        const bool k_v8 = (reinterpret_cast<uintptr_t>(p.K) & 31) == 0;
+        const int64_t kstride = (int64_t)p.Hkv * kD;
+        const int tid = threadIdx.x;
+        for (int g = 0; g < p.Hkv; ++g) {
+            BfPieces P;
+            load_bf_tile(P, p.K + s0 * kstride + g * kD, p.L - s0, kstride, k_v8, tid);
+            put_bf_tile(P, sb + kTgtK + g * kKB_BYTES, tid);
+        }
+        auto load_q = [&](int u, BfPieces& P) {
+            load_bf_tile(P, p.Q + (t0 * p.Hq + u) * kD, p.L - t0, (int64_t)p.Hq * kD, q_v8, tid);
+        };
+        auto put_q = [&](int u, const BfPieces& P) {
+            const int st = u % kStages;
+            put_bf_tile(P, sb + kTgtQ + st * kKB_BYTES, tid);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&misc->kready[st]));
+        };
+        {
+            BfPieces P;
+            load_q(0, P);
+            put_q(0, P);
+            if (nunits > 1) {
+                load_q(1, P);
+                put_q(1, P);
+            }
+        }
+        const int64_t sh = s0 + 64 * h;  // first key of this thread's half
+        float P[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) P[i] = 0.f;
+        for (int u = 0; u < nunits; ++u) {
+            const int b = u & 1;
+            BfPieces qv;
+            if (u + 2 < nunits) load_q(u + 2, qv);
+            const float lse = trow ? p.lse_h[t * p.Hq + u] : 0.f;
+            if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (u >> 1) & 1))
+                misc->abort_flag = 1;
+            if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
+                tc_fence_after();
+                float x[64];
+                tmem_row64(tmem + lane_base + b * 128 + 64 * h, x);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&misc->dsready[b]));
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    if (sh + i <= t) P[i] += kl::ex2(x[i] * p.scale_log2 - lse);
+            }
+            if (u >= 1 && u + 1 < nunits && !misc->abort_flag &&
+                !mbar_wait(smem_u32(&misc->kfree[(u - 1) % kStages]), ((u - 1) / kStages) & 1))
+                misc->abort_flag = 1;
+            if (u + 2 < nunits && !misc->abort_flag) put_q(u + 2, qv);
+        }
+        // KL partial and G over this thread's 64 keys of row t
+        const float inv_h = 1.f / (float)p.Hq;
+        const float lse_I = trow ? p.lse_I[t] : 0.f;
+        float klp = 0.f;
+        const bool gv8 = (p.L & 7) == 0 && (reinterpret_cast<uintptr_t>(p.G) & 31) == 0;
+        if (trow && !misc->abort_flag) {
+            float* grow = p.G + t * p.L + sh;
+            if (gv8) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (sh + 8 * c >= p.L) continue;
+                    uint32_t x[8];
+                    ld_global_v8(grow + 8 * c, x);
+                    float o[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = 8 * c + e;
+                        float gvl = 0.f;
+                        if (sh + i <= t) {
+                            const float pv = P[i] * inv_h;
+                            const float lq = p.scale_I * __uint_as_float(x[e]) - lse_I;
+                            klp += pv > 0.f ? pv * (kl::lg2(pv) * kl::kLn2 - lq) : 0.f;
+                            gvl = p.scale_I * (kl::ex2(lq * kl::kLog2e) - pv);
+                        }
+                        o[e] = gvl;
+                    }
+                    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(grow + 8 * c),
+                                 "f"(o[0]), "f"(o[1]), "f"(o[2]), "f"(o[3]), "f"(o[4]), "f"(o[5]),
+                                 "f"(o[6]), "f"(o[7])
+                                 : "memory");
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    if (sh + i >= p.L) continue;
+                    float gvl = 0.f;
+                    if (sh + i <= t) {
+                        const float pv = P[i] * inv_h;
+                        const float lq = p.scale_I * grow[i] - lse_I;
+                        klp += pv > 0.f ? pv * (kl::lg2(pv) * kl::kLn2 - lq) : 0.f;
+                        gvl = p.scale_I * (kl::ex2(lq * kl::kLog2e) - pv);
+                    }
+                    grow[i] = gvl;
+                }
+            }
+        }
+        if (h == 1) misc->dw[m] = klp;
+        named_bar_sync(1, kWorkers * 32);
+        if (h == 0 && trow && !misc->abort_flag) p.kl_part[t * p.ntiles + kt] = klp + misc->dw[m];
+        if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
     }
 }
 
