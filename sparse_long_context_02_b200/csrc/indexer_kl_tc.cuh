@@ -681,18 +681,6 @@ __device__ __forceinline__ void mma_bf16_tile(uint32_t d_tmem, uint32_t a_tile, 
     }
 }
 
-// 64 columns of a TMEM accumulator row (two 32-column loads).
-__device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&v)[64]) {
-    float a[32], c[32];
-    tmem_ld_32x32b_x32(taddr, a);
-    tmem_ld_32x32b_x32(taddr + 32, c);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        v[i] = a[i];
-        v[32 + i] = c[i];
-    }
-}
-
 constexpr int kFwdQ = 0;                            // bf16 tile of the fixed operand
 constexpr int kFwdS = kFwdQ + kKB_BYTES;            // bf16 streamed tiles [3]
 constexpr int kFwdMisc = kFwdS + kStages * kKB_BYTES;
@@ -799,25 +787,34 @@ __global__ void __launch_bounds__(kThreads, 1) head_lse_tc_kernel(const kl::Para
                 misc->abort_flag = 1;
             if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
                 tc_fence_after();
-                float x[64];
-                tmem_row64(tmem + lane_base + b * 128 + 64 * h, x);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&misc->dsready[b]));
                 const int64_t s0 = (int64_t)kt * kKeys + 64 * h;
-                float mx = -INFINITY;
+                const bool diag = kt == qt;  // only the diagonal tile has keys past a row
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    x[i] = s0 + i <= t ? x[i] * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, x[i]);
+                for (int half = 0; half < 2; ++half) {
+                    float x[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + b * 128 + 64 * h + 32 * half, x);
+                    if (half == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&misc->dsready[b]));
+                    }
+                    if (diag) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (s0 + 32 * half + i > t) x[i] = -INFINITY;
+                    }
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, x[i]);
+                    // scale > 0: the max of the scaled values is the scaled max
+                    const float mn = fmaxf(mrun, mx * p.scale_log2);
+                    const float mu = mn == -INFINITY ? 0.f : mn;
+                    float sum = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) sum += kl::ex2(fmaf(x[i], p.scale_log2, -mu));
+                    lrun = lrun * kl::ex2(mrun - mu) + sum;
+                    mrun = mn;
                 }
-                const float mn = fmaxf(mrun, mx);
-                const float mu = mn == -INFINITY ? 0.f : mn;
-                float sum = 0.f;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) sum += kl::ex2(x[i] - mu);
-                lrun = lrun * kl::ex2(mrun - mu) + sum;
-                mrun = mn;
             }
             if (kt >= 1 && kt + 1 < nkt && !misc->abort_flag &&
                 !mbar_wait(smem_u32(&misc->kfree[(kt - 1) % kStages]), ((kt - 1) / kStages) & 1))
@@ -956,23 +953,32 @@ __global__ void __launch_bounds__(kThreads, 1) target_tc_kernel(const kl::Params
         float P[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) P[i] = 0.f;
+        // Keys past a row (diagonal tile only) accumulate too and are skipped
+        // by the epilogue.  Each head's lse is fetched one head ahead.
+        float lse_next = trow ? p.lse_h[t * p.Hq] : 0.f;
         for (int u = 0; u < nunits; ++u) {
             const int b = u & 1;
             BfPieces qv;
             if (u + 2 < nunits) load_q(u + 2, qv);
-            const float lse = trow ? p.lse_h[t * p.Hq + u] : 0.f;
+            const float lse = lse_next;
+            if (u + 1 < nunits) lse_next = trow ? p.lse_h[t * p.Hq + u + 1] : 0.f;
             if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (u >> 1) & 1))
                 misc->abort_flag = 1;
             if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
                 tc_fence_after();
-                float x[64];
-                tmem_row64(tmem + lane_base + b * 128 + 64 * h, x);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&misc->dsready[b]));
 #pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    if (sh + i <= t) P[i] += kl::ex2(x[i] * p.scale_log2 - lse);
+                for (int half = 0; half < 2; ++half) {
+                    float x[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + b * 128 + 64 * h + 32 * half, x);
+                    if (half == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&misc->dsready[b]));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        P[32 * half + i] += kl::ex2(fmaf(x[i], p.scale_log2, -lse));
+                }
             }
             if (u >= 1 && u + 1 < nunits && !misc->abort_flag &&
                 !mbar_wait(smem_u32(&misc->kfree[(u - 1) % kStages]), ((u - 1) / kStages) & 1))
