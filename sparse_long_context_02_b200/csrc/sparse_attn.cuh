@@ -147,29 +147,22 @@ attn_kernel(const Params p) {
         // ------------------------------------------------ gather producer (16-byte cp.async)
         constexpr int CPR = C::ROW / 16;  // 16-byte chunks per row
         int issued = 0;
-        // Prefill: each chunk's index entries are loaded one chunk ahead, so
-        // their latency overlaps the wait and the copies of the chunk before
-        // (the decode instantiation, with short slices, runs faster without).
+        // Each chunk's index entries are loaded one chunk ahead, so their
+        // latency overlaps the wait and the copies of the chunk before.
         auto load_idx = [&](int c) -> int32_t {
             const int e = c * kNK + lane;
             return lane < kNK && c < nchunks && e < nent ? irow[e] : -1;
         };
-        int32_t pre = SPLIT ? -1 : load_idx(0);
+        int32_t pre = load_idx(0);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
-            int32_t si;
-            if constexpr (SPLIT) {
-                si = -1;
-            } else {
-                si = pre;
-                pre = load_idx(c + 1);
-            }
+            const int32_t si = pre;
+            pre = load_idx(c + 1);
             if (c >= kStages) {
                 bool got = false;
                 if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ((c / kStages) - 1) & 1);
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
             }
-            if constexpr (SPLIT) si = load_idx(c);
             if (si >= nkeys) record_device_error(2);
             const bool valid = si >= 0 && si < nkeys;
             const uint32_t bal = __ballot_sync(0xffffffffu, valid);
