@@ -41,6 +41,11 @@ CASES = [
     dict(L=1000, H_I=4, d_I=64, Hq=8, Hkv=2, d=64, scale_I=1.0 / 128, seed=42),
     # L % 8 == 0 (32-byte G row loads in the tensor-core dq kernel), ragged 128-row tail
     dict(L=1032, H_I=64, d_I=128, Hq=32, Hkv=4, d=128, scale_I=1.0 / 2048, seed=45),
+    # Hkv = 8 (the mma.sync forward), H_I = 4 with d_I = 128 (tensor-core dq/dk,
+    # one head per dk group)
+    dict(L=300, H_I=4, d_I=128, Hq=16, Hkv=8, d=128, scale_I=1.0 / 512, seed=46),
+    # Hkv = 2 on the tensor-core forward, d_I = 64 backward
+    dict(L=450, H_I=64, d_I=64, Hq=8, Hkv=2, d=128, scale_I=1.0 / 1024, seed=47),
     # exactly one tile, and one row
     dict(L=64, H_I=64, d_I=128, Hq=32, Hkv=4, d=128, scale_I=1.0 / 2048, seed=43),
     dict(L=1, H_I=4, d_I=64, Hq=8, Hkv=2, d=64, scale_I=1.0 / 128, seed=44),
