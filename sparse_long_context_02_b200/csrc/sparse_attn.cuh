@@ -30,7 +30,9 @@ namespace dsa {
 namespace attn {
 
 constexpr int kNK = 16;      // keys per stage
-constexpr int kStages = 3;
+// Two stages: 67 KB of shared memory per CTA, so three CTAs (15 warps) fit
+// on an SM (136 registers x 160 threads x 3 also fits the register file).
+constexpr int kStages = 2;
 
 template <int D, int HKV>
 struct Cfg {
