@@ -32,6 +32,7 @@
 namespace dsa {
 namespace attn {
 
+constexpr int kDedupStages = 3;  // gather ring stages of the dedup kernel
 constexpr int kDedupQB = 6;               // query tokens per CTA (three pairs)
 constexpr int kDedupMaxKeys = 1 << 18;    // keys the bitmap covers (32 KB)
 constexpr int kDedupMaxK = 2048;          // index-row length the union buffers allow
@@ -46,13 +47,13 @@ struct DedupCfg {
     static constexpr int STAGE = 2 * kNK * STRIDE;
     static constexpr int UMAX = kDedupQB * kDedupMaxK;   // distinct keys at most
     // the stage ring, at least as large as the phase-1 bitmap that overlays it
-    static constexpr int RING = kStages * STAGE > kDedupMaxKeys / 8 ? kStages * STAGE
+    static constexpr int RING = kDedupStages * STAGE > kDedupMaxKeys / 8 ? kDedupStages * STAGE
                                                                      : kDedupMaxKeys / 8;
     static constexpr int OFF_PREFIX = RING;
     static constexpr int OFF_U = OFF_PREFIX + (kDedupMaxKeys / 32) * 4;
     static constexpr int OFF_MASK = OFF_U + UMAX * 4;
     static constexpr int OFF_BAR = OFF_MASK + UMAX;      // one mask byte per key
-    static constexpr int SMEM = OFF_BAR + 2 * kStages * 8;
+    static constexpr int SMEM = OFF_BAR + 2 * kDedupStages * 8;
     static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
 };
 
@@ -84,7 +85,7 @@ dedup_kernel(const Params p) {
     int32_t* U = reinterpret_cast<int32_t*>(smem + C::OFF_U);
     uint32_t* mask32 = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* empty = full + kStages;
+    uint64_t* empty = full + kDedupStages;
     __shared__ int s_warp[32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -96,7 +97,7 @@ dedup_kernel(const Params p) {
     // ---------------------------------------------------- phase 1: the union
     for (int i = tid; i < nwords; i += NT) bitmap[i] = 0u;
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kDedupStages; ++s) {
             mbar_init(smem_u32(&full[s]), 33);  // 32 copy-completion arrivals + lane 0
             mbar_init(smem_u32(&empty[s]), C::CWARPS);
         }
@@ -156,10 +157,10 @@ dedup_kernel(const Params p) {
         constexpr int CPR = C::ROW / 16;
         int issued = 0;
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c % kStages;
-            if (c >= kStages) {
+            const int s = c % kDedupStages;
+            if (c >= kDedupStages) {
                 bool got = false;
-                if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ((c / kStages) - 1) & 1);
+                if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ((c / kDedupStages) - 1) & 1);
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
             }
             const uint32_t sbase = smem_u32(smem + s * C::STAGE);
@@ -182,8 +183,8 @@ dedup_kernel(const Params p) {
             issued = c + 1;
         }
         if (lane == 0) {
-            for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
-                mbar_wait(smem_u32(&full[c % kStages]), (c / kStages) & 1);
+            for (int c = issued - kDedupStages < 0 ? 0 : issued - kDedupStages; c < issued; ++c)
+                mbar_wait(smem_u32(&full[c % kDedupStages]), (c / kDedupStages) & 1);
         }
         return;
     }
@@ -221,8 +222,8 @@ dedup_kernel(const Params p) {
     const int mi = lane >> 3, ri = lane & 7;
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
-        const int s = c % kStages;
-        const bool got = mbar_wait(smem_u32(&full[s]), (c / kStages) & 1);
+        const int s = c % kDedupStages;
+        const bool got = mbar_wait(smem_u32(&full[s]), (c / kDedupStages) & 1);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         const uint32_t kbase = smem_u32(smem + s * C::STAGE) + g * D * 2;
         const uint32_t vbase = kbase + kNK * C::STRIDE;
