@@ -107,6 +107,54 @@ def test_decode_rejects_bad_arguments_and_small_workspace(L):
     assert f(*bad, need, None) == INVALID
 
 
+def test_indexer_kl_rejects_bad_arguments_and_small_workspaces(L):
+    f = L.dsa_indexer_kl_forward
+    sc, sI = ctypes.c_float(0.088), ctypes.c_float(1.0 / 2048)
+    need = L.dsa_indexer_kl_workspace_size(300, 32)
+    # lse per (row, head) + lse per row + one partial per (row, 64-key tile), 256-byte aligned
+    assert need >= 300 * 32 * 4 + 300 * 4 + 300 * 5 * 4
+    ws = 0x100000  # 256-byte aligned
+    args = [FAKE] * 5 + [300, 64, 128, 32, 4, 128, sc, sI, FAKE, FAKE, ws]
+    assert f(*args, need - 1, None) == WORKSPACE
+    bad = list(args)
+    bad[15] = ws + 16  # workspace not 256-byte aligned
+    assert f(*bad, need, None) == WORKSPACE
+    bad = list(args)
+    bad[3] = None  # Q
+    assert f(*bad, need, None) == INVALID
+    bad = list(args)
+    bad[5] = 1 << 16  # L * L >= 2^31
+    assert f(*bad, need, None) == INVALID
+    bad = list(args)
+    bad[9] = 3  # Hkv does not divide Hq
+    assert f(*bad, need, None) == INVALID
+    bad = list(args)
+    bad[10] = 96  # d
+    assert f(*bad, need, None) == UNSUPPORTED
+    bad = list(args)
+    bad[12] = ctypes.c_float(0.0)  # scale_I
+    assert f(*bad, need, None) == INVALID
+    bad = list(args)
+    bad[6], bad[7] = 16, 128  # an indexer shape the scorer does not have
+    assert f(*bad, need, None) == UNSUPPORTED
+
+    g = L.dsa_indexer_kl_backward
+    nb = L.dsa_indexer_kl_backward_workspace_size(300, 64, 128)
+    assert nb >= 8 * 300 * 128 * 4  # eight head groups of dk partials
+    assert L.dsa_indexer_kl_backward_workspace_size(300, 11, 128) == 256  # one group: no partials
+    bargs = [FAKE] * 4 + [300, 64, 128, FAKE, FAKE, FAKE, ws]
+    assert g(*bargs, nb - 1, None) == WORKSPACE
+    bad = list(bargs)
+    bad[5] = 0  # H_I
+    assert g(*bad, nb, None) == INVALID
+    bad = list(bargs)
+    bad[6] = 96  # d_I
+    assert g(*bad, nb, None) == UNSUPPORTED
+    bad = list(bargs)
+    bad[3] = None  # G
+    assert g(*bad, nb, None) == INVALID
+
+
 def test_device_error_rejects_null(L):
     assert L.dsa_device_error(None, None) == INVALID
 
