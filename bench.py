@@ -43,9 +43,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--prefill-config", type=int, default=3,
+    ap.add_argument("--prefill-config", type=int, default=gen.PREFILL_128K.id,
                     help="workload id of the prefill part (0: no prefill part)")
-    ap.add_argument("--decode-config", type=int, default=4,
+    ap.add_argument("--decode-config", type=int, default=gen.DECODE_B64.id,
                     help="workload id of the decode part (0: no decode part)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="use only the first B sequences of the decode workload (profiling)")
@@ -491,7 +491,7 @@ def workload_config(pcfg, dcfg, world=1):
 
 
 def run_reference(args):
-    pcfg = gen.CONFIGS[args.prefill_config or 3]
+    pcfg = gen.CONFIGS[args.prefill_config or gen.PREFILL_128K.id]
     host = gen.prefill_inputs(pcfg)
     cores = os.cpu_count() or 1
     probe = sample_rows(pcfg.L, max(cores, 8), seed=1)
@@ -569,7 +569,7 @@ def kl_bench(args) -> dict:
     import torch
     import sparse_long_context_02_b200 as dsa
     L = args.kl
-    base = gen.CONFIGS[3]
+    base = gen.PREFILL_128K
     cfg = gen.custom(L=L, H_I=base.H_I, d_I=base.d_I, k=8, Hq=base.Hq, Hkv=base.Hkv, d=base.d,
                      seed=51)
     host = gen.prefill_inputs(cfg)

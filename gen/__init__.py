@@ -152,6 +152,13 @@ CONFIGS: Dict[int, Config] = {
               Hq=32, Hkv=4, d=128, L=262144, video=True),
 }
 
+# The workloads by name.
+TINY_PREFILL = CONFIGS[1]    # tiny prefill L=2048 k=256 (small heads)
+PREFILL_32K = CONFIGS[2]     # prefill L=32768 k=2048
+PREFILL_128K = CONFIGS[3]    # prefill L=131072 k=2048
+DECODE_B64 = CONFIGS[4]      # decode B=64, n ~ U[32768, 262144], k=2048
+VIDEO_256K = CONFIGS[5]      # video prefill L=262144 k=2048
+
 
 def custom(**kw) -> Config:
     """A small prefill (or decode) workload with the i.i.d. recipe; id 0."""

@@ -44,12 +44,12 @@ def test_iid_distributions():
 
 
 def test_workload_shapes():
-    c1 = gen.CONFIGS[1]
+    c1 = gen.TINY_PREFILL
     inp = gen.prefill_inputs(c1)
     assert inp["q_I"].shape == (2048, 4, 64) and inp["k_I"].shape == (2048, 64)
     assert inp["w"].shape == (2048, 4) and inp["Q"].shape == (2048, 8, 64)
     assert inp["K"].shape == (2048, 2, 64) and inp["V"].shape == (2048, 2, 64)
-    c4 = gen.CONFIGS[4]
+    c4 = gen.DECODE_B64
     n = gen.decode_lengths(c4)
     assert n.shape == (64,) and n.min() >= 32768 and n.max() <= 262144
     off = gen.decode_offsets(c4)
@@ -57,7 +57,7 @@ def test_workload_shapes():
 
 
 def test_video_structure():
-    c5 = gen.CONFIGS[5]
+    c5 = gen.VIDEO_256K
     assert c5.frames * (c5.frame_text + c5.frame_vision) + 64 == c5.L
     ft = c5.frame_text + c5.frame_vision
     # three frames' worth of indexer keys

@@ -41,9 +41,9 @@ def sample_rows(L, k, n=16, seed=0, extra=()):
     return np.array(sorted(set(r for r in fixed + strat + list(extra) if 0 <= r < L)), np.int64)
 
 
-@pytest.mark.parametrize("cfg_id", [2, 3, 5])
-def test_prefill_full_size(cfg_id):
-    cfg = gen.CONFIGS[cfg_id]
+@pytest.mark.parametrize("cfg", [gen.PREFILL_32K, gen.PREFILL_128K, gen.VIDEO_256K],
+                         ids=lambda c: c.name)
+def test_prefill_full_size(cfg):
     host = gen.prefill_inputs(cfg)
     idx = dsa.index_topk(dev(host["q_I"]), dev(host["k_I"]), dev(host["w"]), cfg.k)
     O = dsa.sparse_attn_prefill(dev(host["Q"], torch.bfloat16), dev(host["K"], torch.bfloat16),
@@ -55,7 +55,7 @@ def test_prefill_full_size(cfg_id):
     if cfg.video:
         ft = cfg.frame_text + cfg.frame_vision
         extra = [f * ft + o for f in (1, 117, 239) for o in (0, 15, 16, ft - 1)]
-    rows = sample_rows(cfg.L, cfg.k, seed=cfg_id, extra=extra)
+    rows = sample_rows(cfg.L, cfg.k, seed=cfg.id, extra=extra)
     ref_idx = oracle.index_topk(host["q_I"], host["k_I"], host["w"], cfg.k, rows=rows)
     got_idx = idx[torch.from_numpy(rows).cuda()].cpu().numpy()
     bad = [int(r) for r, a, b in zip(rows, got_idx, ref_idx) if not np.array_equal(a, b)]
@@ -69,7 +69,7 @@ def test_prefill_full_size(cfg_id):
 
 
 def test_decode_full_size():
-    cfg = gen.CONFIGS[4]
+    cfg = gen.DECODE_B64
     off = gen.decode_offsets(cfg)
     lens = np.diff(off)
     N = int(off[-1])

@@ -67,7 +67,7 @@ def test_index_scores_worst_case_magnitude_is_exact():
 
 
 def test_index_topk_tiny_workload_bit_exact():
-    cfg = gen.CONFIGS[1]
+    cfg = gen.TINY_PREFILL
     inp = gen.prefill_inputs(cfg)
     ref = oracle.index_topk(inp["q_I"], inp["k_I"], inp["w"], cfg.k)
     got = dsa.index_topk(dev(inp["q_I"]), dev(inp["k_I"]), dev(inp["w"]), cfg.k).cpu().numpy()
@@ -117,7 +117,7 @@ def test_index_topk_is_deterministic():
 # ------------------------------------------------------------------ attention
 
 def test_attention_tiny_workload():
-    cfg = gen.CONFIGS[1]
+    cfg = gen.TINY_PREFILL
     inp = gen.prefill_inputs(cfg)
     idx = oracle.index_topk(inp["q_I"], inp["k_I"], inp["w"], cfg.k)
     ref = oracle.sparse_attn(inp["Q"], inp["K"], inp["V"], idx, cfg.scale)
@@ -169,7 +169,7 @@ def test_attention_empty_rows_are_zero_and_out_of_range_is_flagged():
 
 
 def test_prefill_end_to_end_tiny_workload():
-    cfg = gen.CONFIGS[1]
+    cfg = gen.TINY_PREFILL
     inp = gen.prefill_inputs(cfg)
     idx = dsa.index_topk(dev(inp["q_I"]), dev(inp["k_I"]), dev(inp["w"]), cfg.k)
     O = dsa.sparse_attn_prefill(dev(inp["Q"], torch.bfloat16), dev(inp["K"], torch.bfloat16),

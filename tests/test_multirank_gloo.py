@@ -23,7 +23,7 @@ def _worker(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     tdist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        p, d = bench.rank_workloads(gen.CONFIGS[3], gen.CONFIGS[4], rank, world)
+        p, d = bench.rank_workloads(gen.PREFILL_128K, gen.DECODE_B64, rank, world)
         # each rank draws its own inputs: first indexer-key bytes differ
         first = gen.prefill_kI(p, 0, 4).tobytes()
         times = bench.max_over_ranks([10.0 + rank, 5.0 - rank], world)
@@ -48,6 +48,6 @@ def test_two_ranks_gloo():
 
 def test_single_rank_is_identity():
     import bench
-    p, d = bench.rank_workloads(gen.CONFIGS[3], gen.CONFIGS[4], 0, 1)
-    assert p is gen.CONFIGS[3] and d is gen.CONFIGS[4]
+    p, d = bench.rank_workloads(gen.PREFILL_128K, gen.DECODE_B64, 0, 1)
+    assert p is gen.PREFILL_128K and d is gen.DECODE_B64
     assert np.array_equal(bench.max_over_ranks([1.0, 2.0], 1), [1.0, 2.0])

@@ -249,7 +249,7 @@ def test_sparse_with_k_at_least_t_plus_1_is_dense_causal():
 
 def test_sparse_rows_below_k_are_dense_causal_at_workload_shape():
     # rows t < k of the tiny prefill workload select every visible key
-    cfg = gen.CONFIGS[1].with_(L=300)
+    cfg = gen.TINY_PREFILL.with_(L=300)
     inp = gen.prefill_inputs(cfg)
     rows = np.array([0, 1, 17, 128, 255], np.int64)
     idx = oracle.index_topk(inp["q_I"], inp["k_I"], inp["w"], cfg.k, rows=rows)
