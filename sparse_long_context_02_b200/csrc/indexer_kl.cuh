@@ -14,7 +14,7 @@
 //   dw[t,j] = sum_s G relu(S),  dq_I[t,j] = w[t,j] sum_s G [S > 0] k_I[s],
 //   dk_I[s] = sum_t sum_j G w[t,j] [S > 0] q_I[t,j],   S = q_I[t,j] . k_I[s].
 //
-// Kernels (all tiles are 64 query rows x 64 keys; four warps of 16 rows):
+// Kernels here (tiles of 64 query rows x 64 keys; four warps of 16 rows):
 //   row_lse_kernel     lse of scale_I * I per row (I from the tcgen05 scorer)
 //   head_lse_kernel    lse of every query head's causal attention row
 //   target_kernel      p, the row KL partials and G, written over I in place
@@ -23,8 +23,11 @@
 //   dk_kernel          dk_I for 64 keys, over all later query rows and a group
 //                      of heads (one partial per group)
 //   dk_reduce_kernel   dk_I = sum of the groups' partials, in a fixed order
-// The score products run on the tensor cores (bf16 m16n8k16 for the
-// attention, e4m3 m16n8k32 for the indexer); dS is rounded to bf16 for the
+// Their products use mma.sync (bf16 m16n8k16 for the attention, e4m3
+// m16n8k32 for the indexer).  The 5th-generation tensor-core versions of
+// head_lse, target, dq and dk (indexer_kl_tc.cuh, 128 x 128 tiles, TMEM
+// accumulators) run for d = 128 with Hkv <= 4 (forward) and d_I = 128
+// (backward); these serve the other shapes.  dS is rounded to bf16 for the
 // dq/dk products, as a flash-attention backward does.  Every result is
 // written by exactly one thread, in a fixed order: runs are bit-identical.
 #pragma once
