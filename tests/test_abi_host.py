@@ -164,3 +164,40 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(dsa, "LIB_PATH", "/nonexistent/libdsa_b200.so")
     with pytest.raises(RuntimeError, match="missing"):
         dsa.lib()
+
+
+def test_binding_rejects_host_and_malformed_tensors(L):
+    import torch
+    q = torch.zeros((64, 4, 64), dtype=torch.uint8)
+    k = torch.zeros((64, 64), dtype=torch.uint8)
+    w = torch.zeros((64, 4), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        dsa.index_topk(q, k, w, 8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        dsa.index_scores(q, k, w)
+    Q = torch.zeros((64, 8, 64), dtype=torch.bfloat16)
+    K = torch.zeros((64, 2, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        dsa.indexer_kl_forward(q, k, w, Q, K, 0.125, 1.0,
+                               kl=torch.zeros(64), G=torch.zeros((64, 64)),
+                               workspace=torch.zeros(1 << 20, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        dsa.indexer_kl_backward(q, k, w, torch.zeros((64, 64)),
+                                dq_I=torch.zeros((64, 4, 64)), dk_I=torch.zeros((64, 64)),
+                                dw=torch.zeros((64, 4)),
+                                workspace=torch.zeros(256, dtype=torch.uint8))
+
+
+def test_binding_checks_layout_before_the_call():
+    import torch
+    # a tensor that claims to live on the GPU, to reach the layout checks on a host
+    class FakeCuda(torch.Tensor):
+        @property
+        def is_cuda(self):
+            return True
+    t = torch.zeros((8, 8), dtype=torch.float32).as_subclass(FakeCuda)
+    with pytest.raises(ValueError, match="contiguous"):
+        dsa._dev(t.t(), "x")
+    with pytest.raises(ValueError, match="4-byte elements"):
+        dsa._dev(torch.zeros(8, dtype=torch.float64).as_subclass(FakeCuda), "w", 4)
+    assert dsa._dev(t, "x", 4) == t.data_ptr()
