@@ -19,7 +19,7 @@
  *   dense row-major array with the layout given.  The caller owns all
  *   memory; the library never allocates device memory.
  * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
- *   default stream) and do not synchronize, except dsa_device_error.
+ *   default stream) and do not synchronize, except dsa_check_device_error.
  * - Arguments are validated on the host before anything is launched; a
  *   failing call returns a status, launches nothing and leaves a message in
  *   dsa_last_error().  No C++ exception crosses this boundary.
@@ -31,9 +31,17 @@
  *   indexer values in [-8, 8] with d_I <= 128 and weights in {0..3}.
  * - Index rows list the selected keys in ascending order, then -1 padding.
  *   The result is deterministic: the same inputs give the same bits.
- * - A kernel that detects an error (a bounded wait that timed out, an index
- *   out of range) records a code in a per-device error word instead of
- *   faulting; read it with dsa_device_error.
+ * - Device error word.  A kernel that detects an error (a bounded wait that
+ *   timed out, an index out of range) records a DSA_DEVERR_* code instead
+ *   of faulting, and finishes.  Every launching call takes `err`: a device
+ *   pointer to a caller-owned int32 (4-byte aligned) that the call's kernels
+ *   record into (the first error wins; nothing else is written there), or
+ *   NULL, in which case they record into the library's per-device word.
+ *   Calls that may run at the same time (two streams, two host threads)
+ *   should each pass their own word, so that neither sees nor clears the
+ *   other's error.  The word must hold 0 before the call for a later
+ *   non-zero value to mean "this call failed"; dsa_check_device_error reads
+ *   a word and clears it.
  */
 #ifndef DSA_H_
 #define DSA_H_
@@ -60,7 +68,7 @@ typedef enum {
     DSA_ERR_DEVICE = 5         /* a kernel recorded an error in the device error word */
 } dsa_status_t;
 
-/* Device error word codes (dsa_device_error). */
+/* Device error word codes (dsa_check_device_error). */
 #define DSA_DEVERR_NONE 0
 #define DSA_DEVERR_TIMEOUT 1     /* a bounded wait inside a kernel gave up */
 #define DSA_DEVERR_INDEX 2       /* an index row held a key outside the cache */
@@ -92,7 +100,8 @@ DSA_API const char* dsa_last_error(void);
  * 1 <= L <= 2^30.  Others return DSA_ERR_UNSUPPORTED.
  */
 DSA_API dsa_status_t dsa_index_topk(const void* q_I, const void* k_I, const float* w, int64_t L,
-                            int H_I, int d_I, int k, int32_t* idx, dsa_stream_t stream);
+                            int H_I, int d_I, int k, int32_t* idx, int32_t* err,
+                            dsa_stream_t stream);
 
 /*
  * dsa_index_topk_varlen - dsa_index_topk over a packed batch of sequences
@@ -112,7 +121,8 @@ DSA_API dsa_status_t dsa_index_topk(const void* q_I, const void* k_I, const floa
  */
 DSA_API dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, const float* w,
                                    const int32_t* cu_seqlens, int nseq, int64_t L, int H_I,
-                                   int d_I, int k, int32_t* idx, dsa_stream_t stream);
+                                   int d_I, int k, int32_t* idx, int32_t* err,
+                                   dsa_stream_t stream);
 
 /*
  * dsa_sparse_attn_prefill_dedup - the result of dsa_sparse_attn_prefill,
@@ -128,7 +138,7 @@ DSA_API dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, con
  */
 DSA_API dsa_status_t dsa_sparse_attn_prefill_dedup(const void* Q, const void* K, const void* V,
                                            const int32_t* idx, int64_t L, int Hq, int Hkv,
-                                           int d, int k, float scale, void* O,
+                                           int d, int k, float scale, void* O, int32_t* err,
                                            dsa_stream_t stream);
 
 /*
@@ -156,8 +166,9 @@ DSA_API dsa_status_t dsa_prefill_from_host(const void* q_I_host, const void* k_I
                                    const void* V_host, void* O_host, void* q_I, void* k_I,
                                    float* w, void* Q, void* K, void* V, int32_t* idx, void* O,
                                    int64_t L, int H_I, int d_I, int Hq, int Hkv, int d, int k,
-                                   float scale, int64_t chunk_rows, dsa_stream_t stream,
-                                   dsa_stream_t h2d_stream, dsa_stream_t d2h_stream);
+                                   float scale, int64_t chunk_rows, int32_t* err,
+                                   dsa_stream_t stream, dsa_stream_t h2d_stream,
+                                   dsa_stream_t d2h_stream);
 
 /*
  * dsa_index_scores - the same indexer, writing the dense causal score
@@ -168,7 +179,8 @@ DSA_API dsa_status_t dsa_prefill_from_host(const void* q_I_host, const void* k_I
  * Same shape support as dsa_index_topk; L * L must fit in 2^31 elements.
  */
 DSA_API dsa_status_t dsa_index_scores(const void* q_I, const void* k_I, const float* w, int64_t L,
-                              int H_I, int d_I, float* scores, dsa_stream_t stream);
+                              int H_I, int d_I, float* scores, int32_t* err,
+                              dsa_stream_t stream);
 
 /*
  * dsa_sparse_attn_prefill - sparse GQA attention over selected rows (A3).
@@ -188,7 +200,8 @@ DSA_API dsa_status_t dsa_index_scores(const void* q_I, const void* k_I, const fl
  */
 DSA_API dsa_status_t dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
                                      const int32_t* idx, int64_t L, int Hq, int Hkv, int d,
-                                     int k, float scale, void* O, dsa_stream_t stream);
+                                     int k, float scale, void* O, int32_t* err,
+                                     dsa_stream_t stream);
 
 /*
  * dsa_decode_workspace_size - bytes of device workspace that
@@ -224,7 +237,7 @@ DSA_API dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, con
                                     const void* V_cache, const int64_t* cache_off, int B,
                                     int64_t total_n, int H_I, int d_I, int Hq, int Hkv, int d,
                                     int k, float scale, void* O, int32_t* idx_out,
-                                    void* workspace, size_t workspace_bytes,
+                                    void* workspace, size_t workspace_bytes, int32_t* err,
                                     dsa_stream_t stream);
 
 /*
@@ -236,11 +249,14 @@ DSA_API dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, con
  * image, held by every GPU that loads the library until the process exits.
  * Arguments, layouts and results are those of dsa_sparse_attn_decode.
  *
- * - Sizes whose dsa_decode_workspace_size exceeds 64 MiB are rejected with
- *   DSA_ERR_WORKSPACE before any launch.
+ * - Arguments are checked as dsa_sparse_attn_decode checks them (same
+ *   statuses); then sizes whose dsa_decode_workspace_size exceeds 64 MiB
+ *   are rejected with DSA_ERR_WORKSPACE before any launch.
  * - The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is cached per device and
+ *   context; a call made after the device's context was replaced (e.g. by
+ *   cudaDeviceReset) looks it up again.
  * - All calls share the array and it keeps the last call's contents (no
  *   part of it needs to start at zero).  Calls that overlap on the GPU race
  *   on it: serialize them.
@@ -249,7 +265,8 @@ DSA_API dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, con
 DSA_API dsa_status_t dsa_sparse_attn_decode_noalloc(
     const void* q_I, const float* w, const void* Q, const void* kI_cache, const void* K_cache,
     const void* V_cache, const int64_t* cache_off, int B, int64_t total_n, int H_I, int d_I,
-    int Hq, int Hkv, int d, int k, float scale, void* O, int32_t* idx_out, dsa_stream_t stream);
+    int Hq, int Hkv, int d, int k, float scale, void* O, int32_t* idx_out, int32_t* err,
+    dsa_stream_t stream);
 
 /*
  * Indexer warm-up loss (dense warm-up stage: Kwai Keye-VL-2.0 technical
@@ -287,7 +304,7 @@ DSA_API dsa_status_t dsa_indexer_kl_forward(const void* q_I, const void* k_I, co
                                     const void* Q, const void* K, int64_t L, int H_I, int d_I,
                                     int Hq, int Hkv, int d, float scale, float scale_I, float* kl,
                                     float* G, void* workspace, size_t workspace_bytes,
-                                    dsa_stream_t stream);
+                                    int32_t* err, dsa_stream_t stream);
 
 /*
  * dsa_indexer_kl_backward - gradients of sum_t kl[t] with respect to the
@@ -313,14 +330,17 @@ DSA_API size_t dsa_indexer_kl_backward_workspace_size(int64_t L, int H_I, int d_
 DSA_API dsa_status_t dsa_indexer_kl_backward(const void* q_I, const void* k_I, const float* w,
                                      const float* G, int64_t L, int H_I, int d_I, float* dq_I,
                                      float* dk_I, float* dw, void* workspace,
-                                     size_t workspace_bytes, dsa_stream_t stream);
+                                     size_t workspace_bytes, int32_t* err, dsa_stream_t stream);
 
 /*
- * dsa_device_error - synchronizes `stream`, then reads and clears the
- * current device's error word into *code (DSA_DEVERR_*).  Returns DSA_OK if
- * the word could be read (whatever its value), DSA_ERR_CUDA otherwise.
+ * dsa_check_device_error - synchronizes `stream`, then reads the device
+ * error word `err` (a caller's word as passed to the launching calls, or
+ * NULL for the current device's library word) into *code (DSA_DEVERR_*) and
+ * sets it back to 0.  Returns DSA_OK if the word could be read (whatever its
+ * value), DSA_ERR_INVALID_ARG for a NULL code or a misaligned err,
+ * DSA_ERR_CUDA otherwise.
  */
-DSA_API dsa_status_t dsa_device_error(int* code, dsa_stream_t stream);
+DSA_API dsa_status_t dsa_check_device_error(int32_t* err, int* code, dsa_stream_t stream);
 
 #ifdef __cplusplus
 }

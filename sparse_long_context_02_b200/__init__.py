@@ -47,40 +47,41 @@ def lib() -> ctypes.CDLL:
         L.dsa_last_error.restype = ctypes.c_char_p
         L.dsa_last_error.argtypes = []
         L.dsa_index_topk.restype = i32
-        L.dsa_index_topk.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp]
+        L.dsa_index_topk.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, vp, vp]
         L.dsa_index_scores.restype = i32
-        L.dsa_index_scores.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
+        L.dsa_index_scores.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp, vp]
         L.dsa_sparse_attn_prefill_dedup.restype = i32
         L.dsa_sparse_attn_prefill_dedup.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32,
-                                                    ctypes.c_float, vp, vp]
+                                                    ctypes.c_float, vp, vp, vp]
         L.dsa_prefill_from_host.restype = i32
         L.dsa_prefill_from_host.argtypes = [vp] * 15 + [i64, i32, i32, i32, i32, i32, i32,
-                                                          ctypes.c_float, i64, vp, vp, vp]
+                                                          ctypes.c_float, i64, vp, vp, vp, vp]
         L.dsa_index_topk_varlen.restype = i32
-        L.dsa_index_topk_varlen.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, vp]
+        L.dsa_index_topk_varlen.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp]
         L.dsa_sparse_attn_prefill.restype = i32
         L.dsa_sparse_attn_prefill.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, f32, vp,
-                                              vp]
+                                              vp, vp]
         L.dsa_decode_workspace_size.restype = sz
         L.dsa_decode_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32, i32]
         L.dsa_sparse_attn_decode.restype = i32
         L.dsa_sparse_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
-                                             i32, i32, i32, f32, vp, vp, vp, sz, vp]
+                                             i32, i32, i32, f32, vp, vp, vp, sz, vp, vp]
         L.dsa_sparse_attn_decode_noalloc.restype = i32
         L.dsa_sparse_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
-                                                     i32, i32, i32, i32, i32, f32, vp, vp, vp]
+                                                     i32, i32, i32, i32, i32, f32, vp, vp, vp,
+                                                     vp]
         L.dsa_indexer_kl_workspace_size.restype = sz
         L.dsa_indexer_kl_workspace_size.argtypes = [i64, i32]
         L.dsa_indexer_kl_forward.restype = i32
         L.dsa_indexer_kl_forward.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, f32,
-                                             f32, vp, vp, vp, sz, vp]
+                                             f32, vp, vp, vp, sz, vp, vp]
         L.dsa_indexer_kl_backward.restype = i32
         L.dsa_indexer_kl_backward_workspace_size.restype = sz
         L.dsa_indexer_kl_backward_workspace_size.argtypes = [i64, i32, i32]
         L.dsa_indexer_kl_backward.argtypes = [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz,
-                                              vp]
-        L.dsa_device_error.restype = i32
-        L.dsa_device_error.argtypes = [ctypes.POINTER(i32), vp]
+                                              vp, vp]
+        L.dsa_check_device_error.restype = i32
+        L.dsa_check_device_error.argtypes = [vp, ctypes.POINTER(i32), vp]
         _lib = L
     return _lib
 
@@ -103,6 +104,9 @@ def _stream(stream) -> int:
 def _dev(t: torch.Tensor, name: str, nbytes_per_elem: Optional[int] = None) -> int:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.type == "cuda" and t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, but the library launches on the current "
+                         f"device cuda:{torch.cuda.current_device()}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if nbytes_per_elem is not None and t.element_size() != nbytes_per_elem:
@@ -110,25 +114,41 @@ def _dev(t: torch.Tensor, name: str, nbytes_per_elem: Optional[int] = None) -> i
     return t.data_ptr()
 
 
+def _err(err: Optional[torch.Tensor]) -> Optional[int]:
+    """The caller's device error word (a one-element int32 CUDA tensor), or
+    None for the library's per-device word."""
+    if err is None:
+        return None
+    if err.dtype != torch.int32 or err.numel() < 1:
+        raise ValueError("err must be an int32 CUDA tensor of at least one element")
+    return _dev(err, "err", 4)
+
+
+def error_word(device=None) -> torch.Tensor:
+    """A fresh (zeroed) device error word for the calls of one stream."""
+    return torch.zeros(1, dtype=torch.int32, device=device if device is not None else "cuda")
+
+
 def version() -> int:
     return lib().dsa_version()
 
 
 def index_topk(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, k: int,
-               idx: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+               idx: Optional[torch.Tensor] = None, stream=None, err=None) -> torch.Tensor:
     """Indexer + top-k.  q_I [L][H_I][d_I] and k_I [L][d_I] e4m3 (uint8 or
     float8_e4m3fn), w [L][H_I] float32 -> idx [L][k] int32 (ascending, -1 pad)."""
     L, H, d = q_I.shape
     if idx is None:
         idx = torch.empty((L, k), dtype=torch.int32, device=q_I.device)
     _check(lib().dsa_index_topk(_dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), L, H, d,
-                                k, _dev(idx, "idx", 4), _stream(stream)), "dsa_index_topk")
+                                k, _dev(idx, "idx", 4), _err(err), _stream(stream)),
+           "dsa_index_topk")
     return idx
 
 
 def index_topk_varlen(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor,
                       cu_seqlens: torch.Tensor, k: int, idx: Optional[torch.Tensor] = None,
-                      stream=None) -> torch.Tensor:
+                      stream=None, err=None) -> torch.Tensor:
     """Indexer + top-k over a packed batch: cu_seqlens [nseq + 1] int32 on the
     device (0 ... L); row t of a sequence sees only that sequence's keys up to
     t.  idx holds packed key positions (ascending, -1 pad)."""
@@ -140,26 +160,26 @@ def index_topk_varlen(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor,
     nseq = cu_seqlens.numel() - 1
     _check(lib().dsa_index_topk_varlen(_dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4),
                                        _dev(cu_seqlens, "cu_seqlens", 4), nseq, L, H, d, k,
-                                       _dev(idx, "idx", 4), _stream(stream)),
+                                       _dev(idx, "idx", 4), _err(err), _stream(stream)),
            "dsa_index_topk_varlen")
     return idx
 
 
 def index_scores(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor,
-                 scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                 scores: Optional[torch.Tensor] = None, stream=None, err=None) -> torch.Tensor:
     """Dense causal indexer scores [L][L] float32 (-inf above the diagonal)."""
     L, H, d = q_I.shape
     if scores is None:
         scores = torch.empty((L, L), dtype=torch.float32, device=q_I.device)
     _check(lib().dsa_index_scores(_dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), L, H,
-                                  d, _dev(scores, "scores", 4), _stream(stream)),
+                                  d, _dev(scores, "scores", 4), _err(err), _stream(stream)),
            "dsa_index_scores")
     return scores
 
 
 def sparse_attn_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, idx: torch.Tensor,
                         scale: float, O: Optional[torch.Tensor] = None,
-                        stream=None) -> torch.Tensor:
+                        stream=None, err=None) -> torch.Tensor:
     """Sparse GQA attention.  Q [L][Hq][d], K/V [L][Hkv][d] bf16, idx [L][k]
     int32 -> O [L][Hq][d] bf16."""
     L, Hq, d = Q.shape
@@ -169,19 +189,19 @@ def sparse_attn_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, idx: 
         O = torch.empty_like(Q)
     _check(lib().dsa_sparse_attn_prefill(_dev(Q, "Q", 2), _dev(K, "K", 2), _dev(V, "V", 2),
                                          _dev(idx, "idx", 4), L, Hq, Hkv, d, k, float(scale),
-                                         _dev(O, "O", 2), _stream(stream)),
+                                         _dev(O, "O", 2), _err(err), _stream(stream)),
            "dsa_sparse_attn_prefill")
     return O
 
 
 def _host(t: torch.Tensor, name: str) -> int:
-    if t.is_cuda or not t.is_contiguous():
-        raise DSAError(f"{name} must be a contiguous host tensor")
+    if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host tensor")
     return t.data_ptr()
 
 
 def prefill_from_host(host: dict, dev: dict, k: int, scale: float, chunk_rows: int = 8192,
-                      stream=None, h2d_stream=None, d2h_stream=None) -> None:
+                      stream=None, h2d_stream=None, d2h_stream=None, err=None) -> None:
     """Whole prefill from host inputs with copies and kernels overlapped in
     row chunks.  host: q_I, k_I, w, Q, K, V (inputs) and O (output), pinned
     CPU tensors; dev: device buffers of the same names plus idx [L][k].
@@ -190,18 +210,19 @@ def prefill_from_host(host: dict, dev: dict, k: int, scale: float, chunk_rows: i
     Hq, d = host["Q"].shape[1], host["Q"].shape[2]
     Hkv = host["K"].shape[1]
     if h2d_stream is None or d2h_stream is None:
-        raise DSAError("dsa_prefill_from_host: pass h2d_stream and d2h_stream")
+        raise ValueError("dsa_prefill_from_host: pass h2d_stream and d2h_stream")
     names = ("q_I", "k_I", "w", "Q", "K", "V")
     args = [_host(host[n], n) for n in names] + [_host(host["O"], "O")]
     args += [_dev(dev[n], n) for n in names] + [_dev(dev["idx"], "idx", 4), _dev(dev["O"], "O")]
     _check(lib().dsa_prefill_from_host(*args, L, H, d_I, Hq, Hkv, d, k, float(scale), chunk_rows,
-                                       _stream(stream), _stream(h2d_stream), _stream(d2h_stream)),
+                                       _err(err), _stream(stream), _stream(h2d_stream),
+                                       _stream(d2h_stream)),
            "dsa_prefill_from_host")
 
 
 def sparse_attn_prefill_dedup(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                               idx: torch.Tensor, scale: float, O: Optional[torch.Tensor] = None,
-                              stream=None) -> torch.Tensor:
+                              stream=None, err=None) -> torch.Tensor:
     """sparse_attn_prefill for blocks of 6 adjacent queries that gather the
     union of their index rows once (pays when adjacent rows overlap)."""
     L, Hq, d = Q.shape
@@ -211,7 +232,8 @@ def sparse_attn_prefill_dedup(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
         O = torch.empty_like(Q)
     _check(lib().dsa_sparse_attn_prefill_dedup(_dev(Q, "Q", 2), _dev(K, "K", 2), _dev(V, "V", 2),
                                                _dev(idx, "idx", 4), L, Hq, Hkv, d, k,
-                                               float(scale), _dev(O, "O", 2), _stream(stream)),
+                                               float(scale), _dev(O, "O", 2), _err(err),
+                                               _stream(stream)),
            "dsa_sparse_attn_prefill_dedup")
     return O
 
@@ -222,7 +244,7 @@ def decode_workspace_size(B: int, total_n: int, H_I: int, d_I: int, k: int, Hq: 
 
 
 def sparse_attn_decode(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, k: int, scale: float,
-                       O=None, idx_out=None, workspace=None, stream=None):
+                       O=None, idx_out=None, workspace=None, stream=None, err=None):
     """One new token per sequence.  Returns (O [B][Hq][d] bf16, idx_out or None)."""
     B, H, dI = q_I.shape
     _, Hq, d = Q.shape
@@ -238,13 +260,13 @@ def sparse_attn_decode(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, k: int,
         _dev(K_cache, "K_cache", 2), _dev(V_cache, "V_cache", 2), _dev(cache_off, "cache_off", 8),
         B, total_n, H, dI, Hq, Hkv, d, k, float(scale), _dev(O, "O", 2),
         _dev(idx_out, "idx_out", 4) if idx_out is not None else None,
-        _dev(workspace, "workspace", 1), workspace.numel(), _stream(stream)),
+        _dev(workspace, "workspace", 1), workspace.numel(), _err(err), _stream(stream)),
         "dsa_sparse_attn_decode")
     return O, idx_out
 
 
 def sparse_attn_decode_noalloc(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, k: int,
-                               scale: float, O=None, idx_out=None, stream=None):
+                               scale: float, O=None, idx_out=None, stream=None, err=None):
     """sparse_attn_decode without a workspace argument, for callers that
     cannot allocate device memory at call time: the scratch is a fixed
     64 MiB array inside the library (see include/dsa.h).  Calls that overlap
@@ -259,15 +281,17 @@ def sparse_attn_decode_noalloc(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off,
         _dev(q_I, "q_I", 1), _dev(w, "w", 4), _dev(Q, "Q", 2), _dev(kI_cache, "kI_cache", 1),
         _dev(K_cache, "K_cache", 2), _dev(V_cache, "V_cache", 2), _dev(cache_off, "cache_off", 8),
         B, total_n, H, dI, Hq, Hkv, d, k, float(scale), _dev(O, "O", 2),
-        _dev(idx_out, "idx_out", 4) if idx_out is not None else None, _stream(stream)),
-        "dsa_sparse_attn_decode_noalloc")
+        _dev(idx_out, "idx_out", 4) if idx_out is not None else None, _err(err),
+        _stream(stream)), "dsa_sparse_attn_decode_noalloc")
     return O, idx_out
 
 
-def device_error(stream=None) -> int:
-    """Synchronizes the stream; returns and clears the device error word."""
+def device_error(stream=None, err=None) -> int:
+    """Synchronizes the stream; returns and clears a device error word: the
+    caller's `err` tensor, or the library's per-device word when None."""
     code = ctypes.c_int(0)
-    _check(lib().dsa_device_error(ctypes.byref(code), _stream(stream)), "dsa_device_error")
+    _check(lib().dsa_check_device_error(_err(err), ctypes.byref(code), _stream(stream)),
+           "dsa_check_device_error")
     return code.value
 
 
@@ -278,7 +302,7 @@ def indexer_kl_workspace_size(L: int, Hq: int) -> int:
 def indexer_kl_forward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, Q: torch.Tensor,
                        K: torch.Tensor, scale: float, scale_I: float = 1.0,
                        kl: Optional[torch.Tensor] = None, G: Optional[torch.Tensor] = None,
-                       workspace: Optional[torch.Tensor] = None, stream=None):
+                       workspace: Optional[torch.Tensor] = None, stream=None, err=None):
     """Indexer warm-up loss.  Returns (kl [L] float32, G [L][L] float32 =
     d(sum kl)/dI, zero above the diagonal).  q_I/k_I e4m3, w float32, Q/K
     bf16 (layouts as dsa_indexer_kl_forward)."""
@@ -297,14 +321,14 @@ def indexer_kl_forward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, Q:
         _dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), _dev(Q, "Q", 2),
         _dev(K, "K", 2), L, H_I, d_I, Hq, Hkv, d, float(scale), float(scale_I), _dev(kl, "kl", 4),
         _dev(G, "G", 4), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        _stream(stream)), "dsa_indexer_kl_forward")
+        _err(err), _stream(stream)), "dsa_indexer_kl_forward")
     return kl, G
 
 
 def indexer_kl_backward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, G: torch.Tensor,
                         dq_I: Optional[torch.Tensor] = None, dk_I: Optional[torch.Tensor] = None,
                         dw: Optional[torch.Tensor] = None,
-                        workspace: Optional[torch.Tensor] = None, stream=None):
+                        workspace: Optional[torch.Tensor] = None, stream=None, err=None):
     """Gradients of sum_t kl[t] with respect to q_I, k_I and w, from G.
     Returns (dq_I [L][H_I][d_I], dk_I [L][d_I], dw [L][H_I]), float32."""
     L, H_I, d_I = q_I.shape
@@ -322,5 +346,5 @@ def indexer_kl_backward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, G
         _dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4), _dev(G, "G", 4), L, H_I, d_I,
         _dev(dq_I, "dq_I", 4), _dev(dk_I, "dk_I", 4), _dev(dw, "dw", 4),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        _stream(stream)), "dsa_indexer_kl_backward")
+        _err(err), _stream(stream)), "dsa_indexer_kl_backward")
     return dq_I, dk_I, dw

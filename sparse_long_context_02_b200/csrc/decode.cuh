@@ -68,6 +68,7 @@ struct Params {
     int* cand_cnt;             // [slots]
     uint32_t* cand_th;         // [slots] an ord that at least k of the slot's entries reach
                                // (0 when the slot holds fewer than k or none is known)
+    int* err;                  // the call's device error word (null: the per-device word)
 };
 
 __device__ __forceinline__ bool seq_ok(const Params& p, int b) {
@@ -153,6 +154,7 @@ __device__ __forceinline__ bool make_segment(const Params& p, int b, int64_t r0,
 __global__ void __launch_bounds__(kThreads, 1)
 index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
              const Params p) {
+    bind_error_word(p.err);
     constexpr int N = HI;
     constexpr int KT_BYTES = kKeyTile * DI;
     constexpr uint32_t TMEM_COLS = 512;  // 4 warpgroups x 2 accumulators x 64 columns
@@ -398,6 +400,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
 // smem_cap entries, else in place in the candidate arrays), then selected.
 __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* idx_out,
                                                       int smem_cap) {
+    bind_error_word(p.err);
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ Scratch<1024> S;
     __shared__ int total_s;

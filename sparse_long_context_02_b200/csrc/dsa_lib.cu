@@ -39,6 +39,13 @@ dsa_status_t ok() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The caller's device error word: NULL (the per-device word) or 4-byte aligned.
+#define CHECK_ERR_WORD(p)                                                              \
+    do {                                                                              \
+        if ((reinterpret_cast<uintptr_t>(p) & 3u) != 0)                                \
+            return fail(DSA_ERR_INVALID_ARG, "%s: err is not 4-byte aligned", fn);      \
+    } while (0)
+
 #define CHECK_PTR(p)                                                                  \
     do {                                                                              \
         if ((p) == nullptr) return fail(DSA_ERR_INVALID_ARG, "%s: " #p " is NULL", fn); \
@@ -106,7 +113,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 template <int HI, int DI, bool TOPK>
 dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
                           int64_t L, int k, int32_t* idx, float* scores, const int32_t* cu_seqlens,
-                          int nseq, int64_t row0, int64_t row1, cudaStream_t st) {
+                          int nseq, int64_t row0, int64_t row1, int* err, cudaStream_t st) {
     CUtensorMap mq, mk;
     if (!make_map(&mq, q_I, DI, (uint64_t)L * HI, dsa::idx::kTokens * HI) ||
         !make_map(&mk, k_I, DI, (uint64_t)L, dsa::idx::kKeyTile))
@@ -135,6 +142,7 @@ dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, cons
     p.nblocks = (int)((row1 + dsa::idx::kTokens - 1) / dsa::idx::kTokens) - p.blk0;
     p.cu_seqlens = cu_seqlens;
     p.nseq = nseq;
+    p.err = err;
     kern<<<p.nblocks, dsa::idx::kThreads, smem, st>>>(mq, mk, p);
     CUDA_TRY(cudaGetLastError());
     return ok();
@@ -143,17 +151,17 @@ dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, cons
 template <bool TOPK>
 dsa_status_t dispatch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
                             int64_t L, int H_I, int d_I, int k, int32_t* idx, float* scores,
-                            const int32_t* cu, int nseq, cudaStream_t st, int64_t row0 = 0,
-                            int64_t row1 = -1) {
+                            const int32_t* cu, int nseq, int* err, cudaStream_t st,
+                            int64_t row0 = 0, int64_t row1 = -1) {
     if (row1 < 0) row1 = L;
     if (H_I == 64 && d_I == 128)
-        return launch_index<64, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, st);
+        return launch_index<64, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st);
     if (H_I == 64 && d_I == 64)
-        return launch_index<64, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, st);
+        return launch_index<64, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st);
     if (H_I == 4 && d_I == 128)
-        return launch_index<4, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, st);
+        return launch_index<4, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st);
     if (H_I == 4 && d_I == 64)
-        return launch_index<4, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, st);
+        return launch_index<4, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st);
     return fail(DSA_ERR_UNSUPPORTED, "%s: (H_I, d_I) = (%d, %d) not in {4, 64} x {64, 128}", fn,
                 H_I, d_I);
 }
@@ -210,7 +218,7 @@ dsa_status_t launch_dedup(const char* fn, const dsa::attn::Params& p, int64_t L,
 // checked by the caller).
 dsa_status_t attn_prefill_rows(const char* fn, const void* Q, const void* K, const void* V,
                                const int32_t* idx, int64_t L, int Hq, int Hkv, int d, int k,
-                               float scale, void* O, int64_t row0, int64_t row1,
+                               float scale, void* O, int64_t row0, int64_t row1, int* err,
                                cudaStream_t st) {
     const int G = Hq / Hkv;
     dsa::attn::Params p{};
@@ -222,6 +230,7 @@ dsa_status_t attn_prefill_rows(const char* fn, const void* Q, const void* K, con
     p.k = k;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.O = static_cast<__nv_bfloat16*>(O) + row0 * Hq * d;
+    p.err = err;
     const int64_t rows = row1 - row0;
     if (d == 128 && Hkv == 4 && G == 8) return launch_attn<128, 4, 8, false>(fn, p, rows, st);
     if (d == 64 && Hkv == 2 && G == 4) return launch_attn<64, 2, 4, false>(fn, p, rows, st);
@@ -251,29 +260,33 @@ const char* dsa_status_string(int status) {
 const char* dsa_last_error(void) { return g_last_error; }
 
 dsa_status_t dsa_index_topk(const void* q_I, const void* k_I, const float* w, int64_t L,
-                            int H_I, int d_I, int k, int32_t* idx, dsa_stream_t stream) {
+                            int H_I, int d_I, int k, int32_t* idx, int32_t* err,
+                            dsa_stream_t stream) {
     static const char fn[] = "dsa_index_topk";
     CHECK_PTR(q_I);
     CHECK_PTR(k_I);
     CHECK_PTR(w);
     CHECK_PTR(idx);
+    CHECK_ERR_WORD(err);
     if (L < 1 || L > (int64_t(1) << 30)) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
     if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
     if (k > 2048) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > 2048", fn, k);
     if (L * H_I >= (int64_t(1) << 31))
         return fail(DSA_ERR_UNSUPPORTED, "%s: L * H_I too large", fn);
-    return dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, nullptr, 1,
+    return dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, nullptr, 1, err,
                                 static_cast<cudaStream_t>(stream));
 }
 
 dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, const float* w,
                                    const int32_t* cu_seqlens, int nseq, int64_t L, int H_I,
-                                   int d_I, int k, int32_t* idx, dsa_stream_t stream) {
+                                   int d_I, int k, int32_t* idx, int32_t* err,
+                                   dsa_stream_t stream) {
     static const char fn[] = "dsa_index_topk_varlen";
     CHECK_PTR(q_I);
     CHECK_PTR(k_I);
     CHECK_PTR(w);
     CHECK_PTR(idx);
+    CHECK_ERR_WORD(err);
     if (cu_seqlens == nullptr) return fail(DSA_ERR_INVALID_ARG, "%s: cu_seqlens is null", fn);
     if (nseq < 1) return fail(DSA_ERR_INVALID_ARG, "%s: nseq = %d", fn, nseq);
     if (L < 1 || L > (int64_t(1) << 30)) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
@@ -282,18 +295,20 @@ dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, const float
     if (L * H_I >= (int64_t(1) << 31))
         return fail(DSA_ERR_UNSUPPORTED, "%s: L * H_I too large", fn);
     return dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, cu_seqlens, nseq,
-                                static_cast<cudaStream_t>(stream));
+                                err, static_cast<cudaStream_t>(stream));
 }
 
 dsa_status_t dsa_sparse_attn_prefill_dedup(const void* Q, const void* K, const void* V,
                                            const int32_t* idx, int64_t L, int Hq, int Hkv, int d,
-                                           int k, float scale, void* O, dsa_stream_t stream) {
+                                           int k, float scale, void* O, int32_t* err,
+                                           dsa_stream_t stream) {
     static const char fn[] = "dsa_sparse_attn_prefill_dedup";
     CHECK_PTR(Q);
     CHECK_PTR(K);
     CHECK_PTR(V);
     CHECK_PTR(idx);
     CHECK_PTR(O);
+    CHECK_ERR_WORD(err);
     if (L < 1) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
     if (L > dsa::attn::kDedupMaxKeys)
         return fail(DSA_ERR_UNSUPPORTED, "%s: L = %lld > %d", fn, (long long)L, dsa::attn::kDedupMaxKeys);
@@ -311,6 +326,7 @@ dsa_status_t dsa_sparse_attn_prefill_dedup(const void* Q, const void* K, const v
     p.k = k;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.O = static_cast<__nv_bfloat16*>(O);
+    p.err = err;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     dsa_status_t r;
     if (d == 128 && Hkv == 4 && G == 8) r = launch_dedup<128, 4, 8>(fn, p, L, st);
@@ -325,7 +341,7 @@ dsa_status_t dsa_prefill_from_host(const void* q_I_h, const void* k_I_h, const f
                                    void* q_I, void* k_I, float* w, void* Q, void* K, void* V,
                                    int32_t* idx, void* O, int64_t L, int H_I, int d_I, int Hq,
                                    int Hkv, int d, int k, float scale, int64_t chunk_rows,
-                                   dsa_stream_t stream, dsa_stream_t h2d_stream,
+                                   int32_t* err, dsa_stream_t stream, dsa_stream_t h2d_stream,
                                    dsa_stream_t d2h_stream) {
     static const char fn[] = "dsa_prefill_from_host";
     CHECK_PTR(q_I_h);
@@ -343,6 +359,7 @@ dsa_status_t dsa_prefill_from_host(const void* q_I_h, const void* k_I_h, const f
     CHECK_PTR(V);
     CHECK_PTR(idx);
     CHECK_PTR(O);
+    CHECK_ERR_WORD(err);
     if (L < 1 || L > (int64_t(1) << 30)) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
     if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
     if (k > 2048) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > 2048", fn, k);
@@ -387,9 +404,9 @@ dsa_status_t dsa_prefill_from_host(const void* q_I_h, const void* k_I_h, const f
         // rows [r0, r1) need keys [0, r1): all of them are on the device now
         CUDA_TRY(cudaStreamWaitEvent(st, ev[2 * c], 0));
         dsa_status_t r = dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, nullptr,
-                                              1, st, r0, r1);
+                                              1, err, st, r0, r1);
         if (r != DSA_OK) return r;
-        r = attn_prefill_rows(fn, Q, K, V, idx, L, Hq, Hkv, d, k, scale, O, r0, r1, st);
+        r = attn_prefill_rows(fn, Q, K, V, idx, L, Hq, Hkv, d, k, scale, O, r0, r1, err, st);
         if (r != DSA_OK) return r;
         CUDA_TRY(cudaEventRecord(ev[2 * c + 1], st));
         CUDA_TRY(cudaStreamWaitEvent(sd, ev[2 * c + 1], 0));
@@ -402,33 +419,37 @@ dsa_status_t dsa_prefill_from_host(const void* q_I_h, const void* k_I_h, const f
 }
 
 dsa_status_t dsa_index_scores(const void* q_I, const void* k_I, const float* w, int64_t L,
-                              int H_I, int d_I, float* scores, dsa_stream_t stream) {
+                              int H_I, int d_I, float* scores, int32_t* err,
+                              dsa_stream_t stream) {
     static const char fn[] = "dsa_index_scores";
     CHECK_PTR(q_I);
     CHECK_PTR(k_I);
     CHECK_PTR(w);
     CHECK_PTR(scores);
+    CHECK_ERR_WORD(err);
     if (L < 1 || L * L >= (int64_t(1) << 31))
         return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld (L * L must be < 2^31)", fn, (long long)L);
-    return dispatch_index<false>(fn, q_I, k_I, w, L, H_I, d_I, 1, nullptr, scores, nullptr, 1,
+    return dispatch_index<false>(fn, q_I, k_I, w, L, H_I, d_I, 1, nullptr, scores, nullptr, 1, err,
                                  static_cast<cudaStream_t>(stream));
 }
 
 dsa_status_t dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
                                      const int32_t* idx, int64_t L, int Hq, int Hkv, int d,
-                                     int k, float scale, void* O, dsa_stream_t stream) {
+                                     int k, float scale, void* O, int32_t* err,
+                                     dsa_stream_t stream) {
     static const char fn[] = "dsa_sparse_attn_prefill";
     CHECK_PTR(Q);
     CHECK_PTR(K);
     CHECK_PTR(V);
     CHECK_PTR(idx);
     CHECK_PTR(O);
+    CHECK_ERR_WORD(err);
     if (L < 1 || L > (int64_t(1) << 30)) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
     if (k < 1 || k > 65536) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
     if (Hkv < 1 || Hq < 1 || Hq % Hkv) return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d", fn, Hq, Hkv);
     if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
     const dsa_status_t r = attn_prefill_rows(fn, Q, K, V, idx, L, Hq, Hkv, d, k, scale, O, 0, L,
-                                             static_cast<cudaStream_t>(stream));
+                                             err, static_cast<cudaStream_t>(stream));
     return r == DSA_OK ? ok() : r;
 }
 
@@ -481,14 +502,17 @@ size_t dsa_decode_workspace_size(int B, int64_t total_n, int H_I, int d_I, int k
     return plan_decode(B, total_n, k, Hq, d, num_sms()).total;
 }
 
-dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void* Q,
-                                    const void* kI_cache, const void* K_cache,
-                                    const void* V_cache, const int64_t* cache_off, int B,
-                                    int64_t total_n, int H_I, int d_I, int Hq, int Hkv, int d,
-                                    int k, float scale, void* O, int32_t* idx_out,
-                                    void* workspace, size_t workspace_bytes,
-                                    dsa_stream_t stream) {
-    static const char fn[] = "dsa_sparse_attn_decode";
+}  // extern "C"
+
+namespace {
+
+// Argument checks of the decode calls (with and without a caller workspace):
+// everything but the workspace itself.
+dsa_status_t check_decode_args(const char* fn, const void* q_I, const float* w, const void* Q,
+                               const void* kI_cache, const void* K_cache, const void* V_cache,
+                               const int64_t* cache_off, int B, int64_t total_n, int H_I,
+                               int d_I, int Hq, int Hkv, int d, int k, float scale, void* O,
+                               int32_t* idx_out, int32_t* err) {
     CHECK_PTR(q_I);
     CHECK_PTR(w);
     CHECK_PTR(Q);
@@ -497,7 +521,7 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     CHECK_PTR(V_cache);
     CHECK_PTR(cache_off);
     CHECK_PTR(O);
-    CHECK_PTR(workspace);
+    CHECK_ERR_WORD(err);
     if (idx_out && !aligned16(idx_out))
         return fail(DSA_ERR_INVALID_ARG, "%s: idx_out is not 16-byte aligned", fn);
     if (B < 1 || B > 4096) return fail(DSA_ERR_INVALID_ARG, "%s: B = %d", fn, B);
@@ -508,6 +532,15 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     if (H_I != 64 || d_I != 128 || d != 128 || Hkv != 4 || Hq != 32 || k > 2048)
         return fail(DSA_ERR_UNSUPPORTED,
                     "%s: supported H_I=64, d_I=128, d=128, Hkv=4, Hq=32, k<=2048", fn);
+    return DSA_OK;
+}
+
+// The decode itself, on checked arguments.
+dsa_status_t run_decode(const char* fn, const void* q_I, const float* w, const void* Q,
+                        const void* kI_cache, const void* K_cache, const void* V_cache,
+                        const int64_t* cache_off, int B, int64_t total_n, int k, int Hq, int d,
+                        float scale, void* O, int32_t* idx_out, void* workspace,
+                        size_t workspace_bytes, int32_t* err, dsa_stream_t stream) {
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(DSA_ERR_INVALID_ARG, "%s: workspace is not 256-byte aligned", fn);
     const DecodePlan pl = plan_decode(B, total_n, k, Hq, d, num_sms());
@@ -528,6 +561,7 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     dp.cand_ix = reinterpret_cast<int32_t*>(ws + pl.off_ix);
     dp.cand_cnt = reinterpret_cast<int*>(ws + pl.off_cnt);
     dp.cand_th = reinterpret_cast<uint32_t*>(ws + pl.off_th);
+    dp.err = err;
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + pl.off_idx);
 
     CUtensorMap mq, mk;
@@ -563,6 +597,7 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     ap.nsplit = pl.nsplit;
     ap.part_o = reinterpret_cast<float*>(ws + pl.off_po);
     ap.part_ml = reinterpret_cast<float*>(ws + pl.off_pml);
+    ap.err = err;
     dsa_status_t r = launch_attn<128, 4, 8, true>(fn, ap, (int64_t)B * pl.nsplit, st);
     if (r != DSA_OK) return r;
     CUDA_TRY(launch_chained(dsa::attn::combine_kernel<128, 32>, dim3(B * 32), dim3(128), 0, st,
@@ -572,13 +607,39 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     return ok();
 }
 
-dsa_status_t dsa_device_error(int* code, dsa_stream_t stream) {
-    static const char fn[] = "dsa_device_error";
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void* Q,
+                                    const void* kI_cache, const void* K_cache,
+                                    const void* V_cache, const int64_t* cache_off, int B,
+                                    int64_t total_n, int H_I, int d_I, int Hq, int Hkv, int d,
+                                    int k, float scale, void* O, int32_t* idx_out,
+                                    void* workspace, size_t workspace_bytes, int32_t* err,
+                                    dsa_stream_t stream) {
+    static const char fn[] = "dsa_sparse_attn_decode";
+    dsa_status_t r = check_decode_args(fn, q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, B,
+                                       total_n, H_I, d_I, Hq, Hkv, d, k, scale, O, idx_out, err);
+    if (r != DSA_OK) return r;
+    CHECK_PTR(workspace);
+    return run_decode(fn, q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, B, total_n, k, Hq, d,
+                      scale, O, idx_out, workspace, workspace_bytes, err, stream);
+}
+
+dsa_status_t dsa_check_device_error(int32_t* err, int* code, dsa_stream_t stream) {
+    static const char fn[] = "dsa_check_device_error";
     if (!code) return fail(DSA_ERR_INVALID_ARG, "%s: code is NULL", fn);
+    CHECK_ERR_WORD(err);
     CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
     int v = 0, zero = 0;
-    CUDA_TRY(cudaMemcpyFromSymbol(&v, dsa::g_dsa_device_error, sizeof(int)));
-    CUDA_TRY(cudaMemcpyToSymbol(dsa::g_dsa_device_error, &zero, sizeof(int)));
+    if (err != nullptr) {
+        CUDA_TRY(cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost));
+        CUDA_TRY(cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice));
+    } else {
+        CUDA_TRY(cudaMemcpyFromSymbol(&v, dsa::g_dsa_device_error, sizeof(int)));
+        CUDA_TRY(cudaMemcpyToSymbol(dsa::g_dsa_device_error, &zero, sizeof(int)));
+    }
     *code = v;
     return ok();
 }
@@ -597,15 +658,18 @@ dsa_status_t dsa_device_error(int* code, dsa_stream_t stream) {
 // * Every GPU that loads this library holds the array (kNoAllocScratchBytes)
 //   until the process exits.
 // * Host code cannot use the array's name as a device address; the address
-//   is looked up with cudaGetSymbolAddress once per device, on the first call
-//   made with that device current.  Make that first call before any stream
-//   capture.
+//   is looked up with cudaGetSymbolAddress once per device (and context), on
+//   the first call made with that device current.  Make that first call
+//   before any stream capture.  If the device's context is replaced (a
+//   cudaDeviceReset, for one), the next call sees a different context and
+//   looks the address up again.
 // * All calls share the one array and it keeps the last call's contents.
 //   Nothing in it has to start at zero: every scratch byte a decode reads was
 //   written earlier by the same call.  Calls whose work overlaps on the GPU
 //   (two streams, or two host threads) race on the array and must be
 //   serialized by the caller.
-// * A request whose scratch need exceeds the array is rejected with
+// * Arguments are checked as dsa_sparse_attn_decode checks them; then a
+//   request whose scratch need exceeds the array is rejected with
 //   DSA_ERR_WORKSPACE before anything is launched.
 
 namespace {
@@ -615,18 +679,47 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct NoAllocSlot {
+    CUcontext ctx;  // context the address was looked up in
+    void* ptr;
+};
+NoAllocSlot g_noalloc_slot[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+CUcontext current_ctx() {
+    CUcontext c = nullptr;
+    const CtxGetCurrentFn f = ctx_get_current_fn();
+    if (f == nullptr || f(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
 
 }  // namespace
 
 extern "C" dsa_status_t dsa_sparse_attn_decode_noalloc(
     const void* q_I, const float* w, const void* Q, const void* kI_cache, const void* K_cache,
     const void* V_cache, const int64_t* cache_off, int B, int64_t total_n, int H_I, int d_I,
-    int Hq, int Hkv, int d, int k, float scale, void* O, int32_t* idx_out, dsa_stream_t stream) {
+    int Hq, int Hkv, int d, int k, float scale, void* O, int32_t* idx_out, int32_t* err,
+    dsa_stream_t stream) {
     static const char fn[] = "dsa_sparse_attn_decode_noalloc";
-    if (B < 1 || total_n < 1 || k < 1)
-        return fail(DSA_ERR_INVALID_ARG, "%s: B = %d, total_n = %lld, k = %d", fn, B,
-                    (long long)total_n, k);
+    const dsa_status_t r = check_decode_args(fn, q_I, w, Q, kI_cache, K_cache, V_cache,
+                                             cache_off, B, total_n, H_I, d_I, Hq, Hkv, d, k,
+                                             scale, O, idx_out, err);
+    if (r != DSA_OK) return r;
     const size_t need = dsa_decode_workspace_size(B, total_n, H_I, d_I, k, Hq, Hkv, d);
     if (need > kNoAllocScratchBytes)
         return fail(DSA_ERR_WORKSPACE,
@@ -640,16 +733,18 @@ extern "C" dsa_status_t dsa_sparse_attn_decode_noalloc(
     void* scratch = nullptr;
     {
         std::lock_guard<std::mutex> lock(g_noalloc_mu);
-        if (!g_noalloc_ptr[dev]) {
+        NoAllocSlot& sl = g_noalloc_slot[dev];
+        const CUcontext ctx = current_ctx();
+        if (sl.ptr == nullptr || ctx == nullptr || ctx != sl.ctx) {
             void* p = nullptr;
-            CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-            g_noalloc_ptr[dev] = p;
+            CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));  // sets up the context
+            sl.ptr = p;
+            sl.ctx = current_ctx();
         }
-        scratch = g_noalloc_ptr[dev];
+        scratch = sl.ptr;
     }
-    return dsa_sparse_attn_decode(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, B, total_n,
-                                  H_I, d_I, Hq, Hkv, d, k, scale, O, idx_out, scratch,
-                                  kNoAllocScratchBytes, stream);
+    return run_decode(fn, q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, B, total_n, k, Hq, d,
+                      scale, O, idx_out, scratch, kNoAllocScratchBytes, err, stream);
 }
 
 // ---------------------------------------------------------------- indexer warm-up loss
@@ -760,8 +855,9 @@ dsa_status_t dsa_indexer_kl_forward(const void* q_I, const void* k_I, const floa
                                     const void* Q, const void* K, int64_t L, int H_I, int d_I,
                                     int Hq, int Hkv, int d, float scale, float scale_I, float* kl,
                                     float* G, void* workspace, size_t workspace_bytes,
-                                    dsa_stream_t stream) {
+                                    int32_t* err, dsa_stream_t stream) {
     static const char fn[] = "dsa_indexer_kl_forward";
+    CHECK_ERR_WORD(err);
     CHECK_PTR(q_I);
     CHECK_PTR(k_I);
     CHECK_PTR(w);
@@ -786,7 +882,7 @@ dsa_status_t dsa_indexer_kl_forward(const void* q_I, const void* k_I, const floa
                     workspace_bytes, ws.total);
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     dsa_status_t r = dispatch_index<false>(fn, q_I, k_I, w, L, H_I, d_I, 1, nullptr, G, nullptr, 1,
-                                           st);
+                                           err, st);
     if (r != DSA_OK) return r;
     dsa::kl::Params p{};
     p.Q = static_cast<const __nv_bfloat16*>(Q);
@@ -804,6 +900,7 @@ dsa_status_t dsa_indexer_kl_forward(const void* q_I, const void* k_I, const floa
     p.lse_I = reinterpret_cast<float*>(wsb + ws.lse_I);
     p.kl_part = reinterpret_cast<float*>(wsb + ws.part);
     p.kl = kl;
+    p.err = err;
     r = d == 128 ? launch_kl_forward<128>(fn, p, st) : launch_kl_forward<64>(fn, p, st);
     return r == DSA_OK ? ok() : r;
 }
@@ -811,8 +908,9 @@ dsa_status_t dsa_indexer_kl_forward(const void* q_I, const void* k_I, const floa
 dsa_status_t dsa_indexer_kl_backward(const void* q_I, const void* k_I, const float* w,
                                      const float* G, int64_t L, int H_I, int d_I, float* dq_I,
                                      float* dk_I, float* dw, void* workspace,
-                                     size_t workspace_bytes, dsa_stream_t stream) {
+                                     size_t workspace_bytes, int32_t* err, dsa_stream_t stream) {
     static const char fn[] = "dsa_indexer_kl_backward";
+    CHECK_ERR_WORD(err);
     CHECK_PTR(q_I);
     CHECK_PTR(k_I);
     CHECK_PTR(w);
@@ -845,6 +943,7 @@ dsa_status_t dsa_indexer_kl_backward(const void* q_I, const void* k_I, const flo
     p.dq = dq_I;
     p.dk = dk_I;
     p.dw = dw;
+    p.err = err;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     const dsa_status_t r =
         d_I == 128 ? launch_kl_backward<128>(fn, p, st) : launch_kl_backward<64>(fn, p, st);

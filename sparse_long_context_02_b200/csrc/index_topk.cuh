@@ -179,6 +179,7 @@ struct Params {
     // [cu_seqlens[b], t] of its own sequence b.  Null: one sequence.
     const int32_t* cu_seqlens;  // [nseq + 1], 0 ... L, non-decreasing
     int nseq;
+    int* err;            // the call's device error word (null: the per-device word)
 };
 
 // Start of the sequence that holds row t: cu[b] for the last b with
@@ -200,6 +201,7 @@ template <int HI, int DI, bool TOPK>
 __global__ void __launch_bounds__(kThreads, 1)
 index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
              const Params p) {
+    bind_error_word(p.err);
     constexpr int N = kTokens * HI;
     constexpr int KT_BYTES = kKeyTile * DI;
     constexpr int Q_BYTES = N * DI;

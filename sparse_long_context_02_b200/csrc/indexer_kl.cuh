@@ -64,6 +64,7 @@ struct Params {
     float* lse_I;             // [L]     natural-log lse of scale_I * I[t, 0..t]
     float* kl_part;           // [L][ntiles]: row partials of kl, one per key tile
     int kl_tile_log2;         // key tile of the partials: 64 or 128 keys
+    int* err;                 // the call's device error word (null: the per-device word)
     float* kl;                // [L]
     float* dq;                // [L][HI][DI]
     float* dk;                // [L][DI]

@@ -223,6 +223,7 @@ __device__ __forceinline__ void put_bf_tile(const BfPieces& P, uint32_t tile, in
 // Grid (HI, ceil(L / 128)): the heads of one query tile run side by side;
 // the longest query tiles first.
 __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) {
+    bind_error_word(p.err);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Misc* misc = reinterpret_cast<Misc*>(smem + kMisc);
@@ -461,6 +462,7 @@ constexpr uint32_t kIdescSt = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(k
 // Grid (nsplit, ceil(L / 128)): the groups of one key tile side by side; the
 // longest key tiles (the first) first.
 __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) {
+    bind_error_word(p.err);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Misc* misc = reinterpret_cast<Misc*>(smem + kDkMisc);
@@ -692,6 +694,7 @@ constexpr int kD = 128;                             // attention head dim of the
 // worker keeps an online max and sum over its half of the keys.  Grid (Hq,
 // ceil(L / 128)): the heads of a query tile side by side, longest first.
 __global__ void __launch_bounds__(kThreads, 1) head_lse_tc_kernel(const kl::Params p) {
+    bind_error_word(p.err);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Misc* misc = reinterpret_cast<Misc*>(smem + kFwdMisc);
@@ -857,6 +860,7 @@ static_assert(kTgtSmemBytes <= 232448, "shared memory per block");
 // written over I.  Tiles above the diagonal only write G = 0.  Grid (ntq
 // key tiles, ntq query tiles).  Needs Hkv <= 4.
 __global__ void __launch_bounds__(kThreads, 1) target_tc_kernel(const kl::Params p) {
+    bind_error_word(p.err);
     extern __shared__ uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kt = blockIdx.x, qt = blockIdx.y;

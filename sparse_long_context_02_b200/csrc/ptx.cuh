@@ -8,14 +8,25 @@
 
 namespace dsa {
 
-// Per-device error word (DSA_DEVERR_* codes; first error wins).
+// Device error words (DSA_DEVERR_* codes; the first error of a call wins).
+// A call records into the word its caller passed; a call given none records
+// into the library's per-device word.
 __device__ int g_dsa_device_error;
+
+// The word of the running kernel's call.  Every thread sets it at kernel
+// entry (all to the same value, so no barrier is needed before a thread
+// reads its own write).
+__shared__ int* s_dsa_error_word;
+
+__device__ __forceinline__ void bind_error_word(int* word) {
+    s_dsa_error_word = word != nullptr ? word : &g_dsa_device_error;
+}
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ void record_device_error(int code) {
-    atomicCAS(&g_dsa_device_error, 0, code);
+    atomicCAS(s_dsa_error_word, 0, code);
 }
 
 __device__ __forceinline__ uint64_t globaltimer() {

@@ -56,6 +56,7 @@ struct Params {
     int nsplit;               // index-row slices per sequence (decode)
     float* part_o;            // [B][nsplit][Hq][d]      unnormalised partial O
     float* part_ml;           // [B][nsplit][Hq][2]      running max (log2 units), sum
+    int* err;                 // the call's device error word (null: the per-device word)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -94,6 +95,7 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
 template <int D, int HKV, int G, bool SPLIT>
 __global__ void __launch_bounds__(Cfg<D, HKV>::THREADS)
 attn_kernel(const Params p) {
+    bind_error_word(p.err);
     pdl_wait();  // decode: the index rows come from the merge kernel
     pdl_launch_dependents();
     using C = Cfg<D, HKV>;

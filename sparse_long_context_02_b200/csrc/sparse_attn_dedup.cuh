@@ -75,6 +75,7 @@ __device__ __forceinline__ bool selected(const uint32_t* mask32, int pos, int nU
 template <int D, int HKV, int G>
 __global__ void __launch_bounds__(DedupCfg<D, HKV>::THREADS, 1)
 dedup_kernel(const Params p) {
+    bind_error_word(p.err);
     using C = DedupCfg<D, HKV>;
     constexpr int HQ = HKV * G;
     constexpr int NT = C::THREADS;

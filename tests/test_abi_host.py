@@ -31,7 +31,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for must in ("dsa_index_topk", "dsa_sparse_attn_prefill", "dsa_sparse_attn_decode",
-                 "dsa_index_scores", "dsa_decode_workspace_size", "dsa_device_error",
+                 "dsa_index_scores", "dsa_decode_workspace_size", "dsa_check_device_error",
                  "dsa_last_error", "dsa_status_string", "dsa_version"):
         assert must in names
 
@@ -57,32 +57,32 @@ FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails va
 
 def test_index_topk_rejects_bad_arguments(L):
     f = L.dsa_index_topk
-    assert f(None, FAKE, FAKE, 64, 4, 64, 8, FAKE, None) == INVALID
+    assert f(None, FAKE, FAKE, 64, 4, 64, 8, FAKE, None, None) == INVALID
     assert b"q_I is NULL" in L.dsa_last_error()
-    assert f(FAKE + 4, FAKE, FAKE, 64, 4, 64, 8, FAKE, None) == INVALID
+    assert f(FAKE + 4, FAKE, FAKE, 64, 4, 64, 8, FAKE, None, None) == INVALID
     assert b"aligned" in L.dsa_last_error()
-    assert f(FAKE, FAKE, FAKE, 0, 4, 64, 8, FAKE, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, 64, 4, 64, 0, FAKE, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, 64, 4, 64, 4096, FAKE, None) == UNSUPPORTED
-    assert f(FAKE, FAKE, FAKE, 64, 8, 64, 8, FAKE, None) == UNSUPPORTED
-    assert f(FAKE, FAKE, FAKE, 64, 64, 96, 8, FAKE, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 0, 4, 64, 8, FAKE, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 64, 4, 64, 0, FAKE, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 64, 4, 64, 4096, FAKE, None, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 64, 8, 64, 8, FAKE, None, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 64, 64, 96, 8, FAKE, None, None) == UNSUPPORTED
 
 
 def test_index_scores_rejects_bad_arguments(L):
     f = L.dsa_index_scores
-    assert f(FAKE, FAKE, None, 64, 4, 64, FAKE, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, 1 << 16, 4, 64, FAKE, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, 64, 16, 64, FAKE, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, None, 64, 4, 64, FAKE, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 1 << 16, 4, 64, FAKE, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 64, 16, 64, FAKE, None, None) == UNSUPPORTED
 
 
 def test_prefill_attention_rejects_bad_arguments(L):
     f = L.dsa_sparse_attn_prefill
     sc = ctypes.c_float(0.125)
-    assert f(FAKE, FAKE, FAKE, None, 64, 8, 2, 64, 16, sc, FAKE, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 3, 64, 16, sc, FAKE, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 64, 16, ctypes.c_float(-1.0), FAKE, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 96, 16, sc, FAKE, None) == UNSUPPORTED
-    assert f(FAKE, FAKE, FAKE, FAKE, 64, 16, 1, 64, 16, sc, FAKE, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, None, 64, 8, 2, 64, 16, sc, FAKE, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 3, 64, 16, sc, FAKE, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 64, 16, ctypes.c_float(-1.0), FAKE, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 96, 16, sc, FAKE, None, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 16, 1, 64, 16, sc, FAKE, None, None) == UNSUPPORTED
 
 
 def test_decode_rejects_bad_arguments_and_small_workspace(L):
@@ -91,20 +91,20 @@ def test_decode_rejects_bad_arguments_and_small_workspace(L):
     args = [FAKE] * 7 + [4, 40000, 64, 128, 32, 4, 128, 2048, sc, FAKE, None, FAKE]
     need = L.dsa_decode_workspace_size(4, 40000, 64, 128, 2048, 32, 4, 128)
     assert need > 0
-    assert f(*args, need - 1, None) == WORKSPACE
+    assert f(*args, need - 1, None, None) == WORKSPACE
     assert b"workspace" in L.dsa_last_error()
     bad = list(args)
     bad[0] = None
-    assert f(*bad, need, None) == INVALID
+    assert f(*bad, need, None, None) == INVALID
     bad = list(args)
     bad[7] = 0
-    assert f(*bad, need, None) == INVALID
+    assert f(*bad, need, None, None) == INVALID
     bad = list(args)
     bad[11] = 16  # Hq
-    assert f(*bad, need, None) == UNSUPPORTED
+    assert f(*bad, need, None, None) == UNSUPPORTED
     bad = list(args)
     bad[18] = FAKE + 16  # workspace not 256-byte aligned
-    assert f(*bad, need, None) == INVALID
+    assert f(*bad, need, None, None) == INVALID
 
 
 def test_indexer_kl_rejects_bad_arguments_and_small_workspaces(L):
@@ -115,48 +115,100 @@ def test_indexer_kl_rejects_bad_arguments_and_small_workspaces(L):
     assert need >= 300 * 32 * 4 + 300 * 4 + 300 * 5 * 4
     ws = 0x100000  # 256-byte aligned
     args = [FAKE] * 5 + [300, 64, 128, 32, 4, 128, sc, sI, FAKE, FAKE, ws]
-    assert f(*args, need - 1, None) == WORKSPACE
+    assert f(*args, need - 1, None, None) == WORKSPACE
     bad = list(args)
     bad[15] = ws + 16  # workspace not 256-byte aligned
-    assert f(*bad, need, None) == WORKSPACE
+    assert f(*bad, need, None, None) == WORKSPACE
     bad = list(args)
     bad[3] = None  # Q
-    assert f(*bad, need, None) == INVALID
+    assert f(*bad, need, None, None) == INVALID
     bad = list(args)
     bad[5] = 1 << 16  # L * L >= 2^31
-    assert f(*bad, need, None) == INVALID
+    assert f(*bad, need, None, None) == INVALID
     bad = list(args)
     bad[9] = 3  # Hkv does not divide Hq
-    assert f(*bad, need, None) == INVALID
+    assert f(*bad, need, None, None) == INVALID
     bad = list(args)
     bad[10] = 96  # d
-    assert f(*bad, need, None) == UNSUPPORTED
+    assert f(*bad, need, None, None) == UNSUPPORTED
     bad = list(args)
     bad[12] = ctypes.c_float(0.0)  # scale_I
-    assert f(*bad, need, None) == INVALID
+    assert f(*bad, need, None, None) == INVALID
     bad = list(args)
     bad[6], bad[7] = 16, 128  # an indexer shape the scorer does not have
-    assert f(*bad, need, None) == UNSUPPORTED
+    assert f(*bad, need, None, None) == UNSUPPORTED
 
     g = L.dsa_indexer_kl_backward
     nb = L.dsa_indexer_kl_backward_workspace_size(300, 64, 128)
     assert nb >= 8 * 300 * 128 * 4  # eight head groups of dk partials
     assert L.dsa_indexer_kl_backward_workspace_size(300, 11, 128) == 256  # one group: no partials
     bargs = [FAKE] * 4 + [300, 64, 128, FAKE, FAKE, FAKE, ws]
-    assert g(*bargs, nb - 1, None) == WORKSPACE
+    assert g(*bargs, nb - 1, None, None) == WORKSPACE
     bad = list(bargs)
     bad[5] = 0  # H_I
-    assert g(*bad, nb, None) == INVALID
+    assert g(*bad, nb, None, None) == INVALID
     bad = list(bargs)
     bad[6] = 96  # d_I
-    assert g(*bad, nb, None) == UNSUPPORTED
+    assert g(*bad, nb, None, None) == UNSUPPORTED
     bad = list(bargs)
     bad[3] = None  # G
-    assert g(*bad, nb, None) == INVALID
+    assert g(*bad, nb, None, None) == INVALID
 
 
-def test_device_error_rejects_null(L):
-    assert L.dsa_device_error(None, None) == INVALID
+def test_check_device_error_rejects_bad_arguments(L):
+    code = ctypes.c_int(0)
+    assert L.dsa_check_device_error(None, None, None) == INVALID
+    assert b"code is NULL" in L.dsa_last_error()
+    assert L.dsa_check_device_error(FAKE + 2, ctypes.byref(code), None) == INVALID
+    assert b"4-byte aligned" in L.dsa_last_error()
+
+
+def test_every_launching_call_rejects_a_misaligned_error_word(L):
+    """Each call takes its own device error word (4-byte aligned, or NULL for
+    the per-device word); a misaligned one is refused before any launch."""
+    sc = ctypes.c_float(0.125)
+    bad_err = FAKE + 2
+    calls = {
+        "dsa_index_topk": [FAKE, FAKE, FAKE, 64, 4, 64, 8, FAKE, bad_err, None],
+        "dsa_index_topk_varlen": [FAKE, FAKE, FAKE, FAKE, 1, 64, 4, 64, 8, FAKE, bad_err, None],
+        "dsa_index_scores": [FAKE, FAKE, FAKE, 64, 4, 64, FAKE, bad_err, None],
+        "dsa_sparse_attn_prefill": [FAKE] * 4 + [64, 8, 2, 64, 16, sc, FAKE, bad_err, None],
+        "dsa_sparse_attn_prefill_dedup": [FAKE] * 4 + [64, 8, 2, 64, 16, sc, FAKE, bad_err,
+                                                       None],
+        "dsa_prefill_from_host": [FAKE] * 15 + [64, 4, 64, 8, 2, 64, 16, sc, 128, bad_err, None,
+                                                 None, None],
+        "dsa_sparse_attn_decode": [FAKE] * 7 + [4, 40000, 64, 128, 32, 4, 128, 2048,
+                                                ctypes.c_float(0.088), FAKE, None, FAKE, 1 << 30,
+                                                bad_err, None],
+        "dsa_sparse_attn_decode_noalloc": [FAKE] * 7 + [4, 40000, 64, 128, 32, 4, 128, 2048,
+                                                        ctypes.c_float(0.088), FAKE, None,
+                                                        bad_err, None],
+        "dsa_indexer_kl_forward": [FAKE] * 5 + [300, 64, 128, 32, 4, 128, sc, sc, FAKE, FAKE,
+                                                0x100000, 1 << 30, bad_err, None],
+        "dsa_indexer_kl_backward": [FAKE] * 4 + [300, 64, 128, FAKE, FAKE, FAKE, 0x100000,
+                                                 1 << 30, bad_err, None],
+    }
+    for name, args in calls.items():
+        assert getattr(L, name)(*args) == INVALID, name
+        assert b"err is not 4-byte aligned" in L.dsa_last_error(), name
+
+
+def test_noalloc_checks_arguments_before_the_scratch_size(L):
+    """Bad or unsupported shapes get their own status, as from the decode with
+    a workspace; only a valid request too large for the built-in array gets
+    DSA_ERR_WORKSPACE."""
+    f = L.dsa_sparse_attn_decode_noalloc
+    sc = ctypes.c_float(0.088)
+    # B = 8192 (> 4096): invalid, although its scratch would also exceed 64 MiB
+    args = [FAKE] * 7 + [8192, 1 << 30, 64, 128, 32, 4, 128, 2048, sc, FAKE, None, None, None]
+    assert f(*args) == INVALID
+    # Hq = 16 with a large batch: unsupported, not a workspace error
+    args = [FAKE] * 7 + [4000, 1 << 30, 64, 128, 16, 4, 128, 2048, sc, FAKE, None, None, None]
+    assert f(*args) == UNSUPPORTED
+    # a valid shape whose scratch exceeds the array
+    args = [FAKE] * 7 + [4000, 1 << 30, 64, 128, 32, 4, 128, 2048, sc, FAKE, None, None, None]
+    assert f(*args) == WORKSPACE
+    assert b"64" in L.dsa_last_error() or b"array" in L.dsa_last_error()
 
 
 def test_missing_library_fails_loudly(monkeypatch):
@@ -201,3 +253,34 @@ def test_binding_checks_layout_before_the_call():
     with pytest.raises(ValueError, match="4-byte elements"):
         dsa._dev(torch.zeros(8, dtype=torch.float64).as_subclass(FakeCuda), "w", 4)
     assert dsa._dev(t, "x", 4) == t.data_ptr()
+
+
+def test_binding_host_input_prefill_errors_are_value_errors():
+    """prefill_from_host refuses a device tensor where a host one belongs, and
+    a call without its copy streams, with ValueError (before the library)."""
+    import torch
+
+    class FakeCuda(torch.Tensor):
+        @property
+        def is_cuda(self):
+            return True
+
+    L_, H, dI, Hq, Hkv, d = 64, 4, 64, 8, 2, 64
+    host = dict(q_I=torch.zeros((L_, H, dI), dtype=torch.uint8),
+                k_I=torch.zeros((L_, dI), dtype=torch.uint8),
+                w=torch.zeros((L_, H)), Q=torch.zeros((L_, Hq, d), dtype=torch.bfloat16),
+                K=torch.zeros((L_, Hkv, d), dtype=torch.bfloat16),
+                V=torch.zeros((L_, Hkv, d), dtype=torch.bfloat16),
+                O=torch.zeros((L_, Hq, d), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="h2d_stream"):
+        dsa.prefill_from_host(host, {}, 8, 0.125)
+    bad = dict(host, Q=host["Q"].as_subclass(FakeCuda))
+    with pytest.raises(ValueError, match="contiguous host tensor"):
+        dsa.prefill_from_host(bad, {}, 8, 0.125, h2d_stream=1, d2h_stream=2)
+
+
+def test_binding_error_word_must_be_int32():
+    import torch
+    with pytest.raises(ValueError, match="int32"):
+        dsa._err(torch.zeros(1, dtype=torch.int64))
+    assert dsa._err(None) is None

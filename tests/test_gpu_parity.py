@@ -168,6 +168,31 @@ def test_attention_empty_rows_are_zero_and_out_of_range_is_flagged():
     no_device_error()
 
 
+def test_error_words_of_concurrent_calls_are_separate():
+    """Two calls on two streams, each with its own device error word: the
+    call whose index row holds a key past the end flags DSA_DEVERR_INDEX in
+    its own word only; the clean call's word and the library's per-device
+    word stay 0."""
+    cfg = gen.custom(L=64, Hq=32, Hkv=4, d=128, seed=32)
+    Q, K, V = (dev(gen.prefill_Q(cfg), torch.bfloat16), dev(gen.prefill_K(cfg), torch.bfloat16),
+               dev(gen.prefill_V(cfg), torch.bfloat16))
+    good = np.full((64, 32), -1, np.int32)
+    good[:, 0] = np.arange(64)
+    bad = good.copy()
+    bad[20, 1] = 64  # one past the last key: skipped and flagged
+    good_d, bad_d = dev(good), dev(bad)
+    e_good, e_bad = dsa.error_word(), dsa.error_word()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        dsa.sparse_attn_prefill(Q, K, V, bad_d, cfg.scale, stream=s1, err=e_bad)
+        dsa.sparse_attn_prefill(Q, K, V, good_d, cfg.scale, stream=s2, err=e_good)
+    assert dsa.device_error(stream=s2, err=e_good) == dsa.DEVERR_NONE
+    assert dsa.device_error(stream=s1, err=e_bad) == dsa.DEVERR_INDEX
+    assert dsa.device_error(stream=s1, err=e_bad) == dsa.DEVERR_NONE  # read clears it
+    no_device_error()
+
+
 def test_prefill_end_to_end_tiny_workload():
     cfg = gen.TINY_PREFILL
     inp = gen.prefill_inputs(cfg)

@@ -53,12 +53,37 @@ def test_noalloc_decode_matches_workspace_decode(calls):
         assert err.max().item() <= MAX_ABS and err.mean().item() <= MEAN_ABS
 
 
+def test_noalloc_decode_without_index_output_and_changing_shapes():
+    """Calls whose index rows stay inside the shared scratch (idx_out None),
+    back to back with calls of another batch and another k: stale counts or
+    rows left by the previous call would show up as a difference from the
+    workspace decode."""
+    plan = [([40000, 7, 2048, 12345, 3], 3, 2048, False),
+            ([9000, 300000], 4, 512, True),
+            ([40000, 7, 2048, 12345, 3], 3, 2048, True),
+            ([65, 64, 63], 5, 64, False)]
+    for lens, seed, k, with_idx in plan:
+        cfg, args = _case(lens, seed)
+        B = len(lens)
+        ref_idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+        ref_O, _ = dsa.sparse_attn_decode(*args, k, cfg.scale, idx_out=ref_idx)
+        idx = torch.full((B, k), -7, dtype=torch.int32, device="cuda") if with_idx else None
+        O, _ = dsa.sparse_attn_decode_noalloc(*args, k, cfg.scale, idx_out=idx)
+        torch.cuda.synchronize()
+        assert dsa.device_error() == dsa.DEVERR_NONE
+        if with_idx:
+            assert torch.equal(idx, ref_idx)
+        err = (O.float() - ref_O.float()).abs()
+        assert err.max().item() <= MAX_ABS and err.mean().item() <= MEAN_ABS, (lens, k)
+
+
 def test_noalloc_decode_rejects_sizes_beyond_its_scratch():
     L = dsa.lib()
     need = L.dsa_decode_workspace_size(4096, 1 << 30, 64, 128, 2048, 32, 4, 128)
     assert need > 64 << 20
     fake = 0x10000
     st = L.dsa_sparse_attn_decode_noalloc(fake, fake, fake, fake, fake, fake, fake, 4096, 1 << 30,
-                                          64, 128, 32, 4, 128, 2048, 0.088, fake, None, None)
+                                          64, 128, 32, 4, 128, 2048, 0.088, fake, None, None,
+                                          None)
     assert st == 3  # DSA_ERR_WORKSPACE, before any launch
     assert b"built-in array" in L.dsa_last_error()
