@@ -72,6 +72,9 @@ def forward(Q, K, V, idx, scale: float) -> np.ndarray:
 def backward(Q, K, V, idx, dO, scale: float, magnitudes: bool = False) -> Dict[str, np.ndarray]:
     """dQ [L][Hq][d], dK and dV [n][Hkv][d] (float64) of sum(dO * O).
 
+    Rows of one KV group are handled together (they share the selected K and
+    V rows); each head's softmax is its own row of the [G][m] arrays.
+
     With ``magnitudes``, also the sums of the absolute values of the terms
     behind each output element (what a rounding of the operands perturbs):
     mQ = scale * sum |dS| |K| (+ P E |K|), mK = scale * sum |dS| |Q| (+ P E |Q|),
@@ -89,24 +92,24 @@ def backward(Q, K, V, idx, dO, scale: float, magnitudes: bool = False) -> Dict[s
         s = _rows(idx, t, n)
         if s.size == 0:
             continue
-        for h in range(Hq):
-            g = h // G
-            Ks, Vs = K[s, g, :], V[s, g, :]
-            x = scale * (Ks @ Q[t, h])
-            p = np.exp(x - x.max())
-            p /= p.sum()
-            dp = Vs @ dO[t, h]
-            D = p @ dp
+        for g in range(Hkv):
+            hs = slice(g * G, (g + 1) * G)          # the query heads of group g
+            Ks, Vs = K[s, g, :], V[s, g, :]         # [m][d]
+            x = scale * (Q[t, hs] @ Ks.T)           # [G][m]
+            p = np.exp(x - x.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            dp = dO[t, hs] @ Vs.T                   # [G][m]
+            D = (p * dp).sum(axis=1, keepdims=True)
             ds = p * (dp - D)
-            dQ[t, h] = scale * (ds @ Ks)
-            np.add.at(dK[:, g, :], s, scale * np.outer(ds, Q[t, h]))
-            np.add.at(dV[:, g, :], s, np.outer(p, dO[t, h]))
+            dQ[t, hs] = scale * (ds @ Ks)
+            np.add.at(dK[:, g, :], s, scale * (ds.T @ Q[t, hs]))
+            np.add.at(dV[:, g, :], s, p.T @ dO[t, hs])
             if magnitudes:
-                E = np.abs(dO[t, h]) @ np.abs(p @ Vs)
+                E = (np.abs(dO[t, hs]) * np.abs(p @ Vs)).sum(axis=1, keepdims=True)
                 a = np.abs(ds) + p * E
-                mQ[t, h] = scale * (a @ np.abs(Ks))
-                np.add.at(mK[:, g, :], s, scale * np.outer(a, np.abs(Q[t, h])))
-                np.add.at(mV[:, g, :], s, np.outer(p, np.abs(dO[t, h])))
+                mQ[t, hs] = scale * (a @ np.abs(Ks))
+                np.add.at(mK[:, g, :], s, scale * (a.T @ np.abs(Q[t, hs])))
+                np.add.at(mV[:, g, :], s, p.T @ np.abs(dO[t, hs]))
     out = dict(dQ=dQ, dK=dK, dV=dV)
     if magnitudes:
         out.update(mQ=mQ, mK=mK, mV=mV)

@@ -150,14 +150,18 @@ def test_magnitudes_bound_the_gradients():
 MUTATIONS = {
     "row term D dropped": ("ds = p * (dp - D)", "ds = p * dp"),
     "softmax-backward sign": ("ds = p * (dp - D)", "ds = p * (D - dp)"),
-    "scale missing in dK": ("np.add.at(dK[:, g, :], s, scale * np.outer(ds, Q[t, h]))",
-                            "np.add.at(dK[:, g, :], s, np.outer(ds, Q[t, h]))"),
-    "scale missing in dQ": ("dQ[t, h] = scale * (ds @ Ks)", "dQ[t, h] = ds @ Ks"),
-    "dV from dS": ("np.add.at(dV[:, g, :], s, np.outer(p, dO[t, h]))",
-                   "np.add.at(dV[:, g, :], s, np.outer(ds, dO[t, h]))"),
-    "gqa group h % Hkv": ("            g = h // G\n            Ks, Vs", "            g = h % Hkv\n            Ks, Vs"),
-    "repeated keys counted once": ("np.add.at(dK[:, g, :], s, scale", "dK[s, g, :] += (scale"),
+    "scale missing in dK": ("np.add.at(dK[:, g, :], s, scale * (ds.T @ Q[t, hs]))",
+                            "np.add.at(dK[:, g, :], s, ds.T @ Q[t, hs])"),
+    "scale missing in dQ": ("dQ[t, hs] = scale * (ds @ Ks)", "dQ[t, hs] = ds @ Ks"),
+    "dV from dS": ("np.add.at(dV[:, g, :], s, p.T @ dO[t, hs])",
+                   "np.add.at(dV[:, g, :], s, ds.T @ dO[t, hs])"),
+    "gqa heads of the wrong group": ("hs = slice(g * G, (g + 1) * G)",
+                                     "hs = slice(g, Hq, Hkv)"),
+    "repeated keys counted once": ("np.add.at(dK[:, g, :], s, scale * (ds.T @ Q[t, hs]))",
+                                   "dK[s, g, :] += scale * (ds.T @ Q[t, hs])"),
     "out-of-range entries kept": ("return r[(r >= 0) & (r < n)]", "return r[r >= 0] % n"),
+    "softmax over heads": ("p /= p.sum(axis=1, keepdims=True)\n            dp",
+                           "p /= p.sum(axis=0, keepdims=True)\n            dp"),
 }
 
 
@@ -165,10 +169,7 @@ def _mutant(name):
     old, new = MUTATIONS[name]
     src = open(AB.__file__).read()
     assert old in src, f"mutation site not found: {name}"
-    if name == "repeated keys counted once":
-        src = src.replace(old, new).replace(", np.outer(ds, Q[t, h]))", " * np.outer(ds, Q[t, h]))", 1)
-    else:
-        src = src.replace(old, new)
+    src = src.replace(old, new)
     spec = importlib.util.spec_from_loader("oracle.attn_bwd_mut", loader=None,
                                            origin=AB.__file__)
     mod = importlib.util.module_from_spec(spec)
