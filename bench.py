@@ -62,6 +62,10 @@ def parse():
                     help="instead of timing: run the prefill indexer once and report how many "
                          "distinct keys the index rows of G consecutive queries select together "
                          "(the traffic an adjacent-query dedup would read)")
+    ap.add_argument("--attn-bwd", action="store_true",
+                    help="instead of the inference step: time the sparse attention's training "
+                         "pass (forward with lse, then dsa_sparse_attn_backward) on the prefill "
+                         "workload's index rows")
     ap.add_argument("--kl", type=int, default=0, metavar="L",
                     help="instead of the inference step: time the indexer warm-up KL loss "
                          "(forward: loss and dL/dI; backward: dq_I, dk_I, dw) at sequence "
@@ -637,6 +641,86 @@ def kl_bench(args) -> dict:
                 clocks=ck, mean_kl=float(kl.mean().item()))
 
 
+def attn_bwd_bytes(cfg) -> float:
+    """Backward traffic the method itself implies: per selected row the K and
+    V rows gathered (2 * Hkv * d * 2 B) and the fp32 reductions into dK and
+    dV (2 * Hkv * d * 4 B); per token Q, O and dO (3 * Hq * d * 2 B), lse
+    (Hq * 4 B), the index row (4 k B) and dQ (Hq * d * 4 B)."""
+    L, k = cfg.L, cfg.k
+    sel = k * L - k * (k - 1) / 2.0 if L >= k else L * (L + 1) / 2.0
+    row = 2 * cfg.Hkv * cfg.d * (2 + 4)
+    per_tok = 3 * cfg.Hq * cfg.d * 2 + cfg.Hq * 4 + 4 * k + cfg.Hq * cfg.d * 4
+    return sel * row + L * per_tok
+
+
+def attn_bwd_bench(args) -> dict:
+    """Times the forward (with lse) and dsa_sparse_attn_backward on the prefill
+    workload's own index rows (from dsa_index_topk) with a seeded dO; L2
+    flushed before each timed call."""
+    import torch
+    import sparse_long_context_02_b200 as dsa
+    cfg = gen.CONFIGS[args.prefill_config]
+    host = gen.prefill_inputs(cfg)
+    t = {n: torch.from_numpy(host[n]).cuda() for n in ("q_I", "k_I", "w")}
+    bf = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).cuda()
+          for n in ("Q", "K", "V")}
+    idx = dsa.index_topk(t["q_I"], t["k_I"], t["w"], cfg.k)
+    dO = torch.from_numpy(gen.normal_bf16(cfg.seed_ + 777, 99, 0, bf["Q"].numel()).view(
+        np.int16)).view(torch.bfloat16).reshape(bf["Q"].shape).cuda()
+    O = torch.empty_like(bf["Q"])
+    lse = torch.empty((cfg.L, cfg.Hq), dtype=torch.float32, device="cuda")
+    dQ = torch.empty((cfg.L, cfg.Hq, cfg.d), dtype=torch.float32, device="cuda")
+    dK = torch.empty((cfg.L, cfg.Hkv, cfg.d), dtype=torch.float32, device="cuda")
+    dV = torch.empty_like(dK)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def fwd():
+        dsa.sparse_attn_prefill(bf["Q"], bf["K"], bf["V"], idx, cfg.scale, O=O, lse=lse)
+
+    def bwd():
+        dsa.sparse_attn_backward(bf["Q"], bf["K"], bf["V"], idx, O, lse, dO, cfg.scale,
+                                 dQ=dQ, dK=dK, dV=dV)
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    clocks = Clocks(torch.cuda.current_device())
+    clocks.start()
+    tf, tb = [], []
+    for _ in range(args.steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.zero_()
+        ev[0].record()
+        fwd()
+        ev[1].record()
+        flush.zero_()
+        ev[2].record()
+        bwd()
+        ev[3].record()
+        torch.cuda.synchronize()
+        tf.append(ev[0].elapsed_time(ev[1]))
+        tb.append(ev[2].elapsed_time(ev[3]))
+    ck = clocks.stop()
+    if dsa.device_error() != dsa.DEVERR_NONE:
+        raise RuntimeError("device error in the attention backward")
+    pk = peaks()
+    ms_b = float(np.mean(tb))
+    work = attn_bwd_bytes(cfg)
+    return dict(metric="sparse attention backward query-tokens/s", value=cfg.L / (ms_b * 1e-3),
+                unit="query-tokens/s", higher_is_better=True, steps=args.steps,
+                warmup=args.warmup, dtype="bf16/fp32", data="synthetic",
+                config=dict(workload=cfg.name + " (attention backward)", L=cfg.L, k=cfg.k,
+                            Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d,
+                            l2="flushed before each timed call (256 MiB write)"),
+                forward_ms=float(np.mean(tf)), backward_ms=ms_b,
+                roofline=dict(bound="hbm", achieved=work / (ms_b * 1e-3) / 1e9, peak=pk["hbm"],
+                              unit="GB/s", frac=work / (ms_b * 1e-3) / 1e9 / pk["hbm"],
+                              traffic=None, kernel="dsa_sparse_attn_backward",
+                              work_bytes=work, peak_source=pk["src"] + " (hbm copy)"),
+                clocks=ck, gpu_launches=3 * args.steps)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -654,6 +738,10 @@ def main():
     if args.kl:
         if rank == 0:
             print(json.dumps(kl_bench(args)), flush=True)
+        return
+    if args.attn_bwd:
+        if rank == 0:
+            print(json.dumps(attn_bwd_bench(args)), flush=True)
         return
 
     import datetime

@@ -196,12 +196,48 @@ DSA_API dsa_status_t dsa_index_scores(const void* q_I, const void* k_I, const fl
  *                            an entry >= L is skipped and flagged
  *                            DSA_DEVERR_INDEX
  *   O    [L][Hq][d]   bf16   OUT (a row with no valid entry is all zeros)
+ *   lse  [L][Hq]      fp32   OUT or NULL: natural log of each row's softmax
+ *                            normaliser, log sum_s exp(scale Q[t,h] . K[s,g])
+ *                            (-inf for a row with no valid entry); the
+ *                            backward's input
  * Supported: d in {64, 128}; (Hkv, Hq/Hkv) in {(2, 4), (4, 8)}; k <= 65536.
  */
 DSA_API dsa_status_t dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
                                      const int32_t* idx, int64_t L, int Hq, int Hkv, int d,
-                                     int k, float scale, void* O, int32_t* err,
+                                     int k, float scale, void* O, float* lse, int32_t* err,
                                      dsa_stream_t stream);
+
+/*
+ * dsa_sparse_attn_backward - gradients of a loss through the sparse GQA
+ * attention (the sparse-adaptation training stage: Kwai Keye-VL-2.0
+ * technical-report summary, section 1 -- every parameter is trained on the
+ * next-token loss through the truly sparse attention; the index rows are
+ * fixed).  With P[t,h,i] = exp(scale Q[t,h] . K[s_i,g] - lse[t,h]) over the
+ * valid entries s_i of idx[t] and g = h / (Hq / Hkv):
+ *   dP = dO[t,h] . V[s_i,g],  D = dO[t,h] . O[t,h],  dS = P (dP - D)
+ *   dQ[t,h]   = scale sum_i dS K[s_i,g]
+ *   dK[s,g]   = scale sum over (t, h in g, i with s_i = s) of dS Q[t,h]
+ *   dV[s,g]   = sum over the same of P dO[t,h]
+ * (an index entry that repeats a key counts once per entry, as in the
+ * forward).
+ *
+ *   Q, K, V, idx    as dsa_sparse_attn_prefill
+ *   O    [L][Hq][d]   bf16   the forward's output
+ *   lse  [L][Hq]      fp32   the forward's lse output
+ *   dO   [L][Hq][d]   bf16   gradient of the loss with respect to O
+ *   dQ   [L][Hq][d]   fp32   OUT
+ *   dK, dV [L][Hkv][d] fp32  OUT (overwritten: the call clears them, then
+ *                            accumulates every selecting row's share)
+ * dS and P are rounded to bf16 for their products (fp32 accumulation).  dQ
+ * is deterministic; dK and dV are sums of fp32 reductions whose order varies
+ * from run to run (results agree to rounding).  Supported shapes as
+ * dsa_sparse_attn_prefill.
+ */
+DSA_API dsa_status_t dsa_sparse_attn_backward(const void* Q, const void* K, const void* V,
+                                      const int32_t* idx, const void* O, const float* lse,
+                                      const void* dO, int64_t L, int Hq, int Hkv, int d, int k,
+                                      float scale, float* dQ, float* dK, float* dV,
+                                      int32_t* err, dsa_stream_t stream);
 
 /*
  * dsa_decode_workspace_size - bytes of device workspace that

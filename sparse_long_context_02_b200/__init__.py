@@ -60,7 +60,10 @@ def lib() -> ctypes.CDLL:
         L.dsa_index_topk_varlen.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp]
         L.dsa_sparse_attn_prefill.restype = i32
         L.dsa_sparse_attn_prefill.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, f32, vp,
-                                              vp, vp]
+                                              vp, vp, vp]
+        L.dsa_sparse_attn_backward.restype = i32
+        L.dsa_sparse_attn_backward.argtypes = [vp] * 7 + [i64, i32, i32, i32, i32, f32, vp, vp,
+                                                          vp, vp, vp]
         L.dsa_decode_workspace_size.restype = sz
         L.dsa_decode_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32, i32]
         L.dsa_sparse_attn_decode.restype = i32
@@ -179,9 +182,10 @@ def index_scores(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor,
 
 def sparse_attn_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, idx: torch.Tensor,
                         scale: float, O: Optional[torch.Tensor] = None,
-                        stream=None, err=None) -> torch.Tensor:
+                        stream=None, err=None, lse: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Sparse GQA attention.  Q [L][Hq][d], K/V [L][Hkv][d] bf16, idx [L][k]
-    int32 -> O [L][Hq][d] bf16."""
+    int32 -> O [L][Hq][d] bf16.  With `lse` (a [L][Hq] float32 tensor), also
+    each row's log-sum-exp, the input of sparse_attn_backward."""
     L, Hq, d = Q.shape
     Hkv = K.shape[1]
     k = idx.shape[1]
@@ -189,9 +193,35 @@ def sparse_attn_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, idx: 
         O = torch.empty_like(Q)
     _check(lib().dsa_sparse_attn_prefill(_dev(Q, "Q", 2), _dev(K, "K", 2), _dev(V, "V", 2),
                                          _dev(idx, "idx", 4), L, Hq, Hkv, d, k, float(scale),
-                                         _dev(O, "O", 2), _err(err), _stream(stream)),
+                                         _dev(O, "O", 2),
+                                         _dev(lse, "lse", 4) if lse is not None else None,
+                                         _err(err), _stream(stream)),
            "dsa_sparse_attn_prefill")
     return O
+
+
+def sparse_attn_backward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, idx: torch.Tensor,
+                         O: torch.Tensor, lse: torch.Tensor, dO: torch.Tensor, scale: float,
+                         dQ: Optional[torch.Tensor] = None, dK: Optional[torch.Tensor] = None,
+                         dV: Optional[torch.Tensor] = None, stream=None, err=None):
+    """Gradients through the sparse attention.  Q, K, V, idx as
+    sparse_attn_prefill; O and lse the forward's outputs; dO [L][Hq][d] bf16.
+    Returns (dQ [L][Hq][d], dK [L][Hkv][d], dV [L][Hkv][d]), float32."""
+    L, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    k = idx.shape[1]
+    if dQ is None:
+        dQ = torch.empty((L, Hq, d), dtype=torch.float32, device=Q.device)
+    if dK is None:
+        dK = torch.empty((L, Hkv, d), dtype=torch.float32, device=Q.device)
+    if dV is None:
+        dV = torch.empty((L, Hkv, d), dtype=torch.float32, device=Q.device)
+    _check(lib().dsa_sparse_attn_backward(
+        _dev(Q, "Q", 2), _dev(K, "K", 2), _dev(V, "V", 2), _dev(idx, "idx", 4), _dev(O, "O", 2),
+        _dev(lse, "lse", 4), _dev(dO, "dO", 2), L, Hq, Hkv, d, k, float(scale),
+        _dev(dQ, "dQ", 4), _dev(dK, "dK", 4), _dev(dV, "dV", 4), _err(err), _stream(stream)),
+        "dsa_sparse_attn_backward")
+    return dQ, dK, dV
 
 
 def _host(t: torch.Tensor, name: str) -> int:

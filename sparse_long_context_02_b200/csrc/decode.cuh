@@ -167,7 +167,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     const int64_t r1 = r0 + p.R < p.total_n ? r0 + p.R : p.total_n;
     if (r0 >= r1) return;  // more CTAs than ranges: nothing to do
 
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    extern __shared__ __align__(16) uint8_t smem_raw[];
     // Aligned by pointer arithmetic on the shared array itself (not through an
     // integer), so that the compiler keeps every access in the shared window
     // (ld/st.shared with 32-bit addresses instead of generic ones).

@@ -17,6 +17,7 @@
 #include "sparse_attn_dedup.cuh"
 #include "index_topk.cuh"
 #include "sparse_attn.cuh"
+#include "sparse_attn_bwd.cuh"
 #include "indexer_kl.cuh"
 #include "indexer_kl_tc.cuh"
 
@@ -218,8 +219,8 @@ dsa_status_t launch_dedup(const char* fn, const dsa::attn::Params& p, int64_t L,
 // checked by the caller).
 dsa_status_t attn_prefill_rows(const char* fn, const void* Q, const void* K, const void* V,
                                const int32_t* idx, int64_t L, int Hq, int Hkv, int d, int k,
-                               float scale, void* O, int64_t row0, int64_t row1, int* err,
-                               cudaStream_t st) {
+                               float scale, void* O, float* lse, int64_t row0, int64_t row1,
+                               int* err, cudaStream_t st) {
     const int G = Hq / Hkv;
     dsa::attn::Params p{};
     p.Q = static_cast<const __nv_bfloat16*>(Q) + row0 * Hq * d;
@@ -230,6 +231,7 @@ dsa_status_t attn_prefill_rows(const char* fn, const void* Q, const void* K, con
     p.k = k;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.O = static_cast<__nv_bfloat16*>(O) + row0 * Hq * d;
+    p.lse = lse != nullptr ? lse + row0 * Hq : nullptr;
     p.err = err;
     const int64_t rows = row1 - row0;
     if (d == 128 && Hkv == 4 && G == 8) return launch_attn<128, 4, 8, false>(fn, p, rows, st);
@@ -406,7 +408,8 @@ dsa_status_t dsa_prefill_from_host(const void* q_I_h, const void* k_I_h, const f
         dsa_status_t r = dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, nullptr,
                                               1, err, st, r0, r1);
         if (r != DSA_OK) return r;
-        r = attn_prefill_rows(fn, Q, K, V, idx, L, Hq, Hkv, d, k, scale, O, r0, r1, err, st);
+        r = attn_prefill_rows(fn, Q, K, V, idx, L, Hq, Hkv, d, k, scale, O, nullptr, r0, r1, err,
+                              st);
         if (r != DSA_OK) return r;
         CUDA_TRY(cudaEventRecord(ev[2 * c + 1], st));
         CUDA_TRY(cudaStreamWaitEvent(sd, ev[2 * c + 1], 0));
@@ -435,7 +438,7 @@ dsa_status_t dsa_index_scores(const void* q_I, const void* k_I, const float* w, 
 
 dsa_status_t dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
                                      const int32_t* idx, int64_t L, int Hq, int Hkv, int d,
-                                     int k, float scale, void* O, int32_t* err,
+                                     int k, float scale, void* O, float* lse, int32_t* err,
                                      dsa_stream_t stream) {
     static const char fn[] = "dsa_sparse_attn_prefill";
     CHECK_PTR(Q);
@@ -448,8 +451,84 @@ dsa_status_t dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V
     if (k < 1 || k > 65536) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
     if (Hkv < 1 || Hq < 1 || Hq % Hkv) return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d", fn, Hq, Hkv);
     if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
-    const dsa_status_t r = attn_prefill_rows(fn, Q, K, V, idx, L, Hq, Hkv, d, k, scale, O, 0, L,
-                                             err, static_cast<cudaStream_t>(stream));
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: lse is not 4-byte aligned", fn);
+    const dsa_status_t r = attn_prefill_rows(fn, Q, K, V, idx, L, Hq, Hkv, d, k, scale, O, lse, 0,
+                                             L, err, static_cast<cudaStream_t>(stream));
+    return r == DSA_OK ? ok() : r;
+}
+
+}  // extern "C"
+
+namespace {
+
+template <int D, int HKV, int G>
+dsa_status_t launch_attn_bwd(const char* fn, const dsa::attn::BwdParams& p, int64_t L,
+                             cudaStream_t st) {
+    using C = dsa::attn::Cfg<D, HKV>;
+    auto kern = dsa::attn::attn_bwd_kernel<D, HKV, G>;
+    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    kern<<<(unsigned)L, C::THREADS, C::SMEM, st>>>(p);
+    CUDA_TRY(cudaGetLastError());
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_sparse_attn_backward(const void* Q, const void* K, const void* V,
+                                      const int32_t* idx, const void* O, const float* lse,
+                                      const void* dO, int64_t L, int Hq, int Hkv, int d, int k,
+                                      float scale, float* dQ, float* dK, float* dV, int32_t* err,
+                                      dsa_stream_t stream) {
+    static const char fn[] = "dsa_sparse_attn_backward";
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(idx);
+    CHECK_PTR(O);
+    CHECK_PTR(lse);
+    CHECK_PTR(dO);
+    CHECK_PTR(dQ);
+    CHECK_PTR(dK);
+    CHECK_PTR(dV);
+    CHECK_ERR_WORD(err);
+    if (L < 1 || L > (int64_t(1) << 30)) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
+    if (k < 1 || k > 65536) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (Hkv < 1 || Hq < 1 || Hq % Hkv) return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d", fn, Hq, Hkv);
+    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
+    const int G = Hq / Hkv;
+    const bool shape_ok = (d == 128 && Hkv == 4 && G == 8) || (d == 64 && Hkv == 2 && G == 4) ||
+                          (d == 128 && Hkv == 2 && G == 4) || (d == 64 && Hkv == 4 && G == 8);
+    if (!shape_ok)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: (d, Hkv, Hq/Hkv) = (%d, %d, %d)", fn, d, Hkv, G);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // dK and dV are sums of reductions from every row that selects the key
+    const size_t kv_bytes = (size_t)L * Hkv * d * sizeof(float);
+    CUDA_TRY(cudaMemsetAsync(dK, 0, kv_bytes, st));
+    CUDA_TRY(cudaMemsetAsync(dV, 0, kv_bytes, st));
+    dsa::attn::BwdParams p{};
+    p.Q = static_cast<const __nv_bfloat16*>(Q);
+    p.K = static_cast<const __nv_bfloat16*>(K);
+    p.V = static_cast<const __nv_bfloat16*>(V);
+    p.O = static_cast<const __nv_bfloat16*>(O);
+    p.dO = static_cast<const __nv_bfloat16*>(dO);
+    p.lse = lse;
+    p.idx = idx;
+    p.nkeys = L;
+    p.k = k;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.dQ = dQ;
+    p.dK = dK;
+    p.dV = dV;
+    p.err = err;
+    dsa_status_t r;
+    if (d == 128 && Hkv == 4 && G == 8) r = launch_attn_bwd<128, 4, 8>(fn, p, L, st);
+    else if (d == 64 && Hkv == 2 && G == 4) r = launch_attn_bwd<64, 2, 4>(fn, p, L, st);
+    else if (d == 128 && Hkv == 2 && G == 4) r = launch_attn_bwd<128, 2, 4>(fn, p, L, st);
+    else r = launch_attn_bwd<64, 4, 8>(fn, p, L, st);
     return r == DSA_OK ? ok() : r;
 }
 

@@ -210,7 +210,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     static_assert(N % 16 == 0 && N <= 256, "MMA N");
     static_assert(DI == 64 || DI == 128, "d_I");
 
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    extern __shared__ __align__(16) uint8_t smem_raw[];
     // Aligned by pointer arithmetic on the shared array itself (not through an
     // integer), so that the compiler keeps every access in the shared window
     // (ld/st.shared with 32-bit addresses instead of generic ones).

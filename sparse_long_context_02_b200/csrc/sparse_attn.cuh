@@ -52,6 +52,7 @@ struct Params {
     int k;
     float scale_log2;         // softmax scale * log2(e)
     __nv_bfloat16* O;         // [rows][Hq][d]           (prefill)
+    float* lse;               // [rows][Hq] or null      (prefill) natural-log softmax normaliser
     const int64_t* cache_off; // [B + 1]                 (decode)
     int nsplit;               // index-row slices per sequence (decode)
     float* part_o;            // [B][nsplit][Hq][d]      unnormalised partial O
@@ -101,7 +102,7 @@ attn_kernel(const Params p) {
     using C = Cfg<D, HKV>;
     constexpr int HQ = HKV * G;
     static_assert(G <= 8, "at most 8 query heads per KV group");
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(16) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::STAGE);
     uint64_t* empty = full + kStages;
     uint32_t* mask = reinterpret_cast<uint32_t*>(empty + kStages);
@@ -321,6 +322,9 @@ attn_kernel(const Params p) {
         }
     } else {
         const float inv = l > 0.f ? 1.f / l : 0.f;
+        if (p.lse != nullptr && (lane & 3) == 0)
+            p.lse[(int64_t)orow * HQ + h] =
+                l > 0.f ? (m_run + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         __nv_bfloat16* out = p.O + ((int64_t)orow * HQ + h) * D;
 #pragma unroll
         for (int n = 0; n < D / 8; ++n)

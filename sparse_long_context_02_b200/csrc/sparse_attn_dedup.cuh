@@ -80,7 +80,7 @@ dedup_kernel(const Params p) {
     constexpr int HQ = HKV * G;
     constexpr int NT = C::THREADS;
     static_assert(G <= 8, "at most 8 query heads per KV group");
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(16) uint8_t smem[];
     uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem);  // phase 1 only
     int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
     int32_t* U = reinterpret_cast<int32_t*>(smem + C::OFF_U);

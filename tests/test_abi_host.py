@@ -78,11 +78,31 @@ def test_index_scores_rejects_bad_arguments(L):
 def test_prefill_attention_rejects_bad_arguments(L):
     f = L.dsa_sparse_attn_prefill
     sc = ctypes.c_float(0.125)
-    assert f(FAKE, FAKE, FAKE, None, 64, 8, 2, 64, 16, sc, FAKE, None, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 3, 64, 16, sc, FAKE, None, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 64, 16, ctypes.c_float(-1.0), FAKE, None, None) == INVALID
-    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 96, 16, sc, FAKE, None, None) == UNSUPPORTED
-    assert f(FAKE, FAKE, FAKE, FAKE, 64, 16, 1, 64, 16, sc, FAKE, None, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, None, 64, 8, 2, 64, 16, sc, FAKE, None, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 3, 64, 16, sc, FAKE, None, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 64, 16, ctypes.c_float(-1.0), FAKE, None, None, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 8, 2, 96, 16, sc, FAKE, None, None, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 64, 16, 1, 64, 16, sc, FAKE, None, None, None) == UNSUPPORTED
+
+
+def test_attention_backward_rejects_bad_arguments(L):
+    f = L.dsa_sparse_attn_backward
+    sc = ctypes.c_float(0.125)
+    args = [FAKE] * 7 + [64, 8, 2, 64, 16, sc, FAKE, FAKE, FAKE, None, None]
+    bad = list(args)
+    bad[5] = None  # lse
+    assert f(*bad) == INVALID
+    assert b"lse is NULL" in L.dsa_last_error()
+    bad = list(args)
+    bad[9] = 3  # Hkv does not divide Hq
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[10] = 96  # d
+    assert f(*bad) == UNSUPPORTED
+    bad = list(args)
+    bad[12] = ctypes.c_float(0.0)
+    assert f(*bad) == INVALID
+    assert f(*(args[:7] + [64, 16, 1, 64, 16, sc] + args[13:])) == UNSUPPORTED
 
 
 def test_decode_rejects_bad_arguments_and_small_workspace(L):
@@ -172,7 +192,9 @@ def test_every_launching_call_rejects_a_misaligned_error_word(L):
         "dsa_index_topk": [FAKE, FAKE, FAKE, 64, 4, 64, 8, FAKE, bad_err, None],
         "dsa_index_topk_varlen": [FAKE, FAKE, FAKE, FAKE, 1, 64, 4, 64, 8, FAKE, bad_err, None],
         "dsa_index_scores": [FAKE, FAKE, FAKE, 64, 4, 64, FAKE, bad_err, None],
-        "dsa_sparse_attn_prefill": [FAKE] * 4 + [64, 8, 2, 64, 16, sc, FAKE, bad_err, None],
+        "dsa_sparse_attn_prefill": [FAKE] * 4 + [64, 8, 2, 64, 16, sc, FAKE, None, bad_err, None],
+        "dsa_sparse_attn_backward": [FAKE] * 7 + [64, 8, 2, 64, 16, sc, FAKE, FAKE, FAKE, bad_err,
+                                                  None],
         "dsa_sparse_attn_prefill_dedup": [FAKE] * 4 + [64, 8, 2, 64, 16, sc, FAKE, bad_err,
                                                        None],
         "dsa_prefill_from_host": [FAKE] * 15 + [64, 4, 64, 8, 2, 64, 16, sc, 128, bad_err, None,
