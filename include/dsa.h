@@ -125,6 +125,38 @@ DSA_API dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, con
                                    dsa_stream_t stream);
 
 /*
+ * dsa_index_topk_rows - dsa_index_topk for the query rows [row0, row1) only:
+ * one rank's share when the query tokens of one long sequence are split
+ * across GPUs (each query's selection needs every earlier key, so the keys
+ * are gathered to every rank first; the rows themselves are independent).
+ * Row t's result equals row t of dsa_index_topk over the whole sequence.
+ *
+ *   q_I  [row1-row0][H_I][d_I]  e4m3   the rows' indexer queries
+ *   k_I  [row1][d_I]            e4m3   keys 0 .. row1-1
+ *   w    [row1-row0][H_I]       fp32
+ *   idx  [row1-row0][k]         int32  OUT, as dsa_index_topk
+ * row0 must be a multiple of 4 (the indexer's query block).  Same shape
+ * support as dsa_index_topk.
+ */
+DSA_API dsa_status_t dsa_index_topk_rows(const void* q_I, const void* k_I, const float* w,
+                                 int64_t row0, int64_t row1, int H_I, int d_I, int k,
+                                 int32_t* idx, int32_t* err, dsa_stream_t stream);
+
+/*
+ * dsa_sparse_attn_rows - dsa_sparse_attn_prefill for nrows query rows whose
+ * index rows select among nkeys keys (the query rows of one rank; keys are
+ * positions in K and V).
+ *
+ *   Q    [nrows][Hq][d]  bf16;   K, V [nkeys][Hkv][d] bf16
+ *   idx  [nrows][k]      int32;  O [nrows][Hq][d] bf16 OUT;  lse [nrows][Hq] OUT or NULL
+ * Same shape support as dsa_sparse_attn_prefill.
+ */
+DSA_API dsa_status_t dsa_sparse_attn_rows(const void* Q, const void* K, const void* V,
+                                  const int32_t* idx, int64_t nrows, int64_t nkeys, int Hq,
+                                  int Hkv, int d, int k, float scale, void* O, float* lse,
+                                  int32_t* err, dsa_stream_t stream);
+
+/*
  * dsa_sparse_attn_prefill_dedup - the result of dsa_sparse_attn_prefill,
  * computed for blocks of 6 adjacent query tokens that load the union of
  * their index rows once (adjacent-query dedup, Kwai Keye-VL-2.0 technical
@@ -303,6 +335,99 @@ DSA_API dsa_status_t dsa_sparse_attn_decode_noalloc(
     const void* V_cache, const int64_t* cache_off, int B, int64_t total_n, int H_I, int d_I,
     int Hq, int Hkv, int d, int k, float scale, void* O, int32_t* idx_out, int32_t* err,
     dsa_stream_t stream);
+
+/*
+ * Decode over cache shards.  When one GPU cannot (or should not) hold the
+ * whole cache of a batch, each rank holds one contiguous part of every
+ * sequence's cache (rank r: positions [key_base[b], key_base[b] + n_b) of
+ * sequence b, the parts of rank r preceding those of rank r + 1).  The
+ * selection decomposes exactly: the global top-k of a sequence lies in the
+ * union of the ranks' own top-k lists, under the same order (score, then
+ * lower position), so after one exchange of k (score, key) pairs per
+ * sequence and rank every rank holds the same index rows a single-GPU
+ * decode selects.  The attention decomposes by log-sum-exp: each rank
+ * attends over the selected keys it holds and the partials are merged.  The
+ * two exchanges (all-gathers of [B][k] pairs and of [B][Hq][d + 2] partials)
+ * are the caller's (e.g. NCCL over NVLink); these calls are the per-rank
+ * steps:
+ *
+ *   1. dsa_decode_select_shard   this rank's top-k pairs per sequence
+ *   2. (all-gather the pairs into [P][B][k])
+ *      dsa_decode_merge_shards   the global index rows, on every rank
+ *   3. dsa_decode_attn_shard     this rank's attention partial per (b, h)
+ *   4. (all-gather the partials into [P][B][Hq][d] and [P][B][Hq][2])
+ *      dsa_decode_combine_shards the output rows
+ *
+ * dsa_decode_select_shard - indexer scan and exact top-k of this rank's
+ * rows of each sequence (hot-path step A4, Kwai Keye-VL-2.0 technical
+ * report summary, section 8).
+ *   q_I, w, kI_cache   as dsa_sparse_attn_decode (the rank's cache rows)
+ *   cache_off [B+1]    int64 device: this rank's rows of sequence b are
+ *                      [cache_off[b], cache_off[b+1]); a sequence may have none
+ *   key_base  [B]      int64 device or NULL (0): global position of the rank's
+ *                      first row of each sequence
+ *   ord_out   [B][k]   uint32 OUT: ordered score of each kept key (a monotone
+ *                      map of the fp32 score, larger = better; 0 = padding)
+ *   key_out   [B][k]   int32 OUT: the kept keys (global positions),
+ *                      min(k, n_b) of them ascending, then -1
+ *   workspace          dsa_decode_workspace_size(B, total_n, 64, 128, k, 32,
+ *                      4, 128) bytes, 256-byte aligned
+ * Supported: H_I = 64, d_I = 128, k <= 2048, B <= 4096.
+ */
+DSA_API dsa_status_t dsa_decode_select_shard(const void* q_I, const float* w, const void* kI_cache,
+                                     const int64_t* cache_off, const int64_t* key_base, int B,
+                                     int64_t total_n, int H_I, int d_I, int k, uint32_t* ord_out,
+                                     int32_t* key_out, void* workspace, size_t workspace_bytes,
+                                     int32_t* err, dsa_stream_t stream);
+
+/*
+ * dsa_decode_merge_shards - the exact top-k of each sequence over the P
+ * ranks' lists from dsa_decode_select_shard, gathered rank-major:
+ *   ord_in, key_in [P][B][k]   (rank r's keys all below rank r+1's)
+ *   idx            [B][k]      int32 OUT: global keys ascending, then -1
+ * A gathered run whose keys do not ascend records DSA_DEVERR_INDEX.
+ * Supported: 1 <= P <= 8, k <= 2048.
+ */
+DSA_API dsa_status_t dsa_decode_merge_shards(const uint32_t* ord_in, const int32_t* key_in, int P,
+                                     int B, int k, int32_t* idx, int32_t* err,
+                                     dsa_stream_t stream);
+
+/*
+ * dsa_decode_attn_shard_workspace_size - bytes of workspace for
+ * dsa_decode_attn_shard (256-byte aligned pointer).
+ */
+DSA_API size_t dsa_decode_attn_shard_workspace_size(int B, int64_t total_n, int k, int Hq, int d);
+
+/*
+ * dsa_decode_attn_shard - this rank's share of the decode attention: for
+ * each sequence and query head, the softmax-weighted sum over the entries of
+ * idx[b] that fall in this rank's rows (other entries are skipped), left
+ * unnormalised for the merge:
+ *   part_o  [B][Hq][d]  fp32 OUT: sum_i 2^(x_i - M) V_i, x in log2 units
+ *                       (scale * log2(e) * Q . K)
+ *   part_ml [B][Hq][2]  fp32 OUT: (M, sum_i 2^(x_i - M)); M = -inf and 0 for
+ *                       a head with no key here
+ *   Q, K_cache, V_cache, cache_off, key_base (required)   as above
+ *   idx [B][k]          the global index rows from dsa_decode_merge_shards
+ * Supported: d = 128, Hkv = 4, Hq = 32, k <= 2048.
+ */
+DSA_API dsa_status_t dsa_decode_attn_shard(const void* Q, const void* K_cache, const void* V_cache,
+                                   const int64_t* cache_off, const int64_t* key_base,
+                                   const int32_t* idx, int B, int64_t total_n, int Hq, int Hkv,
+                                   int d, int k, float scale, float* part_o, float* part_ml,
+                                   void* workspace, size_t workspace_bytes, int32_t* err,
+                                   dsa_stream_t stream);
+
+/*
+ * dsa_decode_combine_shards - the output rows from the P ranks' partials,
+ * gathered rank-major (part_o [P][B][Hq][d], part_ml [P][B][Hq][2]):
+ *   O[b,h] = sum_r 2^(M_r - M) part_o[r,b,h] / sum_r 2^(M_r - M) l_r,
+ *   M = max_r M_r;  O [B][Hq][d] bf16 OUT.
+ * Supported: d = 128, Hq = 32.
+ */
+DSA_API dsa_status_t dsa_decode_combine_shards(const float* part_o, const float* part_ml, int P,
+                                       int B, int Hq, int d, void* O, int32_t* err,
+                                       dsa_stream_t stream);
 
 /*
  * Indexer warm-up loss (dense warm-up stage: Kwai Keye-VL-2.0 technical

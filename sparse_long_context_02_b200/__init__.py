@@ -83,6 +83,23 @@ def lib() -> ctypes.CDLL:
         L.dsa_indexer_kl_backward_workspace_size.argtypes = [i64, i32, i32]
         L.dsa_indexer_kl_backward.argtypes = [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz,
                                               vp, vp]
+        L.dsa_index_topk_rows.restype = i32
+        L.dsa_index_topk_rows.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, vp, vp, vp]
+        L.dsa_sparse_attn_rows.restype = i32
+        L.dsa_sparse_attn_rows.argtypes = [vp, vp, vp, vp, i64, i64, i32, i32, i32, i32, f32, vp,
+                                           vp, vp, vp]
+        L.dsa_decode_select_shard.restype = i32
+        L.dsa_decode_select_shard.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, vp,
+                                              vp, sz, vp, vp]
+        L.dsa_decode_merge_shards.restype = i32
+        L.dsa_decode_merge_shards.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
+        L.dsa_decode_attn_shard_workspace_size.restype = sz
+        L.dsa_decode_attn_shard_workspace_size.argtypes = [i32, i64, i32, i32, i32]
+        L.dsa_decode_attn_shard.restype = i32
+        L.dsa_decode_attn_shard.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                            f32, vp, vp, vp, sz, vp, vp]
+        L.dsa_decode_combine_shards.restype = i32
+        L.dsa_decode_combine_shards.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
         L.dsa_check_device_error.restype = i32
         L.dsa_check_device_error.argtypes = [vp, ctypes.POINTER(i32), vp]
         _lib = L
@@ -378,3 +395,108 @@ def indexer_kl_backward(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, G
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _err(err), _stream(stream)), "dsa_indexer_kl_backward")
     return dq_I, dk_I, dw
+
+
+# ------------------------------------------------------------------ sharded calls
+
+def index_topk_rows(q_I: torch.Tensor, k_I: torch.Tensor, w: torch.Tensor, row0: int, k: int,
+                    idx: Optional[torch.Tensor] = None, stream=None, err=None) -> torch.Tensor:
+    """Indexer + top-k for the query rows [row0, row0 + len(q_I)) of a longer
+    sequence: q_I [R][H_I][d_I] and w [R][H_I] hold those rows, k_I holds
+    (at least) keys 0 .. row0 + R - 1.  Returns idx [R][k]."""
+    R, H, d = q_I.shape
+    row1 = row0 + R
+    if k_I.shape[0] < row1:
+        raise ValueError("index_topk_rows: k_I must hold every key up to the last row")
+    if idx is None:
+        idx = torch.empty((R, k), dtype=torch.int32, device=q_I.device)
+    _check(lib().dsa_index_topk_rows(_dev(q_I, "q_I", 1), _dev(k_I, "k_I", 1), _dev(w, "w", 4),
+                                     row0, row1, H, d, k, _dev(idx, "idx", 4), _err(err),
+                                     _stream(stream)), "dsa_index_topk_rows")
+    return idx
+
+
+def sparse_attn_rows(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, idx: torch.Tensor,
+                     scale: float, O: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, stream=None, err=None) -> torch.Tensor:
+    """Sparse attention for R query rows (Q [R][Hq][d], idx [R][k]) over the
+    keys of K / V [n][Hkv][d].  Returns O [R][Hq][d]."""
+    R, Hq, d = Q.shape
+    n, Hkv = K.shape[0], K.shape[1]
+    k = idx.shape[1]
+    if O is None:
+        O = torch.empty_like(Q)
+    _check(lib().dsa_sparse_attn_rows(_dev(Q, "Q", 2), _dev(K, "K", 2), _dev(V, "V", 2),
+                                      _dev(idx, "idx", 4), R, n, Hq, Hkv, d, k, float(scale),
+                                      _dev(O, "O", 2),
+                                      _dev(lse, "lse", 4) if lse is not None else None,
+                                      _err(err), _stream(stream)), "dsa_sparse_attn_rows")
+    return O
+
+
+def decode_select_shard(q_I, w, kI_cache, cache_off, k: int, key_base=None, ord_out=None,
+                        key_out=None, workspace=None, stream=None, err=None):
+    """This rank's exact top-k per sequence over its cache rows: returns
+    (ord_out [B][k] uint32 as int32 bits, key_out [B][k] int32 global keys)."""
+    B, H, dI = q_I.shape
+    total_n = kI_cache.shape[0]
+    dev = q_I.device
+    if ord_out is None:
+        ord_out = torch.empty((B, k), dtype=torch.int32, device=dev)
+    if key_out is None:
+        key_out = torch.empty((B, k), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_size(B, total_n, H, dI, k, 32, 4, 128),
+                                dtype=torch.uint8, device=dev)
+    _check(lib().dsa_decode_select_shard(
+        _dev(q_I, "q_I", 1), _dev(w, "w", 4), _dev(kI_cache, "kI_cache", 1),
+        _dev(cache_off, "cache_off", 8),
+        _dev(key_base, "key_base", 8) if key_base is not None else None, B, total_n, H, dI, k,
+        _dev(ord_out, "ord_out", 4), _dev(key_out, "key_out", 4), _dev(workspace, "workspace", 1),
+        workspace.numel(), _err(err), _stream(stream)), "dsa_decode_select_shard")
+    return ord_out, key_out
+
+
+def decode_merge_shards(ord_in, key_in, idx=None, stream=None, err=None):
+    """Global index rows from the P ranks' gathered lists [P][B][k]."""
+    P, B, k = key_in.shape
+    if idx is None:
+        idx = torch.empty((B, k), dtype=torch.int32, device=key_in.device)
+    _check(lib().dsa_decode_merge_shards(_dev(ord_in, "ord_in", 4), _dev(key_in, "key_in", 4), P,
+                                         B, k, _dev(idx, "idx", 4), _err(err), _stream(stream)),
+           "dsa_decode_merge_shards")
+    return idx
+
+
+def decode_attn_shard(Q, K_cache, V_cache, cache_off, key_base, idx, scale: float, part_o=None,
+                      part_ml=None, workspace=None, stream=None, err=None):
+    """This rank's attention partials (part_o [B][Hq][d], part_ml [B][Hq][2])."""
+    B, Hq, d = Q.shape
+    total_n, Hkv = K_cache.shape[0], K_cache.shape[1]
+    k = idx.shape[1]
+    dev = Q.device
+    if part_o is None:
+        part_o = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    if part_ml is None:
+        part_ml = torch.empty((B, Hq, 2), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(lib().dsa_decode_attn_shard_workspace_size(B, total_n, k, Hq, d),
+                                dtype=torch.uint8, device=dev)
+    _check(lib().dsa_decode_attn_shard(
+        _dev(Q, "Q", 2), _dev(K_cache, "K_cache", 2), _dev(V_cache, "V_cache", 2),
+        _dev(cache_off, "cache_off", 8), _dev(key_base, "key_base", 8), _dev(idx, "idx", 4), B,
+        total_n, Hq, Hkv, d, k, float(scale), _dev(part_o, "part_o", 4),
+        _dev(part_ml, "part_ml", 4), _dev(workspace, "workspace", 1), workspace.numel(),
+        _err(err), _stream(stream)), "dsa_decode_attn_shard")
+    return part_o, part_ml
+
+
+def decode_combine_shards(part_o, part_ml, O=None, stream=None, err=None):
+    """Output rows O [B][Hq][d] bf16 from the gathered partials [P][B][Hq][*]."""
+    P, B, Hq, d = part_o.shape
+    if O is None:
+        O = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=part_o.device)
+    _check(lib().dsa_decode_combine_shards(_dev(part_o, "part_o", 4), _dev(part_ml, "part_ml", 4),
+                                           P, B, Hq, d, _dev(O, "O", 2), _err(err),
+                                           _stream(stream)), "dsa_decode_combine_shards")
+    return O

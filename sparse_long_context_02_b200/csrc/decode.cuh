@@ -69,6 +69,12 @@ struct Params {
     uint32_t* cand_th;         // [slots] an ord that at least k of the slot's entries reach
                                // (0 when the slot holds fewer than k or none is known)
     int* err;                  // the call's device error word (null: the per-device word)
+    // Cache shards (one part of every sequence's cache per rank): the merge
+    // also writes each kept key's ordered score, adds key_base[b] to the
+    // keys, and a sequence with no rows here is not an error.
+    uint32_t* ord_out;         // [B][k] or null
+    const int64_t* key_base;   // [B] or null (0)
+    int allow_empty;
 };
 
 __device__ __forceinline__ bool seq_ok(const Params& p, int b) {
@@ -413,15 +419,21 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
     // previous sequence's owns no slot: it records DSA_DEVERR_INDEX and its
     // index row is all -1 (its output all zeros).
     const bool ordered = b == 0 || p.cache_off[b] >= p.cache_off[b - 1];
+    uint32_t* ord = p.ord_out != nullptr ? p.ord_out + (int64_t)b * p.k : nullptr;
     int s0 = 0, s1 = 0;
     if (seq_ok(p, b) && ordered) {
         s0 = (int)(p.cache_off[b] / p.R) + b;
         s1 = (int)((p.cache_off[b + 1] - 1) / p.R) + b + 1;
-    } else if (tid == 0) {
+    } else if (tid == 0 && !(p.allow_empty && ordered && p.cache_off[b] >= 0 &&
+                             p.cache_off[b] == p.cache_off[b + 1] &&
+                             p.cache_off[b] <= p.total_n)) {
         record_device_error(2);
     }
     if (s1 <= s0) {
-        for (int e = tid; e < p.k; e += 1024) out[e] = -1;
+        for (int e = tid; e < p.k; e += 1024) {
+            out[e] = -1;
+            if (ord) ord[e] = 0u;
+        }
         return;
     }
     if (tid == 0) {
@@ -487,12 +499,86 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
     if (n > p.k) {
         const uint64_t kth = sel::kth_largest<1024, 24>(a, n, p.k, floor_s, S, 0, tid);
         // Only the selected k entries land in the index row.
-        cnt = sel::compact<1024>(a, n, kth, static_cast<uint32_t*>(nullptr), out, S, 0, tid);
+        cnt = sel::compact<1024>(a, n, kth, ord, out, S, 0, tid);
     } else {
-        for (int e = tid; e < n; e += 1024) out[e] = a.index(e);
+        for (int e = tid; e < n; e += 1024) {
+            out[e] = a.index(e);
+            if (ord) ord[e] = a.ord(e);
+        }
     }
     __syncthreads();
-    for (int e = cnt + tid; e < p.k; e += 1024) out[e] = -1;
+    if (p.key_base != nullptr) {
+        const int32_t base = (int32_t)p.key_base[b];
+        for (int e = tid; e < cnt; e += 1024) out[e] += base;
+    }
+    for (int e = cnt + tid; e < p.k; e += 1024) {
+        out[e] = -1;
+        if (ord) ord[e] = 0u;
+    }
+}
+
+// Cache shards: the exact top-k of one sequence over the P shards' kept
+// (ordered score, global key) lists, ord_in / key_in [P][B][k] (each list in
+// ascending key order, -1 padded; shard r's keys all precede shard r+1's).
+// The global top-k is contained in the union of the shards' top-k lists
+// (any key that k keys of its own shard beat is beaten by k keys overall),
+// and the order (score, then lower key) is the same total order, so the row
+// equals the one a single decode over the whole cache selects.  One CTA per
+// sequence; the lists are gathered into shared memory in shard order, which
+// is key order.
+constexpr int kMaxShards = 8;
+
+__global__ void __launch_bounds__(1024) merge_shards_kernel(const uint32_t* ord_in,
+                                                             const int32_t* key_in, int P, int B,
+                                                             int k, int32_t* idx_out, int* err) {
+    bind_error_word(err);
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ Scratch<1024> S;
+    __shared__ int cnt_s[kMaxShards + 1];
+    const int b = blockIdx.x, tid = threadIdx.x;
+    uint32_t* so = reinterpret_cast<uint32_t*>(smem);
+    int32_t* si = reinterpret_cast<int32_t*>(smem + (size_t)P * k * 4);
+    if (tid < P) {  // valid entries lead every list
+        const int32_t* kl = key_in + ((int64_t)tid * B + b) * k;
+        int lo = 0, hi = k;  // the first -1
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (kl[mid] >= 0) lo = mid + 1;
+            else hi = mid;
+        }
+        cnt_s[tid + 1] = lo;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        cnt_s[0] = 0;
+        for (int r = 0; r < P; ++r) cnt_s[r + 1] += cnt_s[r];
+    }
+    __syncthreads();
+    const int n = cnt_s[P];
+    for (int r = 0; r < P; ++r) {
+        const int c0 = cnt_s[r], c = cnt_s[r + 1] - c0;
+        const uint32_t* os = ord_in + ((int64_t)r * B + b) * k;
+        const int32_t* ks = key_in + ((int64_t)r * B + b) * k;
+        for (int e = tid; e < c; e += 1024) {
+            so[c0 + e] = os[e];
+            si[c0 + e] = ks[e];
+        }
+    }
+    __syncthreads();
+    // keys must ascend along the gathered run (the output is written in it)
+    for (int e = tid; e + 1 < n; e += 1024)
+        if (si[e] >= si[e + 1]) record_device_error(2);
+    int32_t* out = idx_out + (int64_t)b * k;
+    const FlatAccess a{so, si};
+    int cnt = n;
+    if (n > k) {
+        const uint64_t kth = sel::kth_largest<1024, 16>(a, n, k, 0u, S, 0, tid);
+        cnt = sel::compact<1024>(a, n, kth, static_cast<uint32_t*>(nullptr), out, S, 0, tid);
+    } else {
+        for (int e = tid; e < n; e += 1024) out[e] = si[e];
+    }
+    __syncthreads();
+    for (int e = cnt + tid; e < k; e += 1024) out[e] = -1;
 }
 
 }  // namespace dec

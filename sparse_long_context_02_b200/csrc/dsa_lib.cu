@@ -114,9 +114,11 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 template <int HI, int DI, bool TOPK>
 dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
                           int64_t L, int k, int32_t* idx, float* scores, const int32_t* cu_seqlens,
-                          int nseq, int64_t row0, int64_t row1, int* err, cudaStream_t st) {
+                          int nseq, int64_t row0, int64_t row1, int* err, cudaStream_t st,
+                          int64_t qrow0) {
+    // q_I / w / idx hold rows [qrow0, L) (qrow0 = 0: the whole sequence)
     CUtensorMap mq, mk;
-    if (!make_map(&mq, q_I, DI, (uint64_t)L * HI, dsa::idx::kTokens * HI) ||
+    if (!make_map(&mq, q_I, DI, (uint64_t)(L - qrow0) * HI, dsa::idx::kTokens * HI) ||
         !make_map(&mk, k_I, DI, (uint64_t)L, dsa::idx::kKeyTile))
         return fail(DSA_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed", fn);
     const dsa::idx::Layout lay(HI, DI, k, TOPK);
@@ -144,6 +146,7 @@ dsa_status_t launch_index(const char* fn, const void* q_I, const void* k_I, cons
     p.cu_seqlens = cu_seqlens;
     p.nseq = nseq;
     p.err = err;
+    p.qrow0 = qrow0;
     kern<<<p.nblocks, dsa::idx::kThreads, smem, st>>>(mq, mk, p);
     CUDA_TRY(cudaGetLastError());
     return ok();
@@ -153,16 +156,16 @@ template <bool TOPK>
 dsa_status_t dispatch_index(const char* fn, const void* q_I, const void* k_I, const float* w,
                             int64_t L, int H_I, int d_I, int k, int32_t* idx, float* scores,
                             const int32_t* cu, int nseq, int* err, cudaStream_t st,
-                            int64_t row0 = 0, int64_t row1 = -1) {
+                            int64_t row0 = 0, int64_t row1 = -1, int64_t qrow0 = 0) {
     if (row1 < 0) row1 = L;
     if (H_I == 64 && d_I == 128)
-        return launch_index<64, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st);
+        return launch_index<64, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st, qrow0);
     if (H_I == 64 && d_I == 64)
-        return launch_index<64, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st);
+        return launch_index<64, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st, qrow0);
     if (H_I == 4 && d_I == 128)
-        return launch_index<4, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st);
+        return launch_index<4, 128, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st, qrow0);
     if (H_I == 4 && d_I == 64)
-        return launch_index<4, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st);
+        return launch_index<4, 64, TOPK>(fn, q_I, k_I, w, L, k, idx, scores, cu, nseq, row0, row1, err, st, qrow0);
     return fail(DSA_ERR_UNSUPPORTED, "%s: (H_I, d_I) = (%d, %d) not in {4, 64} x {64, 128}", fn,
                 H_I, d_I);
 }
@@ -298,6 +301,54 @@ dsa_status_t dsa_index_topk_varlen(const void* q_I, const void* k_I, const float
         return fail(DSA_ERR_UNSUPPORTED, "%s: L * H_I too large", fn);
     return dispatch_index<true>(fn, q_I, k_I, w, L, H_I, d_I, k, idx, nullptr, cu_seqlens, nseq,
                                 err, static_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_index_topk_rows(const void* q_I, const void* k_I, const float* w, int64_t row0,
+                                 int64_t row1, int H_I, int d_I, int k, int32_t* idx,
+                                 int32_t* err, dsa_stream_t stream) {
+    static const char fn[] = "dsa_index_topk_rows";
+    CHECK_PTR(q_I);
+    CHECK_PTR(k_I);
+    CHECK_PTR(w);
+    CHECK_PTR(idx);
+    CHECK_ERR_WORD(err);
+    if (row0 < 0 || row1 <= row0 || row1 > (int64_t(1) << 30))
+        return fail(DSA_ERR_INVALID_ARG, "%s: rows [%lld, %lld)", fn, (long long)row0,
+                    (long long)row1);
+    if (row0 % dsa::idx::kTokens != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: row0 = %lld is not a multiple of %d", fn,
+                    (long long)row0, dsa::idx::kTokens);
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (k > 2048) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > 2048", fn, k);
+    if (row1 * H_I >= (int64_t(1) << 31))
+        return fail(DSA_ERR_UNSUPPORTED, "%s: row1 * H_I too large", fn);
+    return dispatch_index<true>(fn, q_I, k_I, w, row1, H_I, d_I, k, idx, nullptr, nullptr, 1, err,
+                                static_cast<cudaStream_t>(stream), row0, row1, row0);
+}
+
+dsa_status_t dsa_sparse_attn_rows(const void* Q, const void* K, const void* V,
+                                  const int32_t* idx, int64_t nrows, int64_t nkeys, int Hq,
+                                  int Hkv, int d, int k, float scale, void* O, float* lse,
+                                  int32_t* err, dsa_stream_t stream) {
+    static const char fn[] = "dsa_sparse_attn_rows";
+    CHECK_PTR(Q);
+    CHECK_PTR(K);
+    CHECK_PTR(V);
+    CHECK_PTR(idx);
+    CHECK_PTR(O);
+    CHECK_ERR_WORD(err);
+    if (nrows < 1 || nrows > (int64_t(1) << 30) || nkeys < 1 || nkeys > (int64_t(1) << 31) - 1)
+        return fail(DSA_ERR_INVALID_ARG, "%s: nrows = %lld, nkeys = %lld", fn, (long long)nrows,
+                    (long long)nkeys);
+    if (k < 1 || k > 65536) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (Hkv < 1 || Hq < 1 || Hq % Hkv) return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d", fn, Hq, Hkv);
+    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: lse is not 4-byte aligned", fn);
+    const dsa_status_t r = attn_prefill_rows(fn, Q, K, V, idx, nkeys, Hq, Hkv, d, k, scale, O,
+                                             lse, 0, nrows, err,
+                                             static_cast<cudaStream_t>(stream));
+    return r == DSA_OK ? ok() : r;
 }
 
 dsa_status_t dsa_sparse_attn_prefill_dedup(const void* Q, const void* K, const void* V,
@@ -614,22 +665,14 @@ dsa_status_t check_decode_args(const char* fn, const void* q_I, const float* w, 
     return DSA_OK;
 }
 
-// The decode itself, on checked arguments.
-dsa_status_t run_decode(const char* fn, const void* q_I, const float* w, const void* Q,
-                        const void* kI_cache, const void* K_cache, const void* V_cache,
-                        const int64_t* cache_off, int B, int64_t total_n, int k, int Hq, int d,
-                        float scale, void* O, int32_t* idx_out, void* workspace,
-                        size_t workspace_bytes, int32_t* err, dsa_stream_t stream) {
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-        return fail(DSA_ERR_INVALID_ARG, "%s: workspace is not 256-byte aligned", fn);
-    const DecodePlan pl = plan_decode(B, total_n, k, Hq, d, num_sms());
-    if (workspace_bytes < pl.total)
-        return fail(DSA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, workspace_bytes,
-                    pl.total);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-
-    dsa::dec::Params dp;
+// Decode phase 1: the indexer scan over the packed cache and the per-sequence
+// merge into index rows (with ordered scores and global keys for a shard).
+dsa_status_t launch_decode_select(const char* fn, const DecodePlan& pl, uint8_t* ws,
+                                  const void* q_I, const float* w, const void* kI_cache,
+                                  const int64_t* cache_off, int B, int64_t total_n, int k,
+                                  int32_t* idx, uint32_t* ord_out, const int64_t* key_base,
+                                  bool shard, int32_t* err, cudaStream_t st) {
+    dsa::dec::Params dp{};
     dp.w = w;
     dp.cache_off = cache_off;
     dp.B = B;
@@ -641,7 +684,9 @@ dsa_status_t run_decode(const char* fn, const void* q_I, const float* w, const v
     dp.cand_cnt = reinterpret_cast<int*>(ws + pl.off_cnt);
     dp.cand_th = reinterpret_cast<uint32_t*>(ws + pl.off_th);
     dp.err = err;
-    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + pl.off_idx);
+    dp.ord_out = ord_out;
+    dp.key_base = key_base;
+    dp.allow_empty = shard ? 1 : 0;
 
     CUtensorMap mq, mk;
     if (!make_map(&mq, q_I, 128, (uint64_t)B * 64, 64) ||
@@ -664,7 +709,16 @@ dsa_status_t run_decode(const char* fn, const void* q_I, const float* w, const v
     CUDA_TRY(launch_chained(dsa::dec::merge_kernel, dim3(B), dim3(1024), smem_merge, st, dp, idx,
                             merge_smem_cap));
     CUDA_TRY(cudaGetLastError());
+    return DSA_OK;
+}
 
+// Decode phase 2: attention split into nsplit slices of each index row
+// (partials in the workspace).
+dsa_status_t launch_decode_attn(const char* fn, const DecodePlan& pl, uint8_t* ws, const void* Q,
+                                const void* K_cache, const void* V_cache,
+                                const int64_t* cache_off, int B, int k, float scale,
+                                const int32_t* idx, const int64_t* key_base, int32_t* err,
+                                cudaStream_t st) {
     dsa::attn::Params ap{};
     ap.Q = static_cast<const __nv_bfloat16*>(Q);
     ap.K = static_cast<const __nv_bfloat16*>(K_cache);
@@ -677,11 +731,38 @@ dsa_status_t run_decode(const char* fn, const void* q_I, const float* w, const v
     ap.part_o = reinterpret_cast<float*>(ws + pl.off_po);
     ap.part_ml = reinterpret_cast<float*>(ws + pl.off_pml);
     ap.err = err;
-    dsa_status_t r = launch_attn<128, 4, 8, true>(fn, ap, (int64_t)B * pl.nsplit, st);
+    ap.key_base = key_base;
+    ap.skip_foreign = key_base != nullptr ? 1 : 0;
+    return launch_attn<128, 4, 8, true>(fn, ap, (int64_t)B * pl.nsplit, st);
+}
+
+// The decode itself, on checked arguments.
+dsa_status_t run_decode(const char* fn, const void* q_I, const float* w, const void* Q,
+                        const void* kI_cache, const void* K_cache, const void* V_cache,
+                        const int64_t* cache_off, int B, int64_t total_n, int k, int Hq, int d,
+                        float scale, void* O, int32_t* idx_out, void* workspace,
+                        size_t workspace_bytes, int32_t* err, dsa_stream_t stream) {
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: workspace is not 256-byte aligned", fn);
+    const DecodePlan pl = plan_decode(B, total_n, k, Hq, d, num_sms());
+    if (workspace_bytes < pl.total)
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, workspace_bytes,
+                    pl.total);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + pl.off_idx);
+    dsa_status_t r = launch_decode_select(fn, pl, ws, q_I, w, kI_cache, cache_off, B, total_n, k,
+                                          idx, nullptr, nullptr, false, err, st);
     if (r != DSA_OK) return r;
-    CUDA_TRY(launch_chained(dsa::attn::combine_kernel<128, 32>, dim3(B * 32), dim3(128), 0, st,
-                            static_cast<const float*>(ap.part_o), static_cast<const float*>(ap.part_ml),
-                            pl.nsplit, static_cast<__nv_bfloat16*>(O)));
+    r = launch_decode_attn(fn, pl, ws, Q, K_cache, V_cache, cache_off, B, k, scale, idx, nullptr,
+                           err, st);
+    if (r != DSA_OK) return r;
+    const float* po = reinterpret_cast<const float*>(ws + pl.off_po);
+    const float* pml = reinterpret_cast<const float*>(ws + pl.off_pml);
+    CUDA_TRY(launch_chained(dsa::attn::combine_kernel<128, 32, true>, dim3(B * 32), dim3(128), 0,
+                            st, po, pml, pl.nsplit, (int64_t)pl.nsplit, (int64_t)1,
+                            static_cast<__nv_bfloat16*>(O), static_cast<float*>(nullptr),
+                            static_cast<float*>(nullptr)));
     CUDA_TRY(cudaGetLastError());
     return ok();
 }
@@ -704,6 +785,132 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
     CHECK_PTR(workspace);
     return run_decode(fn, q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, B, total_n, k, Hq, d,
                       scale, O, idx_out, workspace, workspace_bytes, err, stream);
+}
+
+// ------------------------------------------------------------ decode over cache shards
+
+dsa_status_t dsa_decode_select_shard(const void* q_I, const float* w, const void* kI_cache,
+                                     const int64_t* cache_off, const int64_t* key_base, int B,
+                                     int64_t total_n, int H_I, int d_I, int k, uint32_t* ord_out,
+                                     int32_t* key_out, void* workspace, size_t workspace_bytes,
+                                     int32_t* err, dsa_stream_t stream) {
+    static const char fn[] = "dsa_decode_select_shard";
+    CHECK_PTR(q_I);
+    CHECK_PTR(w);
+    CHECK_PTR(kI_cache);
+    CHECK_PTR(cache_off);
+    CHECK_PTR(ord_out);
+    CHECK_PTR(key_out);
+    CHECK_PTR(workspace);
+    CHECK_ERR_WORD(err);
+    if (key_base != nullptr && (reinterpret_cast<uintptr_t>(key_base) & 7u) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: key_base is not 8-byte aligned", fn);
+    if (B < 1 || B > 4096) return fail(DSA_ERR_INVALID_ARG, "%s: B = %d", fn, B);
+    if (total_n < 1 || total_n >= (int64_t(1) << 31))
+        return fail(DSA_ERR_INVALID_ARG, "%s: total_n = %lld", fn, (long long)total_n);
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (H_I != 64 || d_I != 128 || k > 2048)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: supported H_I=64, d_I=128, k<=2048", fn);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: workspace is not 256-byte aligned", fn);
+    const DecodePlan pl = plan_decode(B, total_n, k, 32, 128, num_sms());
+    if (workspace_bytes < pl.total)
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, workspace_bytes,
+                    pl.total);
+    const dsa_status_t r = launch_decode_select(
+        fn, pl, static_cast<uint8_t*>(workspace), q_I, w, kI_cache, cache_off, B, total_n, k,
+        key_out, ord_out, key_base, true, err, static_cast<cudaStream_t>(stream));
+    return r == DSA_OK ? ok() : r;
+}
+
+dsa_status_t dsa_decode_merge_shards(const uint32_t* ord_in, const int32_t* key_in, int P, int B,
+                                     int k, int32_t* idx, int32_t* err, dsa_stream_t stream) {
+    static const char fn[] = "dsa_decode_merge_shards";
+    CHECK_PTR(ord_in);
+    CHECK_PTR(key_in);
+    CHECK_PTR(idx);
+    CHECK_ERR_WORD(err);
+    if (P < 1 || P > dsa::dec::kMaxShards)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: P = %d (1..%d shards)", fn, P, dsa::dec::kMaxShards);
+    if (B < 1 || B > 65535) return fail(DSA_ERR_INVALID_ARG, "%s: B = %d", fn, B);
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (k > 2048) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > 2048", fn, k);
+    const int smem = P * k * 8;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CUDA_TRY(cudaFuncSetAttribute(dsa::dec::merge_shards_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    dsa::dec::merge_shards_kernel<<<B, 1024, smem, st>>>(ord_in, key_in, P, B, k, idx, err);
+    CUDA_TRY(cudaGetLastError());
+    return ok();
+}
+
+size_t dsa_decode_attn_shard_workspace_size(int B, int64_t total_n, int k, int Hq, int d) {
+    if (B < 1 || total_n < 1 || k < 1) return 0;
+    return plan_decode(B, total_n, k, Hq, d, num_sms()).total;
+}
+
+dsa_status_t dsa_decode_attn_shard(const void* Q, const void* K_cache, const void* V_cache,
+                                   const int64_t* cache_off, const int64_t* key_base,
+                                   const int32_t* idx, int B, int64_t total_n, int Hq, int Hkv,
+                                   int d, int k, float scale, float* part_o, float* part_ml,
+                                   void* workspace, size_t workspace_bytes, int32_t* err,
+                                   dsa_stream_t stream) {
+    static const char fn[] = "dsa_decode_attn_shard";
+    CHECK_PTR(Q);
+    CHECK_PTR(K_cache);
+    CHECK_PTR(V_cache);
+    CHECK_PTR(cache_off);
+    CHECK_PTR(idx);
+    CHECK_PTR(part_o);
+    CHECK_PTR(part_ml);
+    CHECK_PTR(workspace);
+    CHECK_ERR_WORD(err);
+    if (key_base == nullptr || (reinterpret_cast<uintptr_t>(key_base) & 7u) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: key_base is NULL or not 8-byte aligned", fn);
+    if (B < 1 || B > 4096) return fail(DSA_ERR_INVALID_ARG, "%s: B = %d", fn, B);
+    if (total_n < 1 || total_n >= (int64_t(1) << 31))
+        return fail(DSA_ERR_INVALID_ARG, "%s: total_n = %lld", fn, (long long)total_n);
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
+    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
+    if (d != 128 || Hkv != 4 || Hq != 32 || k > 2048)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: supported d=128, Hkv=4, Hq=32, k<=2048", fn);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: workspace is not 256-byte aligned", fn);
+    const DecodePlan pl = plan_decode(B, total_n, k, Hq, d, num_sms());
+    if (workspace_bytes < pl.total)
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, workspace_bytes,
+                    pl.total);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    dsa_status_t r = launch_decode_attn(fn, pl, ws, Q, K_cache, V_cache, cache_off, B, k, scale,
+                                        idx, key_base, err, st);
+    if (r != DSA_OK) return r;
+    const float* po = reinterpret_cast<const float*>(ws + pl.off_po);
+    const float* pml = reinterpret_cast<const float*>(ws + pl.off_pml);
+    CUDA_TRY(launch_chained(dsa::attn::combine_kernel<128, 32, false>, dim3(B * 32), dim3(128), 0,
+                            st, po, pml, pl.nsplit, (int64_t)pl.nsplit, (int64_t)1,
+                            static_cast<__nv_bfloat16*>(nullptr), part_o, part_ml));
+    CUDA_TRY(cudaGetLastError());
+    return ok();
+}
+
+dsa_status_t dsa_decode_combine_shards(const float* part_o, const float* part_ml, int P, int B,
+                                       int Hq, int d, void* O, int32_t* err,
+                                       dsa_stream_t stream) {
+    static const char fn[] = "dsa_decode_combine_shards";
+    CHECK_PTR(part_o);
+    CHECK_PTR(part_ml);
+    CHECK_PTR(O);
+    CHECK_ERR_WORD(err);
+    if (P < 1 || P > 1024) return fail(DSA_ERR_INVALID_ARG, "%s: P = %d", fn, P);
+    if (B < 1 || B > 65535) return fail(DSA_ERR_INVALID_ARG, "%s: B = %d", fn, B);
+    if (d != 128 || Hq != 32) return fail(DSA_ERR_UNSUPPORTED, "%s: supported d=128, Hq=32", fn);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    dsa::attn::combine_kernel<128, 32, true><<<B * 32, 128, 0, st>>>(
+        part_o, part_ml, P, (int64_t)1, (int64_t)B, static_cast<__nv_bfloat16*>(O), nullptr,
+        nullptr);
+    CUDA_TRY(cudaGetLastError());
+    return ok();
 }
 
 dsa_status_t dsa_check_device_error(int32_t* err, int* code, dsa_stream_t stream) {

@@ -180,6 +180,10 @@ struct Params {
     const int32_t* cu_seqlens;  // [nseq + 1], 0 ... L, non-decreasing
     int nseq;
     int* err;            // the call's device error word (null: the per-device word)
+    // Query rows held by the call: q_I, w and idx start at row qrow0 (a
+    // multiple of kTokens), so row t is element t - qrow0 of each.  Keys are
+    // always rows 0 .. L-1 of k_I.
+    int64_t qrow0;
 };
 
 // Start of the sequence that holds row t: cu[b] for the last b with
@@ -256,7 +260,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     }
     for (int e = threadIdx.x; e < kTokens * HI; e += kThreads) {
         const int64_t t = t0 + e / HI;
-        w_s[e] = t < L ? p.w[t * HI + (e % HI)] : 0.f;
+        w_s[e] = t < L ? p.w[(t - p.qrow0) * HI + (e % HI)] : 0.f;
     }
     tc_fence_before();
     __syncthreads();
@@ -271,7 +275,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             prefetch_tensormap(&tmap_k);
             const uint32_t qbar = smem_u32(&misc->qfull);
             mbar_arrive_expect_tx(qbar, Q_BYTES);
-            tma_load_2d(smem_u32(smem + lay.q), &tmap_q, qbar, 0, (int32_t)(t0 * HI));
+            tma_load_2d(smem_u32(smem + lay.q), &tmap_q, qbar, 0, (int32_t)((t0 - p.qrow0) * HI));
             int issued = 0;
             for (int i = 0; i < ntiles; ++i) {
                 if (misc->abort_flag) break;
@@ -389,7 +393,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
         if constexpr (TOPK) {
             tk.reduce(true);
             if (trow && !misc->abort_flag) {
-                int32_t* out = p.idx + t * p.k;
+                int32_t* out = p.idx + (t - p.qrow0) * p.k;
                 for (int e = tid; e < p.k; e += 128) out[e] = e < tk.cnt ? ix[e] : -1;
             }
         }

@@ -58,6 +58,11 @@ struct Params {
     float* part_o;            // [B][nsplit][Hq][d]      unnormalised partial O
     float* part_ml;           // [B][nsplit][Hq][2]      running max (log2 units), sum
     int* err;                 // the call's device error word (null: the per-device word)
+    // Cache shards (decode): index entries are global keys; this shard holds
+    // keys [key_base[b], key_base[b] + n_b) of sequence b, and entries
+    // outside that range belong to another shard (skipped, not flagged).
+    const int64_t* key_base;  // [B] or null (0)
+    int skip_foreign;
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -113,7 +118,7 @@ attn_kernel(const Params p) {
     const __nv_bfloat16 *Kb = p.K, *Vb = p.V, *qrow;
     const int32_t* irow;
     int nent;
-    int64_t nkeys, orow = 0;
+    int64_t nkeys, orow = 0, koff = 0;
     int split = 0;
     if constexpr (SPLIT) {
         const int64_t b = blockIdx.x / p.nsplit;
@@ -124,6 +129,7 @@ attn_kernel(const Params p) {
         if (nent < 0) nent = 0;
         const int64_t base = p.cache_off[b];
         nkeys = p.cache_off[b + 1] - base;
+        if (p.key_base != nullptr) koff = p.key_base[b];
         Kb = p.K + base * HKV * D;
         Vb = p.V + base * HKV * D;
         irow = p.idx + b * p.k + e0;
@@ -161,15 +167,17 @@ attn_kernel(const Params p) {
         int32_t pre = load_idx(0);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
-            const int32_t si = pre;
+            const int64_t sg = pre;  // the entry: a key of this shard after - koff
             pre = load_idx(c + 1);
             if (c >= kStages) {
                 bool got = false;
                 if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ((c / kStages) - 1) & 1);
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
             }
-            if (si >= nkeys) record_device_error(2);
-            const bool valid = si >= 0 && si < nkeys;
+            const int64_t sl = sg - koff;
+            if (sg >= 0 && sl >= nkeys && !p.skip_foreign) record_device_error(2);
+            const bool valid = sg >= 0 && sl >= 0 && sl < nkeys;
+            const int32_t si = valid ? (int32_t)sl : -1;
             const uint32_t bal = __ballot_sync(0xffffffffu, valid);
             const uint32_t sbase = smem_u32(smem + s * C::STAGE);
             if (bal) {
@@ -334,24 +342,41 @@ attn_kernel(const Params p) {
 
 // Merges the nsplit partial results of each (sequence, head):
 //   M = max_j m_j,  l = sum_j l_j 2^(m_j - M),  O = sum_j O_j 2^(m_j - M) / l.
+// Partial j of sequence b is row (b * bs + j * js) of part_o / part_ml (in
+// units of HQ heads): bs = nsplit, js = 1 for the [B][nsplit] layout of one
+// decode, bs = 1, js = B for the [P][B] layout of P gathered cache shards.
+// FINAL: O is written as bf16; otherwise the merged partial itself (the
+// unnormalised sum relative to M, and M, l) goes to out_o / out_ml, rows
+// [B][HQ], for a later merge with other shards' partials.
 // One CTA per (sequence, head), one thread per output dimension.
-template <int D, int HQ>
+template <int D, int HQ, bool FINAL>
 __global__ void __launch_bounds__(D) combine_kernel(const float* part_o, const float* part_ml,
-                                                    int nsplit, __nv_bfloat16* O) {
+                                                    int nsplit, int64_t bs, int64_t js,
+                                                    __nv_bfloat16* O, float* out_o,
+                                                    float* out_ml) {
     pdl_wait();  // the partials come from the split attention
     const int64_t b = blockIdx.x / HQ;
     const int h = blockIdx.x % HQ, c = threadIdx.x;
+    auto row = [&](int j) { return ((b * bs + (int64_t)j * js) * HQ + h); };
     float M = -INFINITY;
-    for (int j = 0; j < nsplit; ++j) M = fmaxf(M, part_ml[((b * nsplit + j) * HQ + h) * 2]);
+    for (int j = 0; j < nsplit; ++j) M = fmaxf(M, part_ml[row(j) * 2]);
     const float Mu = M == -INFINITY ? 0.f : M;
     float l = 0.f, acc = 0.f;
     for (int j = 0; j < nsplit; ++j) {
-        const float* ml = part_ml + ((b * nsplit + j) * HQ + h) * 2;
+        const float* ml = part_ml + row(j) * 2;
         const float f = ex2(ml[0] - Mu);
         l += ml[1] * f;
-        acc += part_o[((b * nsplit + j) * HQ + h) * D + c] * f;
+        acc += part_o[row(j) * D + c] * f;
     }
-    O[(b * HQ + h) * D + c] = __float2bfloat16_rn(l > 0.f ? acc / l : 0.f);
+    if constexpr (FINAL) {
+        O[(b * HQ + h) * D + c] = __float2bfloat16_rn(l > 0.f ? acc / l : 0.f);
+    } else {
+        out_o[(b * HQ + h) * D + c] = acc;
+        if (c == 0) {
+            out_ml[(b * HQ + h) * 2] = M;
+            out_ml[(b * HQ + h) * 2 + 1] = l;
+        }
+    }
 }
 
 }  // namespace attn
