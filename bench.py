@@ -62,6 +62,15 @@ def parse():
                     help="instead of timing: run the prefill indexer once and report how many "
                          "distinct keys the index rows of G consecutive queries select together "
                          "(the traffic an adjacent-query dedup would read)")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the per-workload lines of the tiny, 32K and 256K-video prefills "
+                         "(timed after the headline step, on one GPU)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with several GPUs: every rank solves its own copy of the workload "
+                         "(weak scaling) instead of sharing one workload")
+    ap.add_argument("--decode-shard", default="batch", choices=["batch", "cache"],
+                    help="with several GPUs: split the decode batch by sequence (no exchange) "
+                         "or every sequence's cache (two all-gathers per step)")
     ap.add_argument("--attn-bwd", action="store_true",
                     help="instead of the inference step: time the sparse attention's training "
                          "pass (forward with lse, then dsa_sparse_attn_backward) on the prefill "
@@ -440,11 +449,273 @@ def run_ours(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and pcfg:
-        cpu = cpu_baseline(pcfg, p_host, args.cpu_seconds)
+        cpu = cpu_baseline(pcfg, p_host, args.cpu_seconds, dcfg)
+
+    others = None
+    if world == 1 and not args.no_other_configs and pcfg is not None:
+        del P, Ph, p_host
+        torch.cuda.empty_cache()
+        others = other_configs(torch, dsa, pk, args, stream, flush)
 
     return dict(value=value, prefill_ms=prefill_ms, decode_ms=decode_ms, decode_tps=decode_tps,
                 clocks=clk, kernels=kernels, roofline=roofline, e2e=e2e, cpu=cpu,
-                launches=launches_per_step * K, pcfg=pcfg, dcfg=dcfg)
+                launches=launches_per_step * K, pcfg=pcfg, dcfg=dcfg, others=others)
+
+
+def other_configs(torch, dsa, pk, args, stream, flush):
+    """The other prefill workloads (tiny, 32K, 256K video), each timed as its
+    own steps (indexer + top-k, then attention; the dedup attention on the
+    video workload), with the same rooflines; min(steps, 5) timed steps."""
+    out = {}
+    fp8_peak = 2.0 * pk["bf16_sus"]
+    for cfg in (gen.TINY_PREFILL, gen.PREFILL_32K, gen.VIDEO_256K):
+        h = gen.prefill_inputs(cfg)
+        t = {n: torch.from_numpy(h[n]).cuda() for n in ("q_I", "k_I", "w")}
+        bf = {n: torch.from_numpy(h[n].view(np.int16)).view(torch.bfloat16).cuda()
+              for n in ("Q", "K", "V")}
+        del h
+        idx = torch.empty((cfg.L, cfg.k), dtype=torch.int32, device="cuda")
+        O = torch.empty_like(bf["Q"])
+        attn = dsa.sparse_attn_prefill_dedup if cfg.video else dsa.sparse_attn_prefill
+
+        def step(ev=None):
+            if ev:
+                ev[0].record(stream)
+            dsa.index_topk(t["q_I"], t["k_I"], t["w"], cfg.k, idx=idx, stream=stream)
+            if ev:
+                ev[1].record(stream)
+            attn(bf["Q"], bf["K"], bf["V"], idx, cfg.scale, O=O, stream=stream)
+            if ev:
+                ev[2].record(stream)
+
+        for _ in range(max(1, args.warmup)):
+            flush.zero_()
+            step()
+        n = max(1, min(args.steps, 5))
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+        if dsa.device_error() != 0:
+            raise RuntimeError(f"device error in the {cfg.name} workload")
+        mi = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+        ma = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        fl, by = prefill_flops(cfg), prefill_attn_bytes(cfg)
+        out[cfg.name] = dict(
+            steps=n, ms_per_step=mi + ma, value=cfg.L / ((mi + ma) / 1e3),
+            unit="query-tokens/s",
+            kernels={"dsa_index_topk": dict(bound="tensor", ms=mi, achieved=fl / (mi / 1e3) / 1e12,
+                                            peak=fp8_peak, unit="TFLOP/s",
+                                            frac=fl / (mi / 1e3) / 1e12 / fp8_peak),
+                     attn.__name__: dict(bound="l2 (gathered rows)", ms=ma,
+                                         achieved=by / (ma / 1e3) / 1e9, unit="GB/s",
+                                         hbm_frac=by / (ma / 1e3) / 1e9 / pk["hbm"])})
+        del t, bf, idx, O
+        torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------------ one workload on N GPUs
+
+def run_sharded(args, rank, world, local_rank):
+    """One workload shared by the N ranks (strong scaling).  Prefill: the
+    query rows in zig-zag blocks, one NCCL exchange step (all-gather of the
+    blocks of k_I, K and V) and then each rank's selection and attention for
+    its rows.  Decode: batch shards (each rank its own sequences), or cache
+    shards (each rank part of every sequence, two all-gathers).  The step
+    time is the max over ranks of each rank's device time."""
+    import torch
+    import torch.distributed as tdist
+    import sparse_long_context_02_b200 as dsa
+    from sparse_long_context_02_b200 import dist, shards
+
+    torch.cuda.set_device(local_rank)
+    pcfg = gen.CONFIGS[args.prefill_config] if args.prefill_config else None
+    dcfg = gen.CONFIGS[args.decode_config] if args.decode_config else None
+    if dcfg is not None and args.decode_batch:
+        dcfg = dcfg.with_(B=args.decode_batch)
+    stream = torch.cuda.current_stream()
+    dev = torch.device("cuda", local_rank)
+    bf = torch.bfloat16
+
+    e2e_on = not args.no_e2e
+    h2d = []  # (pinned host, device) pairs of the rank's inputs, for the e2e leg
+
+    def t_(a, dt=None, inp=True):
+        x = torch.from_numpy(np.ascontiguousarray(a))
+        x = x.view(dt) if dt is not None else x
+        if e2e_on and inp:
+            x = x.pin_memory()
+            d_ = x.to(dev)
+            h2d.append((x, d_))
+            return d_
+        return x.to(dev)
+
+    # ---- prefill: this rank's rows and key blocks
+    Pf = {}
+    if pcfg:
+        L = pcfg.L
+        blocks = shards.zigzag_blocks(L, world)
+        blk = blocks[0][1] - blocks[0][0]
+        rows = shards.zigzag_rows(L, world, rank)
+        mine = {n: [] for n in ("q_I", "w", "Q", "idx", "O")}
+        own = {n: [] for n in ("k_I", "K", "V")}
+        for b in (rank, 2 * world - 1 - rank):
+            a, z = blocks[b]
+            n = z - a
+            pad = lambda x: np.concatenate([x, np.zeros((blk - n,) + x.shape[1:], x.dtype)])  # noqa: E731
+            mine["q_I"].append(t_(pad(gen.prefill_qI(pcfg, a, z))))
+            mine["w"].append(t_(pad(gen.prefill_w(pcfg, a, z))))
+            mine["Q"].append(t_(pad(gen.prefill_Q(pcfg, a, z)).view(np.int16), bf))
+            mine["idx"].append(torch.empty((blk, pcfg.k), dtype=torch.int32, device=dev))
+            mine["O"].append(torch.empty((blk, pcfg.Hq, pcfg.d), dtype=bf, device=dev))
+            own["k_I"].append(t_(pad(gen.prefill_kI(pcfg, a, z))))
+            own["K"].append(t_(pad(gen.prefill_K(pcfg, a, z)).view(np.int16), bf))
+            own["V"].append(t_(pad(gen.prefill_V(pcfg, a, z)).view(np.int16), bf))
+        keys = dict(k_I=torch.empty((2 * world * blk, pcfg.d_I), dtype=torch.uint8, device=dev),
+                    K=torch.empty((2 * world * blk, pcfg.Hkv, pcfg.d), dtype=bf, device=dev),
+                    V=torch.empty((2 * world * blk, pcfg.Hkv, pcfg.d), dtype=bf, device=dev))
+        Pf = dict(rows=rows, mine=mine, own=own, keys=keys)
+
+    # ---- decode: batch shards or cache shards
+    Df = {}
+    if dcfg:
+        off = gen.decode_offsets(dcfg)
+        lens = np.diff(off)
+        q = gen.decode_queries(dcfg)
+
+        def cache_rows(segs):
+            """Packed cache of (global start, length) pieces, in order."""
+            n = int(sum(m for _, m in segs))
+            kI = torch.empty((n, dcfg.d_I), dtype=torch.uint8, device=dev)
+            K = torch.empty((n, dcfg.Hkv, dcfg.d), dtype=bf, device=dev)
+            V = torch.empty_like(K)
+            at = 0
+            for s0, m in segs:
+                for c0 in range(0, m, 1 << 19):
+                    c1 = min(m, c0 + (1 << 19))
+                    r0, r1 = s0 + c0, s0 + c1
+                    kI[at + c0:at + c1].copy_(torch.from_numpy(gen.decode_kI_rows(dcfg, r0, r1)))
+                    K[at + c0:at + c1].copy_(torch.from_numpy(
+                        gen.decode_K_rows(dcfg, r0, r1).view(np.int16)).view(bf))
+                    V[at + c0:at + c1].copy_(torch.from_numpy(
+                        gen.decode_V_rows(dcfg, r0, r1).view(np.int16)).view(bf))
+                at += m
+            return kI, K, V
+
+        if args.decode_shard == "batch":
+            seqs = dist.deal_sequences(lens, world)[rank]
+            kI, K, V = cache_rows([(int(off[b]), int(lens[b])) for b in seqs])
+            off_r = np.concatenate([[0], np.cumsum(lens[seqs])]).astype(np.int64)
+            if not seqs:
+                off_r = np.zeros(1, np.int64)
+            Df = dict(mode="batch", seqs=seqs, q_I=t_(q["q_I"][seqs]), w=t_(q["w"][seqs]),
+                      Q=t_(q["Q"][seqs].view(np.int16), bf), kI=kI, K=K, V=V, off=t_(off_r),
+                      O=torch.empty((len(seqs), dcfg.Hq, dcfg.d), dtype=bf, device=dev),
+                      idx=torch.empty((len(seqs), dcfg.k), dtype=torch.int32, device=dev))
+            Df["ws"] = torch.empty(dsa.decode_workspace_size(
+                len(seqs), int(off_r[-1]), dcfg.H_I, dcfg.d_I, dcfg.k, dcfg.Hq, dcfg.Hkv, dcfg.d),
+                dtype=torch.uint8, device=dev)
+        else:
+            part = shards.cache_parts(lens, world)[rank]
+            kI, K, V = cache_rows([(int(off[b]) + int(part["base"][b]), int(part["lens"][b]))
+                                   for b in range(dcfg.B)])
+            Df = dict(mode="cache", q_I=t_(q["q_I"]), w=t_(q["w"]), Q=t_(q["Q"].view(np.int16), bf),
+                      kI=kI, K=K, V=V, off=t_(part["off"]), base=t_(part["base"]), work={})
+
+    def prefill():
+        if not Pf:
+            return
+        for name in ("k_I", "K", "V"):
+            dist.gather_zigzag(Pf["own"][name], Pf["keys"][name], pcfg.L, world)
+        dist.prefill_rows_step(dsa, Pf["rows"], Pf["mine"], Pf["keys"], pcfg.k, pcfg.scale,
+                               stream=stream)
+
+    def decode():
+        if not Df:
+            return
+        if Df["mode"] == "batch":
+            if Df["seqs"]:
+                dsa.sparse_attn_decode(Df["q_I"], Df["w"], Df["Q"], Df["kI"], Df["K"], Df["V"],
+                                       Df["off"], dcfg.k, dcfg.scale, O=Df["O"],
+                                       idx_out=Df["idx"], workspace=Df["ws"], stream=stream)
+        else:
+            dist.decode_cache_step(dsa, Df["q_I"], Df["w"], Df["Q"], Df["kI"], Df["K"], Df["V"],
+                                   Df["off"], Df["base"], dcfg.k, dcfg.scale, world,
+                                   stream=stream, work=Df["work"])
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        prefill()
+        decode()
+    torch.cuda.synchronize()
+    if dsa.device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = Clocks(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ
+                    else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    tdist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        prefill()
+        evs[i][1].record(stream)
+        decode()
+        evs[i][2].record(stream)
+    torch.cuda.synchronize()
+    tdist.barrier()
+    clk = clocks.stop()
+    if dsa.device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+    t_p = sum(e[0].elapsed_time(e[1]) for e in evs)
+    t_d = sum(e[1].elapsed_time(e[2]) for e in evs)
+    tot = max_over_ranks([t_p, t_d], world, device=dev)
+    K_ = args.steps
+    prefill_ms, decode_ms = tot[0] / K_, tot[1] / K_
+
+    # ---- end to end: every step copies the rank's inputs from pinned host
+    # memory and its output rows back
+    e2e = None
+    if e2e_on:
+        outs = (Pf["mine"]["O"] if Pf else []) + ([Df["O"]] if Df.get("mode") == "batch" else [])
+        d2h = [(torch.empty(o.shape, dtype=o.dtype).pin_memory(), o) for o in outs]
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
+        tdist.barrier()
+        torch.cuda.synchronize()
+        for i in range(K_):
+            flush.zero_()
+            ev2[i][0].record(stream)
+            for h, d_ in h2d:
+                d_.copy_(h, non_blocking=True)
+            prefill()
+            decode()
+            for h, d_ in d2h:
+                h.copy_(d_, non_blocking=True)
+            ev2[i][1].record(stream)
+        torch.cuda.synchronize()
+        tdist.barrier()
+        et = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in ev2)], world, device=dev)[0]
+        bi = sum(h.numel() * h.element_size() for h, _ in h2d)
+        bo = sum(h.numel() * h.element_size() for h, _ in d2h)
+        e2e = dict(value=(pcfg.L / (et / K_ / 1e3)) if pcfg else 0.0, unit="query-tokens/s",
+                   h2d_bytes_per_step=int(bi), d2h_bytes_per_step=int(bo),
+                   ms_per_step=float(et / K_), note="rank 0's bytes; every rank copies its own")
+    launches = (4 if pcfg else 0) + (4 if (dcfg and args.decode_shard == "batch") else
+                                     (6 if dcfg else 0))
+    par = []
+    if pcfg:
+        par.append(f"prefill: {2 * world} zig-zag row blocks, NCCL all-gather of k_I/K/V")
+    if dcfg:
+        par.append("decode: batch shards" if args.decode_shard == "batch" else
+                   "decode: cache shards, NCCL all-gather of top-k pairs and partials")
+    return dict(value=(pcfg.L / (prefill_ms / 1e3)) if pcfg else 0.0, prefill_ms=prefill_ms,
+                decode_ms=decode_ms, decode_tps=(dcfg.B / (decode_ms / 1e3)) if dcfg else 0.0,
+                clocks=clk, launches=launches * K_, pcfg=pcfg, dcfg=dcfg, parallelism="; ".join(par),
+                e2e=e2e)
 
 
 # ------------------------------------------------------------------ oracle timing
@@ -464,7 +735,12 @@ def oracle_prefill_rows(pcfg, host, rows, nthreads=0):
                        nthreads=nthreads, idx_by_row=True)
 
 
-def cpu_baseline(pcfg, host, seconds):
+def cpu_baseline(pcfg, host, seconds, dcfg=None):
+    """The oracle on this host's cores: prefill rows per second on a
+    stratified sample of the workload's rows (the sample's mean causal length
+    matches the sequence's, so the rate extrapolates to the whole prefill by
+    the row count), and decode tokens per second on the decode workload's two
+    shortest sequences (extrapolated to the batch by cached rows)."""
     cores = os.cpu_count() or 1
     # calibrate on a small stratified sample, then size the timed sample
     probe = sample_rows(pcfg.L, max(cores, 8), seed=1)
@@ -476,10 +752,32 @@ def cpu_baseline(pcfg, host, seconds):
     t0 = time.perf_counter()
     oracle_prefill_rows(pcfg, host, rows)
     dt = time.perf_counter() - t0
-    return dict(value=n / dt, unit="query-tokens/s", cores=cores, kind="oracle",
-                sample=f"{n} query rows stratified over t in [0, {pcfg.L}) of the "
-                       f"{pcfg.name} workload (indexer + top-k + attention per row), "
-                       f"{dt:.1f} s")
+    out = dict(value=n / dt, unit="query-tokens/s", cores=cores, kind="oracle",
+               extrapolated=True, rows=n,
+               sample=f"{n} query rows stratified over t in [0, {pcfg.L}) of the "
+                      f"{pcfg.name} workload (indexer + top-k + attention per row), "
+                      f"{dt:.1f} s; rate extrapolated to all {pcfg.L} rows")
+    if dcfg is not None:
+        import oracle
+        off = gen.decode_offsets(dcfg)
+        lens = np.diff(off)
+        seqs = [int(b) for b in np.argsort(lens)[:2]]
+        q = gen.decode_queries(dcfg)
+        sub = np.concatenate([[0], np.cumsum(lens[seqs])]).astype(np.int64)
+        kI = np.concatenate([gen.decode_kI_rows(dcfg, off[b], off[b + 1]) for b in seqs])
+        K = np.concatenate([gen.decode_K_rows(dcfg, off[b], off[b + 1]) for b in seqs])
+        V = np.concatenate([gen.decode_V_rows(dcfg, off[b], off[b + 1]) for b in seqs])
+        t0 = time.perf_counter()
+        oracle.decode(q["q_I"][seqs], q["w"][seqs], q["Q"][seqs], kI, K, V, sub, dcfg.k,
+                      dcfg.scale)
+        dd = time.perf_counter() - t0
+        rows_per_s = float(sub[-1]) / dd
+        out["decode"] = dict(value=rows_per_s / float(lens.sum()) * dcfg.B, unit="tokens/s",
+                             extrapolated=True,
+                             sample=f"sequences {seqs} ({int(sub[-1])} cached rows), {dd:.1f} s; "
+                                    f"rate per cached row extrapolated to the batch's "
+                                    f"{int(lens.sum())} rows")
+    return out
 
 
 def workload_config(pcfg, dcfg, world=1):
@@ -751,11 +1049,27 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                  device_id=torch.device("cuda", local_rank))
     try:
-        r = run_ours(args, rank, world, local_rank)
+        if world > 1 and not args.replicas:
+            r = run_sharded(args, rank, world, local_rank)
+        else:
+            r = run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             tdist.destroy_process_group()
     if rank != 0:
+        return
+    if "parallelism" in r:
+        pcfg, dcfg = r["pcfg"], r["dcfg"]
+        cfg = workload_config(pcfg, dcfg, world)
+        cfg["parallelism"] = r["parallelism"]
+        print(json.dumps(dict(
+            metric=METRIC, value=r["value"], unit="query-tokens/s", n_gpus=world,
+            steps=args.steps, warmup=args.warmup, ms_per_step=r["prefill_ms"] + r["decode_ms"],
+            higher_is_better=True, scaling="strong", vs_baseline=None, dtype="fp8-e4m3/bf16",
+            data="synthetic", config=cfg,
+            decode=dict(value=r["decode_tps"], unit="tokens/s", ms_per_step=r["decode_ms"]),
+            prefill_ms=r["prefill_ms"], clocks=r["clocks"], gpu_launches=r["launches"],
+            **({"e2e": r["e2e"]} if r["e2e"] else {}))), flush=True)
         return
     pcfg, dcfg = r["pcfg"], r["dcfg"]
     out = dict(
@@ -773,6 +1087,8 @@ def main():
         out["e2e"] = r["e2e"]
     if r["cpu"] is not None:
         out["cpu_baseline"] = r["cpu"]
+    if r.get("others"):
+        out["configs"] = r["others"]
     print(json.dumps(out), flush=True)
 
 

@@ -174,10 +174,16 @@ attn_kernel(const Params p) {
                 if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ((c / kStages) - 1) & 1);
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
             }
-            const int64_t sl = sg - koff;
-            if (sg >= 0 && sl >= nkeys && !p.skip_foreign) record_device_error(2);
-            const bool valid = sg >= 0 && sl >= 0 && sl < nkeys;
-            const int32_t si = valid ? (int32_t)sl : -1;
+            int32_t si;
+            if constexpr (SPLIT) {  // global keys of a cache shard, or sequence-local ones
+                const int64_t sl = sg - koff;
+                if (sg >= 0 && sl >= nkeys && !p.skip_foreign) record_device_error(2);
+                si = sg >= 0 && sl >= 0 && sl < nkeys ? (int32_t)sl : -1;
+            } else {
+                si = (int32_t)sg;
+                if (si >= nkeys) record_device_error(2);
+            }
+            const bool valid = si >= 0 && si < nkeys;
             const uint32_t bal = __ballot_sync(0xffffffffu, valid);
             const uint32_t sbase = smem_u32(smem + s * C::STAGE);
             if (bal) {
