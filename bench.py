@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--prefill-config", type=int, default=gen.PREFILL_128K.id,
                     help="workload id of the prefill part (0: no prefill part)")
+    ap.add_argument("--prefill-L", type=int, default=0,
+                    help="run the prefill workload at this sequence length instead of its own "
+                         "(a smaller case of the same recipe, for profiling)")
     ap.add_argument("--decode-config", type=int, default=gen.DECODE_B64.id,
                     help="workload id of the decode part (0: no decode part)")
     ap.add_argument("--decode-batch", type=int, default=0,
@@ -118,17 +121,15 @@ def decode_bytes(cfg, lens) -> float:
 
 # ------------------------------------------------------------------ DRAM traffic
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch,
-# from one ncu capture of the prefill L=32768 case (its summary under
-# profiles/ncu_prefill32k_decode4_index_attn.md), per prefill query token:
-# the indexer's DRAM traffic is its queries, weights and index rows (the keys
-# stay in L2), so it grows with L.  Valid only for the kernel sources the
-# counters were taken on (the SHA-256 of the files listed); otherwise null.
-TRAFFIC = {
-    "dsa_index_topk": dict(bytes_per_query_token=(282554880 + 228671232) / 32768,
-                           sources=("index_topk.cuh", "topk_select.cuh", "ptx.cuh"),
-                           src_sha256="f56f3ee75da1563ddaf911e63c7f34293912a3187bf81711c5c279f1b18ad11c"),
-}
+# DRAM bytes of one launch per unit of work, from the committed measurement
+# record of single-kernel ncu captures (profiles/dram_traffic.json); valid
+# only for the kernel sources the counters were taken on.
+def traffic_record() -> dict:
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
 
 
 def csrc_sha256(sources) -> str:
@@ -143,10 +144,37 @@ def csrc_sha256(sources) -> str:
 
 
 def dram_traffic(kernel: str, pcfg):
-    t = TRAFFIC.get(kernel)
-    if t is None or pcfg is None or t["src_sha256"] != csrc_sha256(t["sources"]):
-        return None
-    return t["bytes_per_query_token"] * pcfg.L
+    """(bytes per launch or None, why) for the bench's prefill workload."""
+    t = traffic_record().get(kernel)
+    if t is None or pcfg is None:
+        return None, "no capture"
+    if not t.get("scales_with_units"):
+        return None, f"measured at {t['workload']}; does not scale with L"
+    if t["src_sha256"] != csrc_sha256(t["sources"]):
+        return None, "kernel sources changed since the capture"
+    per = (t["dram_read_bytes"] + t["dram_write_bytes"]) / t["units"]
+    return per * pcfg.L, f"{t['summary']}, scaled by L from {t['workload']}"
+
+
+def l2_copy_peak(torch) -> float:
+    """GB/s of a device-to-device copy whose source and destination (32 MiB
+    each) stay in L2: the bound of a kernel whose reads hit L2 (read + write
+    bytes, best of 20)."""
+    a = torch.empty(8 << 20, dtype=torch.float32, device="cuda")
+    b = torch.empty_like(a)
+    a.fill_(1.0)
+    for _ in range(5):
+        b.copy_(a)
+    best = 0.0
+    for _ in range(20):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            b.copy_(a)
+        e1.record()
+        torch.cuda.synchronize()
+        best = max(best, 10 * 2 * a.numel() * 4 / (e0.elapsed_time(e1) / 1e3) / 1e9)
+    return best
 
 
 # ------------------------------------------------------------------ ranks
@@ -292,6 +320,8 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     pcfg = gen.CONFIGS[args.prefill_config] if args.prefill_config else None
+    if pcfg is not None and args.prefill_L:
+        pcfg = pcfg.with_(L=args.prefill_L, name=f"{pcfg.name} at L={args.prefill_L}")
     dcfg = gen.CONFIGS[args.decode_config] if args.decode_config else None
     if dcfg is not None and args.decode_batch:
         dcfg = dcfg.with_(B=args.decode_batch)
@@ -384,10 +414,14 @@ def run_ours(args, rank, world, local_rank):
         kernels["dsa_index_topk"] = dict(
             bound="tensor", ms=ms_idx, work=prefill_flops(pcfg),
             achieved=prefill_flops(pcfg) / (ms_idx / 1e3) / 1e12, peak=fp8_peak, unit="TFLOP/s")
+        # the gathered rows mostly hit L2 (94 % at L = 65536): its bound is
+        # L2 bandwidth, measured here as an L2-resident copy
+        l2pk = l2_copy_peak(torch)
         kernels["dsa_sparse_attn_prefill"] = dict(
-            bound="hbm", ms=ms_att, work=prefill_attn_bytes(pcfg),
-            achieved=prefill_attn_bytes(pcfg) / (ms_att / 1e3) / 1e9, peak=pk["hbm"],
-            unit="GB/s")
+            bound="l2", ms=ms_att, work=prefill_attn_bytes(pcfg),
+            achieved=prefill_attn_bytes(pcfg) / (ms_att / 1e3) / 1e9, peak=l2pk,
+            peak_source="measured here: L2-resident device copy (read + write bytes)",
+            unit="GB/s", hbm_peak=pk["hbm"])
     if dcfg:
         kernels["dsa_sparse_attn_decode"] = dict(
             bound="hbm", ms=ms_dec, work=decode_bytes(dcfg, lens),
@@ -397,9 +431,9 @@ def run_ours(args, rank, world, local_rank):
         v["frac"] = v["achieved"] / v["peak"]
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     dk = kernels[dom]
-    traffic = dram_traffic(dom, pcfg)
+    traffic, traffic_src = dram_traffic(dom, pcfg)
     roofline = dict(bound=dk["bound"], achieved=dk["achieved"], peak=dk["peak"], unit=dk["unit"],
-                    frac=dk["frac"], traffic=traffic, kernel=dom,
+                    frac=dk["frac"], traffic=traffic, traffic_source=traffic_src, kernel=dom,
                     peak_source=f"{pk['src']} ({'2 x sustained bf16' if dk['bound'] == 'tensor' else 'hbm copy'})")
 
     # ---- end to end through the public API with host buffers
@@ -468,6 +502,7 @@ def other_configs(torch, dsa, pk, args, stream, flush):
     video workload), with the same rooflines; min(steps, 5) timed steps."""
     out = {}
     fp8_peak = 2.0 * pk["bf16_sus"]
+    l2pk = l2_copy_peak(torch)
     for cfg in (gen.TINY_PREFILL, gen.PREFILL_32K, gen.VIDEO_256K):
         h = gen.prefill_inputs(cfg)
         t = {n: torch.from_numpy(h[n]).cuda() for n in ("q_I", "k_I", "w")}
@@ -508,9 +543,9 @@ def other_configs(torch, dsa, pk, args, stream, flush):
             kernels={"dsa_index_topk": dict(bound="tensor", ms=mi, achieved=fl / (mi / 1e3) / 1e12,
                                             peak=fp8_peak, unit="TFLOP/s",
                                             frac=fl / (mi / 1e3) / 1e12 / fp8_peak),
-                     attn.__name__: dict(bound="l2 (gathered rows)", ms=ma,
-                                         achieved=by / (ma / 1e3) / 1e9, unit="GB/s",
-                                         hbm_frac=by / (ma / 1e3) / 1e9 / pk["hbm"])})
+                     attn.__name__: dict(bound="l2", ms=ma, achieved=by / (ma / 1e3) / 1e9,
+                                         peak=l2pk, unit="GB/s",
+                                         frac=by / (ma / 1e3) / 1e9 / l2pk)})
         del t, bf, idx, O
         torch.cuda.empty_cache()
     return out
@@ -532,6 +567,8 @@ def run_sharded(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     pcfg = gen.CONFIGS[args.prefill_config] if args.prefill_config else None
+    if pcfg is not None and args.prefill_L:
+        pcfg = pcfg.with_(L=args.prefill_L, name=f"{pcfg.name} at L={args.prefill_L}")
     dcfg = gen.CONFIGS[args.decode_config] if args.decode_config else None
     if dcfg is not None and args.decode_batch:
         dcfg = dcfg.with_(B=args.decode_batch)
