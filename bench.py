@@ -156,24 +156,32 @@ def dram_traffic(kernel: str, pcfg):
     return per * pcfg.L, f"{t['summary']}, scaled by L from {t['workload']}"
 
 
-def l2_copy_peak(torch) -> float:
-    """GB/s of a device-to-device copy whose source and destination (32 MiB
-    each) stay in L2: the bound of a kernel whose reads hit L2 (read + write
-    bytes, best of 20)."""
-    a = torch.empty(8 << 20, dtype=torch.float32, device="cuda")
-    b = torch.empty_like(a)
-    a.fill_(1.0)
-    for _ in range(5):
-        b.copy_(a)
+def l2_read_peak(torch) -> float:
+    """GB/s of reads that hit L2: 16-byte ld.global.cg loads over a buffer
+    small enough to stay in L2 (24 or 48 MiB), 100 passes, best of the
+    sizes and of 5 runs (libdsa_probe.so, a measurement utility built beside
+    the library).  The bound of a kernel whose gathered rows hit L2."""
+    import ctypes
+    from sparse_long_context_02_b200 import build as dsa_build
+    L = ctypes.CDLL(dsa_build.build_probe())
+    L.dsa_probe_l2_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_void_p, ctypes.c_void_p]
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    sink = torch.zeros(4, dtype=torch.int32, device="cuda")
+    st = torch.cuda.current_stream()
     best = 0.0
-    for _ in range(20):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(10):
-            b.copy_(a)
-        e1.record()
-        torch.cuda.synchronize()
-        best = max(best, 10 * 2 * a.numel() * 4 / (e0.elapsed_time(e1) / 1e3) / 1e9)
+    for mib in (24, 48):
+        buf = torch.ones((mib << 20) // 4, dtype=torch.float32, device="cuda")
+        for rep in range(6):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            if L.dsa_probe_l2_read(buf.data_ptr(), buf.numel() * 4, 100, 4 * sms,
+                                   sink.data_ptr(), st.cuda_stream) != 0:
+                raise RuntimeError("L2 probe launch failed")
+            e1.record(st)
+            torch.cuda.synchronize()
+            if rep:  # the first run warms the buffer into L2
+                best = max(best, 100 * buf.numel() * 4 / (e0.elapsed_time(e1) / 1e3) / 1e9)
     return best
 
 
@@ -415,12 +423,12 @@ def run_ours(args, rank, world, local_rank):
             bound="tensor", ms=ms_idx, work=prefill_flops(pcfg),
             achieved=prefill_flops(pcfg) / (ms_idx / 1e3) / 1e12, peak=fp8_peak, unit="TFLOP/s")
         # the gathered rows mostly hit L2 (94 % at L = 65536): its bound is
-        # L2 bandwidth, measured here as an L2-resident copy
-        l2pk = l2_copy_peak(torch)
+        # L2 read bandwidth, measured here
+        l2pk = l2_read_peak(torch)
         kernels["dsa_sparse_attn_prefill"] = dict(
             bound="l2", ms=ms_att, work=prefill_attn_bytes(pcfg),
             achieved=prefill_attn_bytes(pcfg) / (ms_att / 1e3) / 1e9, peak=l2pk,
-            peak_source="measured here: L2-resident device copy (read + write bytes)",
+            peak_source="measured here: L2-resident 16-byte reads (libdsa_probe.so)",
             unit="GB/s", hbm_peak=pk["hbm"])
     if dcfg:
         kernels["dsa_sparse_attn_decode"] = dict(
@@ -496,13 +504,34 @@ def run_ours(args, rank, world, local_rank):
                 launches=launches_per_step * K, pcfg=pcfg, dcfg=dcfg, others=others)
 
 
+def dedup_attn_bytes(torch, cfg, idx, G: int) -> float:
+    """Bytes the adjacent-query dedup attention moves: the K and V rows of
+    every distinct key of each block of G consecutive queries, plus Q, O and
+    the index rows (counted on the device from the index rows)."""
+    L, k = idx.shape
+    nb = (L + G - 1) // G
+    pad = nb * G - L
+    total = 0
+    for b0 in range(0, nb, 2048):
+        b1 = min(nb, b0 + 2048)
+        x = idx[b0 * G:min(L, b1 * G)]
+        if b1 == nb and pad:
+            x = torch.cat([x, torch.full((pad, k), -1, dtype=x.dtype, device=x.device)])
+        x, _ = torch.sort(x.reshape(b1 - b0, G * k), dim=1)
+        new = torch.ones_like(x, dtype=torch.bool)
+        new[:, 1:] = x[:, 1:] != x[:, :-1]
+        total += int(((x >= 0) & new).sum().item())
+    row = 2 * cfg.Hkv * cfg.d * 2
+    return total * row + L * (2 * cfg.Hq * cfg.d * 2 + 4 * k)
+
+
 def other_configs(torch, dsa, pk, args, stream, flush):
     """The other prefill workloads (tiny, 32K, 256K video), each timed as its
     own steps (indexer + top-k, then attention; the dedup attention on the
     video workload), with the same rooflines; min(steps, 5) timed steps."""
     out = {}
     fp8_peak = 2.0 * pk["bf16_sus"]
-    l2pk = l2_copy_peak(torch)
+    l2pk = l2_read_peak(torch)
     for cfg in (gen.TINY_PREFILL, gen.PREFILL_32K, gen.VIDEO_256K):
         h = gen.prefill_inputs(cfg)
         t = {n: torch.from_numpy(h[n]).cuda() for n in ("q_I", "k_I", "w")}
@@ -537,6 +566,8 @@ def other_configs(torch, dsa, pk, args, stream, flush):
         mi = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
         ma = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
         fl, by = prefill_flops(cfg), prefill_attn_bytes(cfg)
+        if cfg.video:  # the dedup kernel gathers each distinct key of a 6-query block once
+            by = dedup_attn_bytes(torch, cfg, idx, 6)
         out[cfg.name] = dict(
             steps=n, ms_per_step=mi + ma, value=cfg.L / ((mi + ma) / 1e3),
             unit="query-tokens/s",

@@ -9,6 +9,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB_PATH = os.path.join(HERE, "libdsa_b200.so")
 SOURCES = [os.path.join(CSRC, "dsa_lib.cu")]
+# the benchmark's L2 bandwidth probe: a separate library, not part of the ABI
+PROBE_SOURCE = os.path.join(CSRC, "probe_l2.cu")
+PROBE_PATH = os.path.join(HERE, "libdsa_probe.so")
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(ROOT, "include", "dsa.h")]
 
@@ -25,7 +28,18 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
+def build_probe(force: bool = False) -> str:
+    if (not force and os.path.exists(PROBE_PATH)
+            and os.path.getmtime(PROBE_PATH) >= os.path.getmtime(PROBE_SOURCE)):
+        return PROBE_PATH
+    tmp = PROBE_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call([nvcc(), *NVCC_FLAGS, "-o", tmp, PROBE_SOURCE])
+    os.replace(tmp, PROBE_PATH)
+    return PROBE_PATH
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    build_probe(force)
     if (not force and os.path.exists(LIB_PATH)
             and os.path.getmtime(LIB_PATH) >= max(os.path.getmtime(d) for d in DEPS)):
         return LIB_PATH
