@@ -160,7 +160,6 @@ __device__ __forceinline__ bool make_segment(const Params& p, int b, int64_t r0,
 __global__ void __launch_bounds__(kThreads, 1)
 index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
              const Params p) {
-    bind_error_word(p.err);
     constexpr int N = HI;
     constexpr int KT_BYTES = kKeyTile * DI;
     constexpr uint32_t TMEM_COLS = 512;  // 4 warpgroups x 2 accumulators x 64 columns
@@ -173,7 +172,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     const int64_t r1 = r0 + p.R < p.total_n ? r0 + p.R : p.total_n;
     if (r0 >= r1) return;  // more CTAs than ranges: nothing to do
 
-    extern __shared__ __align__(16) uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     // Aligned by pointer arithmetic on the shared array itself (not through an
     // integer), so that the compiler keeps every access in the shared window
     // (ld/st.shared with 32-bit addresses instead of generic ones).
@@ -221,7 +220,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             for (int b = b_first; ok && b < p.B && p.cache_off[b] < r1; ++b) {
                 if (!make_segment(p, b, r0, r1, g)) continue;
                 // the previous segment's MMAs must be done with the query block
-                if (nseg > 0 && !mbar_wait(smem_u32(&misc->qfree), (nseg - 1) & 1)) {
+                if (nseg > 0 && !mbar_wait_to(p.err, smem_u32(&misc->qfree), (nseg - 1) & 1)) {
                     misc->abort_flag = 1;
                     break;
                 }
@@ -235,7 +234,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                         if (misc->abort_flag) { ok = false; break; }
                         const int s = i % kStages;
                         if (i >= kStages &&
-                            !mbar_wait(smem_u32(&misc->empty[s]), ((i / kStages) - 1) & 1)) {
+                            !mbar_wait_to(p.err, smem_u32(&misc->empty[s]), ((i / kStages) - 1) & 1)) {
                             misc->abort_flag = 1;
                             ok = false;
                             break;
@@ -249,9 +248,9 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                     }
             }
             // Never leave with a copy in flight.
-            if (nseg > 0) mbar_wait(qbar, (nseg - 1) & 1);
+            if (nseg > 0) mbar_wait_to(p.err, qbar, (nseg - 1) & 1);
             for (int e = i - kStages < 0 ? 0 : i - kStages; e < i; ++e)
-                mbar_wait(smem_u32(&misc->full[e % kStages]), (e / kStages) & 1);
+                mbar_wait_to(p.err, smem_u32(&misc->full[e % kStages]), (e / kStages) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
@@ -263,7 +262,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             Segment g;
             for (int b = b_first; ok && b < p.B && p.cache_off[b] < r1; ++b) {
                 if (!make_segment(p, b, r0, r1, g)) continue;
-                ok = mbar_wait(smem_u32(&misc->qfull), nseg & 1);
+                ok = mbar_wait_to(p.err, smem_u32(&misc->qfull), nseg & 1);
                 ++nseg;
                 const int nt0 = g.tiles(0);
                 for (int u = 0; ok && u < nt0; ++u)
@@ -274,9 +273,9 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                         const int s = i % kStages;
                         const int use = uses[w]++;
                         const int buf = use & 1;
-                        ok = mbar_wait(smem_u32(&misc->full[s]), (i / kStages) & 1);
+                        ok = mbar_wait_to(p.err, smem_u32(&misc->full[s]), (i / kStages) & 1);
                         if (ok && use >= 2)
-                            ok = mbar_wait(smem_u32(&misc->accempty[w][buf]), ((use >> 1) - 1) & 1);
+                            ok = mbar_wait_to(p.err, smem_u32(&misc->accempty[w][buf]), ((use >> 1) - 1) & 1);
                         if (!ok) continue;
                         tc_fence_after();
                         const uint64_t adesc =
@@ -294,7 +293,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             }
             if (!ok) misc->abort_flag = 1;
             umma_commit(smem_u32(&misc->mma_done));
-            mbar_wait(smem_u32(&misc->mma_done), 0);
+            mbar_wait_to(p.err, smem_u32(&misc->mma_done), 0);
         }
     } else {
         // ------------------------------------------------ epilogue (warps 0-15)
@@ -333,7 +332,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                     if (u >= ntw) continue;
                     const int buf = use & 1;
                     if (!misc->abort_flag &&
-                        !mbar_wait(smem_u32(&misc->accfull[w][buf]), (use >> 1) & 1))
+                        !mbar_wait_to(p.err, smem_u32(&misc->accfull[w][buf]), (use >> 1) & 1))
                         misc->abort_flag = 1;
                     tc_fence_after();
                     const uint32_t taddr =
@@ -406,7 +405,6 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
 // smem_cap entries, else in place in the candidate arrays), then selected.
 __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* idx_out,
                                                       int smem_cap) {
-    bind_error_word(p.err);
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ Scratch<1024> S;
     __shared__ int total_s;
@@ -427,7 +425,7 @@ __global__ void __launch_bounds__(1024) merge_kernel(const Params p, int32_t* id
     } else if (tid == 0 && !(p.allow_empty && ordered && p.cache_off[b] >= 0 &&
                              p.cache_off[b] == p.cache_off[b + 1] &&
                              p.cache_off[b] <= p.total_n)) {
-        record_device_error(2);
+        record_error_to(p.err, 2);
     }
     if (s1 <= s0) {
         for (int e = tid; e < p.k; e += 1024) {
@@ -531,7 +529,6 @@ constexpr int kMaxShards = 8;
 __global__ void __launch_bounds__(1024) merge_shards_kernel(const uint32_t* ord_in,
                                                              const int32_t* key_in, int P, int B,
                                                              int k, int32_t* idx_out, int* err) {
-    bind_error_word(err);
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ Scratch<1024> S;
     __shared__ int cnt_s[kMaxShards + 1];
@@ -567,7 +564,7 @@ __global__ void __launch_bounds__(1024) merge_shards_kernel(const uint32_t* ord_
     __syncthreads();
     // keys must ascend along the gathered run (the output is written in it)
     for (int e = tid; e + 1 < n; e += 1024)
-        if (si[e] >= si[e + 1]) record_device_error(2);
+        if (si[e] >= si[e + 1]) record_error_to(err, 2);
     int32_t* out = idx_out + (int64_t)b * k;
     const FlatAccess a{so, si};
     int cnt = n;

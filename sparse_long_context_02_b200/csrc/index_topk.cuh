@@ -205,7 +205,6 @@ template <int HI, int DI, bool TOPK>
 __global__ void __launch_bounds__(kThreads, 1)
 index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
              const Params p) {
-    bind_error_word(p.err);
     constexpr int N = kTokens * HI;
     constexpr int KT_BYTES = kKeyTile * DI;
     constexpr int Q_BYTES = N * DI;
@@ -214,7 +213,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     static_assert(N % 16 == 0 && N <= 256, "MMA N");
     static_assert(DI == 64 || DI == 128, "d_I");
 
-    extern __shared__ __align__(16) uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     // Aligned by pointer arithmetic on the shared array itself (not through an
     // integer), so that the compiler keeps every access in the shared window
     // (ld/st.shared with 32-bit addresses instead of generic ones).
@@ -238,7 +237,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                             : (int)((L + kKeyTile - 1) / kKeyTile);  // tiles tile0, tile0 + 1, ...
     if (TOPK && p.cu_seqlens != nullptr && blockIdx.x == 0 && threadIdx.x == 0 &&
         (p.cu_seqlens[0] != 0 || (int64_t)p.cu_seqlens[p.nseq] != L))
-        record_device_error(2);  // cu_seqlens must run from 0 to L
+        record_error_to(p.err, 2);  // cu_seqlens must run from 0 to L
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -281,7 +280,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 if (misc->abort_flag) break;
                 const int s = i % kStages;
                 if (i >= kStages &&
-                    !mbar_wait(smem_u32(&misc->empty[s]), ((i / kStages) - 1) & 1)) {
+                    !mbar_wait_to(p.err, smem_u32(&misc->empty[s]), ((i / kStages) - 1) & 1)) {
                     misc->abort_flag = 1;
                     break;
                 }
@@ -292,21 +291,21 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 issued = i + 1;
             }
             // Never leave with a copy in flight.
-            mbar_wait(qbar, 0);
+            mbar_wait_to(p.err, qbar, 0);
             for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
-                mbar_wait(smem_u32(&misc->full[i % kStages]), (i / kStages) & 1);
+                mbar_wait_to(p.err, smem_u32(&misc->full[i % kStages]), (i / kStages) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            bool ok = mbar_wait(smem_u32(&misc->qfull), 0);
+            bool ok = mbar_wait_to(p.err, smem_u32(&misc->qfull), 0);
             const uint64_t bdesc = smem_desc_kmajor(smem_u32(smem + lay.q), DI);
             for (int i = 0; ok && i < ntiles; ++i) {
                 if (misc->abort_flag) break;
                 const int s = i % kStages;
                 const int buf = i & 1;
-                ok = mbar_wait(smem_u32(&misc->full[s]), (i / kStages) & 1);
-                if (ok && i >= 2) ok = mbar_wait(smem_u32(&misc->accempty[buf]), ((i >> 1) - 1) & 1);
+                ok = mbar_wait_to(p.err, smem_u32(&misc->full[s]), (i / kStages) & 1);
+                if (ok && i >= 2) ok = mbar_wait_to(p.err, smem_u32(&misc->accempty[buf]), ((i >> 1) - 1) & 1);
                 if (!ok) break;
                 tc_fence_after();
                 const uint64_t adesc =
@@ -322,7 +321,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             if (!ok) misc->abort_flag = 1;
             // All MMAs of this CTA retired before TMEM is released.
             umma_commit(smem_u32(&misc->mma_done));
-            mbar_wait(smem_u32(&misc->mma_done), 0);
+            mbar_wait_to(p.err, smem_u32(&misc->mma_done), 0);
         }
     } else if (warp < kEpiWarps) {
         // ------------------------------------------------ epilogue (warps 0-15)
@@ -367,7 +366,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
                 o[u] = 0;
                 if (i >= ntiles) continue;
                 const int buf = i & 1;
-                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->accfull[buf]), (i >> 1) & 1))
+                if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->accfull[buf]), (i >> 1) & 1))
                     misc->abort_flag = 1;
                 tc_fence_after();
                 const uint32_t taddr =

@@ -196,7 +196,7 @@ __device__ __forceinline__ void qk_bf16(float (&S)[8][4], const uint32_t (&qa)[D
 // Grid (ntiles, Hq); the longest query tiles first.
 template <int D>
 __global__ void __launch_bounds__(kThreads) head_lse_kernel(const Params p) {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const int qt = p.ntiles - 1 - blockIdx.x, h = blockIdx.y;
     const int g = h / (p.Hq / p.Hkv);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kThreads) head_lse_kernel(const Params p) {
 // only write G = 0.  Grid (ntiles keys, ntiles queries).
 template <int D>
 __global__ void __launch_bounds__(kThreads) target_kernel(const Params p) {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const int kt = blockIdx.x, qt = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
     const int64_t t_a = (int64_t)qt * kTile + warp * 16 + r, t_b = t_a + 8;
@@ -486,7 +486,7 @@ __device__ __forceinline__ void ds_times_rows(float (&acc)[DI / 8][4], const flo
 // heads of one query tile run side by side and share its G band in L2.
 template <int DI>
 __global__ void __launch_bounds__(kThreads) dq_kernel(const Params p) {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const int qt = p.ntiles - 1 - blockIdx.y, j = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
     const int64_t t_a = (int64_t)qt * kTile + warp * 16 + r, t_b = t_a + 8;
@@ -567,7 +567,7 @@ constexpr int kWStride = kTile + 1;
 
 template <int DI>
 __global__ void __launch_bounds__(kThreads) dk_kernel(const Params p) {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const int split = blockIdx.x, kt = blockIdx.y;
     const int hps = p.HI / p.nsplit, j0 = split * hps;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;

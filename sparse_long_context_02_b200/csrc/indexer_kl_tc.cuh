@@ -223,7 +223,6 @@ __device__ __forceinline__ void put_bf_tile(const BfPieces& P, uint32_t tile, in
 // Grid (HI, ceil(L / 128)): the heads of one query tile run side by side;
 // the longest query tiles first.
 __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) {
-    bind_error_word(p.err);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Misc* misc = reinterpret_cast<Misc*>(smem + kMisc);
@@ -263,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) 
             const uint64_t adesc_q = sdesc_sw128(sb + kQ, 16, 1024);
             auto dq_tile = [&](int kt) {
                 const int b = kt & 1, st = kt % kStages;
-                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->dsready[b]), (kt >> 1) & 1))
+                if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->dsready[b]), (kt >> 1) & 1))
                     misc->abort_flag = 1;
                 if (misc->abort_flag) return;
                 tc_fence_after();
@@ -278,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) 
             };
             for (int kt = 0; kt < nkt; ++kt) {
                 const int b = kt & 1, st = kt % kStages;
-                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->kready[st]), (kt / kStages) & 1))
+                if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->kready[st]), (kt / kStages) & 1))
                     misc->abort_flag = 1;
                 if (misc->abort_flag) break;
                 tc_fence_after();
@@ -356,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) 
 #pragma unroll
                 for (int i = 0; i < 64; ++i) g[i] = trow && s0 + i <= t ? p.Gin[t * p.L + s0 + i] : 0.f;
             }
-            if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (kt >> 1) & 1))
+            if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->sfull[b]), (kt >> 1) & 1))
                 misc->abort_flag = 1;
             if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
                 tc_fence_after();
@@ -401,12 +400,12 @@ __global__ void __launch_bounds__(kThreads, 1) dq_tc_kernel(const kl::Params p) 
             // iteration writes its dS buffer and before tile kt + 2 takes its
             // key stage.
             if (kt >= 1 && kt + 1 < nkt && !misc->abort_flag &&
-                !mbar_wait(smem_u32(&misc->kfree[(kt - 1) % kStages]), ((kt - 1) / kStages) & 1))
+                !mbar_wait_to(p.err, smem_u32(&misc->kfree[(kt - 1) % kStages]), ((kt - 1) / kStages) & 1))
                 misc->abort_flag = 1;
             if (kt + 2 < nkt && !misc->abort_flag) put_k(kt + 2, kv);
         }
         // dq and dw
-        if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
+        if (!mbar_wait_to(p.err, smem_u32(&misc->done), 0)) misc->abort_flag = 1;
         tc_fence_after();
         if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // the TMEM loads are warp-collective
             float a[32], c[32];
@@ -462,7 +461,6 @@ constexpr uint32_t kIdescSt = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(k
 // Grid (nsplit, ceil(L / 128)): the groups of one key tile side by side; the
 // longest key tiles (the first) first.
 __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) {
-    bind_error_word(p.err);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Misc* misc = reinterpret_cast<Misc*>(smem + kDkMisc);
@@ -502,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) 
         if (lane == 0) {
             auto dk_unit = [&](int u) {
                 const int b = u & 1, st = u % kStages;
-                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->dsready[b]), (u >> 1) & 1))
+                if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->dsready[b]), (u >> 1) & 1))
                     misc->abort_flag = 1;
                 if (misc->abort_flag) return;
                 tc_fence_after();
@@ -517,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) 
             };
             for (int u = 0; u < nunits; ++u) {
                 const int b = u & 1, st = u % kStages;
-                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->kready[st]), (u / kStages) & 1))
+                if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->kready[st]), (u / kStages) & 1))
                     misc->abort_flag = 1;
                 if (misc->abort_flag) break;
                 tc_fence_after();
@@ -598,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) 
                 }
                 named_bar_sync(1, kWorkers * 32);
             }
-            if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (u >> 1) & 1))
+            if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->sfull[b]), (u >> 1) & 1))
                 misc->abort_flag = 1;
             if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
                 tc_fence_after();
@@ -639,11 +637,11 @@ __global__ void __launch_bounds__(kThreads, 1) dk_tc_kernel(const kl::Params p) 
                 if (lane == 0) mbar_arrive(smem_u32(&misc->dsready[b]));
             }
             if (u >= 1 && u + 1 < nunits && !misc->abort_flag &&
-                !mbar_wait(smem_u32(&misc->kfree[(u - 1) % kStages]), ((u - 1) / kStages) & 1))
+                !mbar_wait_to(p.err, smem_u32(&misc->kfree[(u - 1) % kStages]), ((u - 1) / kStages) & 1))
                 misc->abort_flag = 1;
             if (u + 2 < nunits && !misc->abort_flag) put_q(u + 2, qv);
         }
-        if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
+        if (!mbar_wait_to(p.err, smem_u32(&misc->done), 0)) misc->abort_flag = 1;
         tc_fence_after();
         if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // the TMEM loads are warp-collective
             float a[32], c[32];
@@ -694,7 +692,6 @@ constexpr int kD = 128;                             // attention head dim of the
 // worker keeps an online max and sum over its half of the keys.  Grid (Hq,
 // ceil(L / 128)): the heads of a query tile side by side, longest first.
 __global__ void __launch_bounds__(kThreads, 1) head_lse_tc_kernel(const kl::Params p) {
-    bind_error_word(p.err);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Misc* misc = reinterpret_cast<Misc*>(smem + kFwdMisc);
@@ -732,10 +729,10 @@ __global__ void __launch_bounds__(kThreads, 1) head_lse_tc_kernel(const kl::Para
         if (lane == 0) {
             for (int kt = 0; kt < nkt; ++kt) {
                 const int b = kt & 1, st = kt % kStages;
-                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->kready[st]), (kt / kStages) & 1))
+                if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->kready[st]), (kt / kStages) & 1))
                     misc->abort_flag = 1;
                 if (!misc->abort_flag && kt >= 2 &&
-                    !mbar_wait(smem_u32(&misc->dsready[b]), ((kt - 2) >> 1) & 1))
+                    !mbar_wait_to(p.err, smem_u32(&misc->dsready[b]), ((kt - 2) >> 1) & 1))
                     misc->abort_flag = 1;
                 if (misc->abort_flag) break;
                 tc_fence_after();
@@ -786,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1) head_lse_tc_kernel(const kl::Para
             const int b = kt & 1;
             BfPieces kv;
             if (kt + 2 < nkt) load_k(kt + 2, kv);
-            if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (kt >> 1) & 1))
+            if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->sfull[b]), (kt >> 1) & 1))
                 misc->abort_flag = 1;
             if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
                 tc_fence_after();
@@ -820,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1) head_lse_tc_kernel(const kl::Para
                 }
             }
             if (kt >= 1 && kt + 1 < nkt && !misc->abort_flag &&
-                !mbar_wait(smem_u32(&misc->kfree[(kt - 1) % kStages]), ((kt - 1) / kStages) & 1))
+                !mbar_wait_to(p.err, smem_u32(&misc->kfree[(kt - 1) % kStages]), ((kt - 1) / kStages) & 1))
                 misc->abort_flag = 1;
             if (kt + 2 < nkt && !misc->abort_flag) put_k(kt + 2, kv);
         }
@@ -838,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1) head_lse_tc_kernel(const kl::Para
             const float l = lrun * kl::ex2(mrun - mu) + lo * kl::ex2(mo - mu);
             if (trow && !misc->abort_flag) p.lse_h[t * p.Hq + hq] = mt + kl::lg2(l);
         }
-        if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
+        if (!mbar_wait_to(p.err, smem_u32(&misc->done), 0)) misc->abort_flag = 1;
     }
     tc_fence_before();
     __syncthreads();
@@ -860,7 +857,6 @@ static_assert(kTgtSmemBytes <= 232448, "shared memory per block");
 // written over I.  Tiles above the diagonal only write G = 0.  Grid (ntq
 // key tiles, ntq query tiles).  Needs Hkv <= 4.
 __global__ void __launch_bounds__(kThreads, 1) target_tc_kernel(const kl::Params p) {
-    bind_error_word(p.err);
     extern __shared__ uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kt = blockIdx.x, qt = blockIdx.y;
@@ -904,10 +900,10 @@ __global__ void __launch_bounds__(kThreads, 1) target_tc_kernel(const kl::Params
         if (lane == 0) {
             for (int u = 0; u < nunits; ++u) {
                 const int b = u & 1, st = u % kStages;
-                if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->kready[st]), (u / kStages) & 1))
+                if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->kready[st]), (u / kStages) & 1))
                     misc->abort_flag = 1;
                 if (!misc->abort_flag && u >= 2 &&
-                    !mbar_wait(smem_u32(&misc->dsready[b]), ((u - 2) >> 1) & 1))
+                    !mbar_wait_to(p.err, smem_u32(&misc->dsready[b]), ((u - 2) >> 1) & 1))
                     misc->abort_flag = 1;
                 if (misc->abort_flag) break;
                 tc_fence_after();
@@ -966,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1) target_tc_kernel(const kl::Params
             if (u + 2 < nunits) load_q(u + 2, qv);
             const float lse = lse_next;
             if (u + 1 < nunits) lse_next = trow ? p.lse_h[t * p.Hq + u + 1] : 0.f;
-            if (!misc->abort_flag && !mbar_wait(smem_u32(&misc->sfull[b]), (u >> 1) & 1))
+            if (!misc->abort_flag && !mbar_wait_to(p.err, smem_u32(&misc->sfull[b]), (u >> 1) & 1))
                 misc->abort_flag = 1;
             if (!__any_sync(0xffffffffu, misc->abort_flag)) {  // warp-uniform: TMEM loads below
                 tc_fence_after();
@@ -985,7 +981,7 @@ __global__ void __launch_bounds__(kThreads, 1) target_tc_kernel(const kl::Params
                 }
             }
             if (u >= 1 && u + 1 < nunits && !misc->abort_flag &&
-                !mbar_wait(smem_u32(&misc->kfree[(u - 1) % kStages]), ((u - 1) / kStages) & 1))
+                !mbar_wait_to(p.err, smem_u32(&misc->kfree[(u - 1) % kStages]), ((u - 1) / kStages) & 1))
                 misc->abort_flag = 1;
             if (u + 2 < nunits && !misc->abort_flag) put_q(u + 2, qv);
         }
@@ -1038,7 +1034,7 @@ __global__ void __launch_bounds__(kThreads, 1) target_tc_kernel(const kl::Params
         if (h == 1) misc->dw[m] = klp;
         named_bar_sync(1, kWorkers * 32);
         if (h == 0 && trow && !misc->abort_flag) p.kl_part[t * p.ntiles + kt] = klp + misc->dw[m];
-        if (!mbar_wait(smem_u32(&misc->done), 0)) misc->abort_flag = 1;
+        if (!mbar_wait_to(p.err, smem_u32(&misc->done), 0)) misc->abort_flag = 1;
     }
     tc_fence_before();
     __syncthreads();

@@ -9,24 +9,16 @@
 namespace dsa {
 
 // Device error words (DSA_DEVERR_* codes; the first error of a call wins).
-// A call records into the word its caller passed; a call given none records
-// into the library's per-device word.
+// Every kernel takes its call's word as a parameter (the caller's, or null
+// for this library's per-device word) and records into it; kernels never
+// trap.
 __device__ int g_dsa_device_error;
-
-// The word of the running kernel's call.  Every thread sets it at kernel
-// entry (all to the same value, so no barrier is needed before a thread
-// reads its own write).
-__shared__ int* s_dsa_error_word;
-
-__device__ __forceinline__ void bind_error_word(int* word) {
-    s_dsa_error_word = word != nullptr ? word : &g_dsa_device_error;
-}
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-__device__ __forceinline__ void record_device_error(int code) {
-    atomicCAS(s_dsa_error_word, 0, code);
+__device__ __forceinline__ void record_error_to(int* word, int code) {
+    atomicCAS(word != nullptr ? word : &g_dsa_device_error, 0, code);
 }
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -77,14 +69,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, records DSA_DEVERR_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// kWaitLimitNs, records DSA_DEVERR_TIMEOUT in the call's error word and
+// returns false.
+__device__ __forceinline__ bool mbar_wait_to(int* word, uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (globaltimer() - t0 > kWaitLimitNs) {
-            record_device_error(1);
+            record_error_to(word, 1);
             return false;
         }
     }

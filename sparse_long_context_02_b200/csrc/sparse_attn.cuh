@@ -101,13 +101,12 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
 template <int D, int HKV, int G, bool SPLIT>
 __global__ void __launch_bounds__(Cfg<D, HKV>::THREADS)
 attn_kernel(const Params p) {
-    bind_error_word(p.err);
     pdl_wait();  // decode: the index rows come from the merge kernel
     pdl_launch_dependents();
     using C = Cfg<D, HKV>;
     constexpr int HQ = HKV * G;
     static_assert(G <= 8, "at most 8 query heads per KV group");
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::STAGE);
     uint64_t* empty = full + kStages;
     uint32_t* mask = reinterpret_cast<uint32_t*>(empty + kStages);
@@ -171,17 +170,17 @@ attn_kernel(const Params p) {
             pre = load_idx(c + 1);
             if (c >= kStages) {
                 bool got = false;
-                if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ((c / kStages) - 1) & 1);
+                if (lane == 0) got = mbar_wait_to(p.err, smem_u32(&empty[s]), ((c / kStages) - 1) & 1);
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
             }
             int32_t si;
             if constexpr (SPLIT) {  // global keys of a cache shard, or sequence-local ones
                 const int64_t sl = sg - koff;
-                if (sg >= 0 && sl >= nkeys && !p.skip_foreign) record_device_error(2);
+                if (sg >= 0 && sl >= nkeys && !p.skip_foreign) record_error_to(p.err, 2);
                 si = sg >= 0 && sl >= 0 && sl < nkeys ? (int32_t)sl : -1;
             } else {
                 si = (int32_t)sg;
-                if (si >= nkeys) record_device_error(2);
+                if (si >= nkeys) record_error_to(p.err, 2);
             }
             const bool valid = si >= 0 && si < nkeys;
             const uint32_t bal = __ballot_sync(0xffffffffu, valid);
@@ -215,7 +214,7 @@ attn_kernel(const Params p) {
         }
         if (lane == 0) {
             for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
-                mbar_wait(smem_u32(&full[c % kStages]), (c / kStages) & 1);
+                mbar_wait_to(p.err, smem_u32(&full[c % kStages]), (c / kStages) & 1);
         }
         return;
     }
@@ -247,7 +246,7 @@ attn_kernel(const Params p) {
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % kStages;
-        bool got = mbar_wait(smem_u32(&full[s]), (c / kStages) & 1);
+        bool got = mbar_wait_to(p.err, smem_u32(&full[s]), (c / kStages) & 1);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         const uint32_t msk = mask[s];
         if (msk) {

@@ -77,11 +77,10 @@ __device__ __forceinline__ uint32_t bf16_bits(const __nv_bfloat16* p) {
 template <int D, int HKV, int G>
 __global__ void __launch_bounds__(Cfg<D, HKV>::THREADS)
 attn_bwd_kernel(const BwdParams p) {
-    bind_error_word(p.err);
     using C = Cfg<D, HKV>;
     constexpr int HQ = HKV * G;
     static_assert(G <= 8, "at most 8 query heads per KV group");
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::STAGE);
     uint64_t* empty = full + kStages;
     uint32_t* mask = reinterpret_cast<uint32_t*>(empty + kStages);
@@ -117,10 +116,10 @@ attn_bwd_kernel(const BwdParams p) {
             pre = load_idx(c + 1);
             if (c >= kStages) {
                 bool got = false;
-                if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ((c / kStages) - 1) & 1);
+                if (lane == 0) got = mbar_wait_to(p.err, smem_u32(&empty[s]), ((c / kStages) - 1) & 1);
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
             }
-            if (si >= nkeys) record_device_error(2);
+            if (si >= nkeys) record_error_to(p.err, 2);
             const bool valid = si >= 0 && si < nkeys;
             const uint32_t bal = __ballot_sync(0xffffffffu, valid);
             const uint32_t sbase = smem_u32(smem + s * C::STAGE);
@@ -151,7 +150,7 @@ attn_bwd_kernel(const BwdParams p) {
         }
         if (lane == 0) {
             for (int c = issued - kStages < 0 ? 0 : issued - kStages; c < issued; ++c)
-                mbar_wait(smem_u32(&full[c % kStages]), (c / kStages) & 1);
+                mbar_wait_to(p.err, smem_u32(&full[c % kStages]), (c / kStages) & 1);
         }
         return;
     }
@@ -219,7 +218,7 @@ attn_bwd_kernel(const BwdParams p) {
         const int e0 = c * kNK + r, e1 = e0 + 8;
         const int32_t key0 = e0 < nent ? irow[e0] : -1;
         const int32_t key1 = e1 < nent ? irow[e1] : -1;
-        bool got = mbar_wait(smem_u32(&full[s]), (c / kStages) & 1);
+        bool got = mbar_wait_to(p.err, smem_u32(&full[s]), (c / kStages) & 1);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         const uint32_t msk = mask[s];
         if (msk) {

@@ -75,12 +75,11 @@ __device__ __forceinline__ bool selected(const uint32_t* mask32, int pos, int nU
 template <int D, int HKV, int G>
 __global__ void __launch_bounds__(DedupCfg<D, HKV>::THREADS, 1)
 dedup_kernel(const Params p) {
-    bind_error_word(p.err);
     using C = DedupCfg<D, HKV>;
     constexpr int HQ = HKV * G;
     constexpr int NT = C::THREADS;
     static_assert(G <= 8, "at most 8 query heads per KV group");
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem);  // phase 1 only
     int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
     int32_t* U = reinterpret_cast<int32_t*>(smem + C::OFF_U);
@@ -109,7 +108,7 @@ dedup_kernel(const Params p) {
     for (int e = tid; e < ne; e += NT) {
         const int32_t u = p.idx[(q0 + e / p.k) * p.k + e % p.k];
         if (u >= 0 && u < L) atomicOr(&bitmap[u >> 5], 1u << (u & 31));
-        else if (u >= L) record_device_error(2);
+        else if (u >= L) record_error_to(p.err, 2);
     }
     __syncthreads();
     // words [w0, w1) of this thread: count, block scan, prefix, list
@@ -161,7 +160,7 @@ dedup_kernel(const Params p) {
             const int s = c % kDedupStages;
             if (c >= kDedupStages) {
                 bool got = false;
-                if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ((c / kDedupStages) - 1) & 1);
+                if (lane == 0) got = mbar_wait_to(p.err, smem_u32(&empty[s]), ((c / kDedupStages) - 1) & 1);
                 if (!__shfl_sync(0xffffffffu, got, 0)) break;
             }
             const uint32_t sbase = smem_u32(smem + s * C::STAGE);
@@ -185,7 +184,7 @@ dedup_kernel(const Params p) {
         }
         if (lane == 0) {
             for (int c = issued - kDedupStages < 0 ? 0 : issued - kDedupStages; c < issued; ++c)
-                mbar_wait(smem_u32(&full[c % kDedupStages]), (c / kDedupStages) & 1);
+                mbar_wait_to(p.err, smem_u32(&full[c % kDedupStages]), (c / kDedupStages) & 1);
         }
         return;
     }
@@ -224,7 +223,7 @@ dedup_kernel(const Params p) {
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % kDedupStages;
-        const bool got = mbar_wait(smem_u32(&full[s]), (c / kDedupStages) & 1);
+        const bool got = mbar_wait_to(p.err, smem_u32(&full[s]), (c / kDedupStages) & 1);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         const uint32_t kbase = smem_u32(smem + s * C::STAGE) + g * D * 2;
         const uint32_t vbase = kbase + kNK * C::STRIDE;
