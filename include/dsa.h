@@ -309,6 +309,31 @@ DSA_API dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, con
                                     dsa_stream_t stream);
 
 /*
+ * dsa_decode_from_host - one decode step whose new inputs and outputs live in
+ * host memory while the caches stay resident on the device (a serving loop:
+ * the caller appends the new token's cache rows, then calls this).  On
+ * `stream`: the B query rows (q_I, w, Q) are copied from the host into the
+ * caller's device buffers, dsa_sparse_attn_decode runs, and O (and, with
+ * idx_host, the index rows) are copied back.  Host buffers must be
+ * page-locked for the copies to be asynchronous; O_host holds the result
+ * once `stream` reaches the end of this call's work.
+ *
+ *   q_I_host, w_host, Q_host, O_host, idx_host (or NULL)   host pointers,
+ *       layouts as q_I, w, Q, O, idx_out of dsa_sparse_attn_decode
+ *   q_I, w, Q                 device buffers the queries are copied into
+ *   everything else           as dsa_sparse_attn_decode (idx_out is
+ *                             required with idx_host)
+ */
+DSA_API dsa_status_t dsa_decode_from_host(const void* q_I_host, const float* w_host,
+                                  const void* Q_host, void* O_host, int32_t* idx_host,
+                                  void* q_I, float* w, void* Q, const void* kI_cache,
+                                  const void* K_cache, const void* V_cache,
+                                  const int64_t* cache_off, int B, int64_t total_n, int H_I,
+                                  int d_I, int Hq, int Hkv, int d, int k, float scale, void* O,
+                                  int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                                  int32_t* err, dsa_stream_t stream);
+
+/*
  * dsa_sparse_attn_decode_noalloc - dsa_sparse_attn_decode for callers that
  * cannot pass a workspace (the pages have no counterpart: this is a
  * deployment convenience).  Callers that run inside a host framework owning

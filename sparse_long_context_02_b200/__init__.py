@@ -69,6 +69,9 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_attn_decode.restype = i32
         L.dsa_sparse_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
                                              i32, i32, i32, f32, vp, vp, vp, sz, vp, vp]
+        L.dsa_decode_from_host.restype = i32
+        L.dsa_decode_from_host.argtypes = [vp] * 11 + [vp, i32, i64, i32, i32, i32, i32, i32, i32,
+                                                       f32, vp, vp, vp, sz, vp, vp]
         L.dsa_sparse_attn_decode_noalloc.restype = i32
         L.dsa_sparse_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
                                                      i32, i32, i32, i32, i32, f32, vp, vp, vp,
@@ -310,6 +313,29 @@ def sparse_attn_decode(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, k: int,
         _dev(workspace, "workspace", 1), workspace.numel(), _err(err), _stream(stream)),
         "dsa_sparse_attn_decode")
     return O, idx_out
+
+
+def decode_from_host(host: dict, dev: dict, cache_off, k: int, scale: float, stream=None,
+                     err=None) -> None:
+    """One decode step with the queries in (pinned) host memory and the caches
+    on the device: host q_I, w, Q (inputs) and O (output, optionally idx);
+    dev q_I, w, Q, kI_cache, K_cache, V_cache, O, workspace (optionally idx).
+    Asynchronous on `stream` (host["O"] is filled when it completes)."""
+    B, H, dI = host["q_I"].shape
+    Hq, d = host["Q"].shape[1], host["Q"].shape[2]
+    total_n, Hkv = dev["kI_cache"].shape[0], dev["K_cache"].shape[1]
+    ih = _host(host["idx"], "idx") if host.get("idx") is not None else None
+    idx = dev.get("idx")
+    ws = dev["workspace"]
+    _check(lib().dsa_decode_from_host(
+        _host(host["q_I"], "q_I"), _host(host["w"], "w"), _host(host["Q"], "Q"),
+        _host(host["O"], "O"), ih, _dev(dev["q_I"], "q_I", 1), _dev(dev["w"], "w", 4),
+        _dev(dev["Q"], "Q", 2), _dev(dev["kI_cache"], "kI_cache", 1),
+        _dev(dev["K_cache"], "K_cache", 2), _dev(dev["V_cache"], "V_cache", 2),
+        _dev(cache_off, "cache_off", 8), B, total_n, H, dI, Hq, Hkv, d, k, float(scale),
+        _dev(dev["O"], "O", 2), _dev(idx, "idx", 4) if idx is not None else None,
+        _dev(ws, "workspace", 1), ws.numel(), _err(err), _stream(stream)),
+        "dsa_decode_from_host")
 
 
 def sparse_attn_decode_noalloc(q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, k: int,

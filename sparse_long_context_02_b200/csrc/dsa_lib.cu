@@ -787,6 +787,43 @@ dsa_status_t dsa_sparse_attn_decode(const void* q_I, const float* w, const void*
                       scale, O, idx_out, workspace, workspace_bytes, err, stream);
 }
 
+dsa_status_t dsa_decode_from_host(const void* q_I_host, const float* w_host, const void* Q_host,
+                                  void* O_host, int32_t* idx_host, void* q_I, float* w, void* Q,
+                                  const void* kI_cache, const void* K_cache, const void* V_cache,
+                                  const int64_t* cache_off, int B, int64_t total_n, int H_I,
+                                  int d_I, int Hq, int Hkv, int d, int k, float scale, void* O,
+                                  int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                                  int32_t* err, dsa_stream_t stream) {
+    static const char fn[] = "dsa_decode_from_host";
+    CHECK_PTR(q_I_host);
+    CHECK_PTR(w_host);
+    CHECK_PTR(Q_host);
+    CHECK_PTR(O_host);
+    if (idx_host != nullptr && idx_out == nullptr)
+        return fail(DSA_ERR_INVALID_ARG, "%s: idx_host needs idx_out", fn);
+    dsa_status_t r = check_decode_args(fn, q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, B,
+                                       total_n, H_I, d_I, Hq, Hkv, d, k, scale, O, idx_out, err);
+    if (r != DSA_OK) return r;
+    CHECK_PTR(workspace);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: workspace is not 256-byte aligned", fn);
+    const size_t need = plan_decode(B, total_n, k, Hq, d, num_sms()).total;
+    if (workspace_bytes < need)  // checked before any copy is queued
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", fn, workspace_bytes, need);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the step's new inputs: one query row per sequence (the caches stay on the device)
+    CUDA_TRY(cudaMemcpyAsync(q_I, q_I_host, (size_t)B * H_I * d_I, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(w, w_host, (size_t)B * H_I * 4, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(Q, Q_host, (size_t)B * Hq * d * 2, cudaMemcpyHostToDevice, st));
+    r = run_decode(fn, q_I, w, Q, kI_cache, K_cache, V_cache, cache_off, B, total_n, k, Hq, d,
+                   scale, O, idx_out, workspace, workspace_bytes, err, stream);
+    if (r != DSA_OK) return r;
+    CUDA_TRY(cudaMemcpyAsync(O_host, O, (size_t)B * Hq * d * 2, cudaMemcpyDeviceToHost, st));
+    if (idx_host != nullptr)
+        CUDA_TRY(cudaMemcpyAsync(idx_host, idx_out, (size_t)B * k * 4, cudaMemcpyDeviceToHost, st));
+    return ok();
+}
+
 // ------------------------------------------------------------ decode over cache shards
 
 dsa_status_t dsa_decode_select_shard(const void* q_I, const float* w, const void* kI_cache,

@@ -85,6 +85,26 @@ def test_prefill_attention_rejects_bad_arguments(L):
     assert f(FAKE, FAKE, FAKE, FAKE, 64, 16, 1, 64, 16, sc, FAKE, None, None, None) == UNSUPPORTED
 
 
+def test_decode_from_host_rejects_bad_arguments(L):
+    f = L.dsa_decode_from_host
+    sc = ctypes.c_float(0.088)
+    args = [FAKE] * 12 + [4, 40000, 64, 128, 32, 4, 128, 2048, sc, FAKE, FAKE, FAKE, 1 << 30,
+                          None, None]
+    bad = list(args)
+    bad[0] = None  # q_I_host
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[22] = None  # idx_out NULL while idx_host is given
+    assert f(*bad) == INVALID
+    assert b"idx_host needs idx_out" in L.dsa_last_error()
+    bad = list(args)
+    bad[16] = 16  # Hq
+    assert f(*bad) == UNSUPPORTED
+    bad = list(args)
+    bad[24] = 100  # workspace too small
+    assert f(*bad) == WORKSPACE
+
+
 def test_attention_backward_rejects_bad_arguments(L):
     f = L.dsa_sparse_attn_backward
     sc = ctypes.c_float(0.125)
@@ -202,6 +222,9 @@ def test_every_launching_call_rejects_a_misaligned_error_word(L):
         "dsa_sparse_attn_decode": [FAKE] * 7 + [4, 40000, 64, 128, 32, 4, 128, 2048,
                                                 ctypes.c_float(0.088), FAKE, None, FAKE, 1 << 30,
                                                 bad_err, None],
+        "dsa_decode_from_host": [FAKE] * 12 + [4, 40000, 64, 128, 32, 4, 128, 2048,
+                                               ctypes.c_float(0.088), FAKE, FAKE, FAKE, 1 << 30,
+                                               bad_err, None],
         "dsa_sparse_attn_decode_noalloc": [FAKE] * 7 + [4, 40000, 64, 128, 32, 4, 128, 2048,
                                                         ctypes.c_float(0.088), FAKE, None,
                                                         bad_err, None],

@@ -231,6 +231,40 @@ def test_decode_small_batch():
     check_attn(O, ref_O)
 
 
+def test_decode_from_host_buffers():
+    """The host-input decode step (queries copied in, outputs copied out, the
+    caches resident) gives the device-input decode's index rows and outputs
+    bit for bit, and the oracle's rows."""
+    lens = [3, 2048, 9000, 40001]
+    cfg, off, qs, kI, K, V = _decode_case(lens, seed=43)
+    B = len(lens)
+    ref_idx, _ = oracle.decode(qs["q_I"], qs["w"], qs["Q"], kI, K, V, off, cfg.k, cfg.scale)
+    caches = dict(kI_cache=dev(kI), K_cache=dev(K, torch.bfloat16), V_cache=dev(V, torch.bfloat16))
+    d_off = dev(off)
+    idx1 = torch.empty((B, cfg.k), dtype=torch.int32, device="cuda")
+    O1, _ = dsa.sparse_attn_decode(dev(qs["q_I"]), dev(qs["w"]), dev(qs["Q"], torch.bfloat16),
+                                   caches["kI_cache"], caches["K_cache"], caches["V_cache"], d_off,
+                                   cfg.k, cfg.scale, idx_out=idx1)
+    pin = lambda a, dt=None: (torch.from_numpy(np.ascontiguousarray(a)).view(dt) if dt else  # noqa: E731
+                              torch.from_numpy(np.ascontiguousarray(a))).pin_memory()
+    host = dict(q_I=pin(qs["q_I"]), w=pin(qs["w"]), Q=pin(qs["Q"].view(np.int16), torch.bfloat16),
+                O=torch.empty((B, cfg.Hq, cfg.d), dtype=torch.bfloat16).pin_memory(),
+                idx=torch.empty((B, cfg.k), dtype=torch.int32).pin_memory())
+    need = dsa.decode_workspace_size(B, int(off[-1]), 64, 128, cfg.k, 32, 4, 128)
+    devb = dict(q_I=torch.empty((B, 64, 128), dtype=torch.uint8, device="cuda"),
+                w=torch.empty((B, 64), dtype=torch.float32, device="cuda"),
+                Q=torch.empty((B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda"),
+                O=torch.empty((B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda"),
+                idx=torch.empty((B, cfg.k), dtype=torch.int32, device="cuda"),
+                workspace=torch.empty(need, dtype=torch.uint8, device="cuda"), **caches)
+    dsa.decode_from_host(host, devb, d_off, cfg.k, cfg.scale)
+    torch.cuda.synchronize()
+    no_device_error()
+    assert torch.equal(host["idx"], idx1.cpu())
+    assert np.array_equal(host["idx"].numpy(), ref_idx)
+    assert torch.equal(host["O"], O1.cpu())
+
+
 def test_decode_equals_prefill_last_row():
     cfg = gen.custom(L=6000, H_I=64, d_I=128, k=2048, Hq=32, Hkv=4, d=128, seed=51)
     inp = gen.prefill_inputs(cfg)
