@@ -347,12 +347,20 @@ def run_ours(args, rank, world, local_rank):
         dsa.index_topk(P["q_I"], P["k_I"], P["w"], pcfg.k, idx=P["idx"], stream=stream)
 
     use_dedup = pcfg is not None and (args.attn == "dedup" or (args.attn == "auto" and pcfg.video))
+    dd_ws = None
+    if use_dedup:
+        dd_ws = torch.empty(dsa.dedup_workspace_size(pcfg.L, pcfg.Hq, pcfg.Hkv, pcfg.d, pcfg.k),
+                            dtype=torch.uint8, device="cuda")
 
     def attn():
         if pcfg is None:
             return
-        f = dsa.sparse_attn_prefill_dedup if use_dedup else dsa.sparse_attn_prefill
-        f(P["Q"], P["K"], P["V"], P["idx"], pcfg.scale, O=P["O"], stream=stream)
+        if use_dedup:
+            dsa.sparse_attn_prefill_dedup(P["Q"], P["K"], P["V"], P["idx"], pcfg.scale, O=P["O"],
+                                          workspace=dd_ws, stream=stream)
+        else:
+            dsa.sparse_attn_prefill(P["Q"], P["K"], P["V"], P["idx"], pcfg.scale, O=P["O"],
+                                    stream=stream)
 
     def decode():
         if dcfg is None:
@@ -361,7 +369,14 @@ def run_ours(args, rank, world, local_rank):
                                D["V_cache"], D["cache_off"], dcfg.k, dcfg.scale, O=D["O"],
                                idx_out=D["idx"], workspace=D["ws"], stream=stream)
 
-    launches_per_step = (2 if pcfg else 0) + (4 if dcfg else 0)  # decode: index, merge, attention, combine
+    # prefill: the indexer, then the attention (the dedup attention: a plan and a
+    # tensor-core kernel per wave of 4096 blocks of 128 / G queries);
+    # decode: index, merge, attention, combine
+    n_attn = 1
+    if use_dedup:
+        qb = 128 // (pcfg.Hq // pcfg.Hkv)
+        n_attn = 2 * (-(-(-(-pcfg.L // qb)) // 4096))
+    launches_per_step = ((1 + n_attn) if pcfg else 0) + (4 if dcfg else 0)
 
     def step(ev=None):
         if ev is not None:
@@ -425,11 +440,17 @@ def run_ours(args, rank, world, local_rank):
         # the gathered rows mostly hit L2 (94 % at L = 65536): its bound is
         # L2 read bandwidth, measured here
         l2pk = l2_read_peak(torch)
-        kernels["dsa_sparse_attn_prefill"] = dict(
-            bound="l2", ms=ms_att, work=prefill_attn_bytes(pcfg),
-            achieved=prefill_attn_bytes(pcfg) / (ms_att / 1e3) / 1e9, peak=l2pk,
+        a_by, a_fl = (dedup_attn_cost(torch, pcfg, P["idx"]) if use_dedup
+                      else (prefill_attn_bytes(pcfg), None))
+        aname = "dsa_sparse_attn_prefill_dedup" if use_dedup else "dsa_sparse_attn_prefill"
+        kernels[aname] = dict(
+            bound="l2", ms=ms_att, work=a_by, achieved=a_by / (ms_att / 1e3) / 1e9, peak=l2pk,
             peak_source="measured here: L2-resident 16-byte reads (libdsa_probe.so)",
             unit="GB/s", hbm_peak=pk["hbm"])
+        if a_fl is not None:
+            kernels[aname]["tensor"] = dict(achieved=a_fl / (ms_att / 1e3) / 1e12,
+                                            peak=pk["bf16_sus"], unit="TFLOP/s",
+                                            frac=a_fl / (ms_att / 1e3) / 1e12 / pk["bf16_sus"])
     if dcfg:
         kernels["dsa_sparse_attn_decode"] = dict(
             bound="hbm", ms=ms_dec, work=decode_bytes(dcfg, lens),
@@ -508,25 +529,39 @@ def run_ours(args, rank, world, local_rank):
                 launches=launches_per_step * K, pcfg=pcfg, dcfg=dcfg, others=others)
 
 
-def dedup_attn_bytes(torch, cfg, idx, G: int) -> float:
-    """Bytes the adjacent-query dedup attention moves: the K and V rows of
-    every distinct key of each block of G consecutive queries, plus Q, O and
-    the index rows (counted on the device from the index rows)."""
+def dedup_stats(torch, idx, qb: int):
+    """(distinct keys, distinct keys rounded up to the 64-key chunk) summed
+    over the blocks of qb consecutive index rows (counted on the device)."""
     L, k = idx.shape
-    nb = (L + G - 1) // G
-    pad = nb * G - L
-    total = 0
+    nb = (L + qb - 1) // qb
+    pad = nb * qb - L
+    distinct = chunked = 0
     for b0 in range(0, nb, 2048):
         b1 = min(nb, b0 + 2048)
-        x = idx[b0 * G:min(L, b1 * G)]
+        x = idx[b0 * qb:min(L, b1 * qb)]
         if b1 == nb and pad:
             x = torch.cat([x, torch.full((pad, k), -1, dtype=x.dtype, device=x.device)])
-        x, _ = torch.sort(x.reshape(b1 - b0, G * k), dim=1)
+        x, _ = torch.sort(x.reshape(b1 - b0, qb * k), dim=1)
         new = torch.ones_like(x, dtype=torch.bool)
         new[:, 1:] = x[:, 1:] != x[:, :-1]
-        total += int(((x >= 0) & new).sum().item())
-    row = 2 * cfg.Hkv * cfg.d * 2
-    return total * row + L * (2 * cfg.Hq * cfg.d * 2 + 4 * k)
+        per = ((x >= 0) & new).sum(dim=1)
+        distinct += int(per.sum().item())
+        chunked += int(((per + 63) // 64 * 64).sum().item())
+    return distinct, chunked
+
+
+def dedup_attn_cost(torch, cfg, idx):
+    """Algorithmic cost of the adjacent-query dedup attention (blocks of
+    128 / G queries): bytes = the K and V rows of every distinct key of a
+    block, once per block, plus Q, O and the index rows; FLOPs = the two
+    products of the 128-row tiles over each block's chunked key list, for
+    every KV group."""
+    qb = 128 // (cfg.Hq // cfg.Hkv)
+    distinct, chunked = dedup_stats(torch, idx, qb)
+    L, k = idx.shape
+    by = distinct * 2 * cfg.Hkv * cfg.d * 2 + L * (2 * cfg.Hq * cfg.d * 2 + 4 * k)
+    fl = 2.0 * 2 * 128 * cfg.d * chunked * cfg.Hkv
+    return by, fl
 
 
 def other_configs(torch, dsa, pk, args, stream, flush):
@@ -545,6 +580,11 @@ def other_configs(torch, dsa, pk, args, stream, flush):
         idx = torch.empty((cfg.L, cfg.k), dtype=torch.int32, device="cuda")
         O = torch.empty_like(bf["Q"])
         attn = dsa.sparse_attn_prefill_dedup if cfg.video else dsa.sparse_attn_prefill
+        kw = {}
+        if cfg.video:
+            kw["workspace"] = torch.empty(dsa.dedup_workspace_size(cfg.L, cfg.Hq, cfg.Hkv, cfg.d,
+                                                                   cfg.k),
+                                          dtype=torch.uint8, device="cuda")
 
         def step(ev=None):
             if ev:
@@ -552,7 +592,7 @@ def other_configs(torch, dsa, pk, args, stream, flush):
             dsa.index_topk(t["q_I"], t["k_I"], t["w"], cfg.k, idx=idx, stream=stream)
             if ev:
                 ev[1].record(stream)
-            attn(bf["Q"], bf["K"], bf["V"], idx, cfg.scale, O=O, stream=stream)
+            attn(bf["Q"], bf["K"], bf["V"], idx, cfg.scale, O=O, stream=stream, **kw)
             if ev:
                 ev[2].record(stream)
 
@@ -570,8 +610,9 @@ def other_configs(torch, dsa, pk, args, stream, flush):
         mi = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
         ma = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
         fl, by = prefill_flops(cfg), prefill_attn_bytes(cfg)
-        if cfg.video:  # the dedup kernel gathers each distinct key of a 6-query block once
-            by = dedup_attn_bytes(torch, cfg, idx, 6)
+        afl = None
+        if cfg.video:  # the dedup kernel gathers each distinct key of a block once
+            by, afl = dedup_attn_cost(torch, cfg, idx)
         out[cfg.name] = dict(
             steps=n, ms_per_step=mi + ma, value=cfg.L / ((mi + ma) / 1e3),
             unit="query-tokens/s",
@@ -581,7 +622,11 @@ def other_configs(torch, dsa, pk, args, stream, flush):
                      attn.__name__: dict(bound="l2", ms=ma, achieved=by / (ma / 1e3) / 1e9,
                                          peak=l2pk, unit="GB/s",
                                          frac=by / (ma / 1e3) / 1e9 / l2pk)})
-        del t, bf, idx, O
+        if afl is not None:  # the dedup kernel's tensor work, against the bf16 peak
+            out[cfg.name]["kernels"][attn.__name__]["tensor"] = dict(
+                achieved=afl / (ma / 1e3) / 1e12, peak=pk["bf16_sus"], unit="TFLOP/s",
+                frac=afl / (ma / 1e3) / 1e12 / pk["bf16_sus"])
+        del t, bf, idx, O, kw
         torch.cuda.empty_cache()
     return out
 

@@ -158,19 +158,34 @@ DSA_API dsa_status_t dsa_sparse_attn_rows(const void* Q, const void* K, const vo
 
 /*
  * dsa_sparse_attn_prefill_dedup - the result of dsa_sparse_attn_prefill,
- * computed for blocks of 6 adjacent query tokens that load the union of
- * their index rows once (adjacent-query dedup, Kwai Keye-VL-2.0 technical
- * report summary, section 8).  Each key a block selects is gathered once;
- * each query keeps only its own keys through a mask in the products.  It
- * pays when adjacent rows overlap strongly (clustered video tokens); its
- * products grow with the union, so on unclustered rows it is slower.
- * Arguments and layouts as dsa_sparse_attn_prefill; an index row must not
- * repeat a key (a repeat counts once here).  Supported: (d, Hkv, Hq/Hkv) in
- * {(128, 4, 8), (64, 2, 4)}, k <= 2048, L <= 262144.
+ * computed for blocks of adjacent query tokens that load the union of their
+ * index rows once (adjacent-query dedup, Kwai Keye-VL-2.0 technical report
+ * summary, section 8, item 2).  A block holds 128 / G tokens (G = Hq / Hkv
+ * query heads per KV group), so that its tokens times the G heads of one
+ * group are the 128 rows of one tensor-core tile; each key the block selects
+ * is gathered once per group, and each token keeps only its own keys through
+ * a mask applied to the score tile.  It pays when adjacent rows overlap
+ * strongly (clustered video tokens); its products grow with the union, so
+ * on unclustered rows it is slower than dsa_sparse_attn_prefill.
+ *   Q [L][Hq][d], K, V [L][Hkv][d] bf16; idx [L][k] int32 (entries < 0 are
+ *   holes; entries >= L are skipped and record DSA_DEVERR_INDEX; a key that
+ *   repeats within one row counts once); O [L][Hq][d] bf16 OUT (a row
+ *   without keys is zeros).
+ *   workspace / workspace_bytes: device memory of at least
+ *   dsa_sparse_attn_prefill_dedup_workspace_size(L, Hq, Hkv, d, k) bytes,
+ *   16-byte aligned, owned by the caller and not read before it is written;
+ *   the blocks run in waves of at most 4096, which bounds its size.
+ * Supported: d in {64, 128}, Hq / Hkv in {4, 8}, L <= 262144, and at most
+ * 32768 distinct keys per block ((128 / G) x k, or L when smaller).
+ * Errors: null or misaligned pointers, bad sizes (DSA_ERR_INVALID_ARG),
+ * other shapes (DSA_ERR_UNSUPPORTED), a short workspace (DSA_ERR_WORKSPACE).
  */
+DSA_API size_t dsa_sparse_attn_prefill_dedup_workspace_size(int64_t L, int Hq, int Hkv, int d,
+                                                            int k);
 DSA_API dsa_status_t dsa_sparse_attn_prefill_dedup(const void* Q, const void* K, const void* V,
                                            const int32_t* idx, int64_t L, int Hq, int Hkv,
-                                           int d, int k, float scale, void* O, int32_t* err,
+                                           int d, int k, float scale, void* O, void* workspace,
+                                           size_t workspace_bytes, int32_t* err,
                                            dsa_stream_t stream);
 
 /*

@@ -52,7 +52,9 @@ def lib() -> ctypes.CDLL:
         L.dsa_index_scores.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp, vp]
         L.dsa_sparse_attn_prefill_dedup.restype = i32
         L.dsa_sparse_attn_prefill_dedup.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32,
-                                                    ctypes.c_float, vp, vp, vp]
+                                                    ctypes.c_float, vp, vp, sz, vp, vp]
+        L.dsa_sparse_attn_prefill_dedup_workspace_size.restype = sz
+        L.dsa_sparse_attn_prefill_dedup_workspace_size.argtypes = [i64, i32, i32, i32, i32]
         L.dsa_prefill_from_host.restype = i32
         L.dsa_prefill_from_host.argtypes = [vp] * 15 + [i64, i32, i32, i32, i32, i32, i32,
                                                           ctypes.c_float, i64, vp, vp, vp, vp]
@@ -270,20 +272,33 @@ def prefill_from_host(host: dict, dev: dict, k: int, scale: float, chunk_rows: i
            "dsa_prefill_from_host")
 
 
+def dedup_workspace_size(L: int, Hq: int, Hkv: int, d: int, k: int) -> int:
+    """Bytes of workspace sparse_attn_prefill_dedup needs (0: shape unsupported)."""
+    return lib().dsa_sparse_attn_prefill_dedup_workspace_size(L, Hq, Hkv, d, k)
+
+
 def sparse_attn_prefill_dedup(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                               idx: torch.Tensor, scale: float, O: Optional[torch.Tensor] = None,
-                              stream=None, err=None) -> torch.Tensor:
-    """sparse_attn_prefill for blocks of 6 adjacent queries that gather the
-    union of their index rows once (pays when adjacent rows overlap)."""
+                              workspace: Optional[torch.Tensor] = None, stream=None,
+                              err=None) -> torch.Tensor:
+    """sparse_attn_prefill for blocks of 128 / (Hq / Hkv) adjacent queries
+    that gather the union of their index rows once (pays when adjacent rows
+    overlap).  `workspace`: a uint8 device tensor of at least
+    dedup_workspace_size(...) bytes, allocated here when None."""
     L, Hq, d = Q.shape
     Hkv = K.shape[1]
     k = idx.shape[1]
     if O is None:
         O = torch.empty_like(Q)
+    need = dedup_workspace_size(L, Hq, Hkv, d, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=Q.device)
     _check(lib().dsa_sparse_attn_prefill_dedup(_dev(Q, "Q", 2), _dev(K, "K", 2), _dev(V, "V", 2),
                                                _dev(idx, "idx", 4), L, Hq, Hkv, d, k,
-                                               float(scale), _dev(O, "O", 2), _err(err),
-                                               _stream(stream)),
+                                               float(scale), _dev(O, "O", 2),
+                                               _dev(workspace, "workspace", 1),
+                                               workspace.numel() * workspace.element_size(),
+                                               _err(err), _stream(stream)),
            "dsa_sparse_attn_prefill_dedup")
     return O
 

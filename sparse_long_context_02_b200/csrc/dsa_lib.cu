@@ -205,17 +205,68 @@ dsa_status_t launch_attn(const char* fn, const dsa::attn::Params& p, int64_t gri
     return DSA_OK;
 }
 
-template <int D, int HKV, int G>
-dsa_status_t launch_dedup(const char* fn, const dsa::attn::Params& p, int64_t L, cudaStream_t st) {
-    using C = dsa::attn::DedupCfg<D, HKV>;
-    auto kern = dsa::attn::dedup_kernel<D, HKV, G>;
-    if (C::SMEM > max_optin_smem())
-        return fail(DSA_ERR_UNSUPPORTED, "%s: needs %d bytes of shared memory", fn, C::SMEM);
-    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
-    const int64_t grid = (L + dsa::attn::kDedupQB - 1) / dsa::attn::kDedupQB;
-    kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(p);
-    CUDA_TRY(cudaGetLastError());
+// Workspace layout of the dedup attention (one wave of blocks).
+template <int G>
+dsa::dedup::Layout dedup_layout(int64_t L, int k) {
+    constexpr int QB = 128 / G;
+    const int64_t nblk = (L + QB - 1) / QB;
+    return dsa::dedup::Layout{nblk < dsa::dedup::kWave ? nblk : dsa::dedup::kWave,
+                              dsa::dedup::block_cap(L, QB, k), QB};
+}
+
+// The dedup attention's wave loop: per wave of blocks, the plan kernel and
+// then the tensor-core kernel (one CTA per KV group and block).
+template <int D, int G>
+dsa_status_t launch_dedup(const char* fn, dsa::dedup::TcParams tp, const int32_t* idx, int k,
+                          void* workspace, cudaStream_t st) {
+    namespace dd = dsa::dedup;
+    using C = dd::TcCfg<D, G>;
+    constexpr int QB = C::QB;
+    const int64_t L = tp.L;
+    const int64_t nblk = (L + QB - 1) / QB;
+    const dd::Layout lay = dedup_layout<G>(L, k);
+    const int plan_smem = dd::plan_smem_bytes(L, lay.cap, QB);
+    if (plan_smem > max_optin_smem() || C::SMEM_LAUNCH > max_optin_smem())
+        return fail(DSA_ERR_UNSUPPORTED, "%s: needs %d bytes of shared memory", fn,
+                    plan_smem > C::SMEM_LAUNCH ? plan_smem : C::SMEM_LAUNCH);
+    auto plan = dd::plan_kernel<QB>;
+    auto tc = dd::tc_kernel<D, G>;
+    CUDA_TRY(cudaFuncSetAttribute(plan, cudaFuncAttributeMaxDynamicSharedMemorySize, plan_smem));
+    CUDA_TRY(cudaFuncSetAttribute(tc, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_LAUNCH));
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    dd::PlanParams pp{};
+    pp.idx = idx;
+    pp.L = L;
+    pp.k = k;
+    pp.cap = lay.cap;
+    pp.nU = reinterpret_cast<int32_t*>(ws + lay.n_off());
+    pp.keys = reinterpret_cast<int32_t*>(ws + lay.keys_off());
+    pp.masks = reinterpret_cast<uint64_t*>(ws + lay.masks_off());
+    pp.err = tp.err;
+    tp.nU = pp.nU;
+    tp.keys = pp.keys;
+    tp.masks = pp.masks;
+    tp.cap = lay.cap;
+    for (int64_t b0 = 0; b0 < nblk; b0 += lay.nslot) {
+        const int64_t nb = nblk - b0 < lay.nslot ? nblk - b0 : lay.nslot;
+        pp.blk0 = b0;
+        tp.blk0 = b0;
+        plan<<<(unsigned)nb, dd::kPlanThreads, plan_smem, st>>>(pp);
+        CUDA_TRY(cudaGetLastError());
+        tc<<<dim3((unsigned)tp.Hkv, (unsigned)nb), C::THREADS, C::SMEM_LAUNCH, st>>>(tp);
+        CUDA_TRY(cudaGetLastError());
+    }
     return DSA_OK;
+}
+
+// Dedup workspace bytes, or 0 for an unsupported shape.
+size_t dedup_workspace_bytes(int64_t L, int Hq, int Hkv, int d, int k) {
+    if (L < 1 || k < 1 || Hkv < 1 || Hq < 1 || Hq % Hkv) return 0;
+    const int G = Hq / Hkv;
+    if (d != 64 && d != 128) return 0;
+    if (G == 8) return (size_t)dedup_layout<8>(L, k).bytes();
+    if (G == 4) return (size_t)dedup_layout<4>(L, k).bytes();
+    return 0;
 }
 
 // Attention for query rows [row0, row1) over keys [0, L) (arguments
@@ -351,9 +402,14 @@ dsa_status_t dsa_sparse_attn_rows(const void* Q, const void* K, const void* V,
     return r == DSA_OK ? ok() : r;
 }
 
+size_t dsa_sparse_attn_prefill_dedup_workspace_size(int64_t L, int Hq, int Hkv, int d, int k) {
+    return dedup_workspace_bytes(L, Hq, Hkv, d, k);
+}
+
 dsa_status_t dsa_sparse_attn_prefill_dedup(const void* Q, const void* K, const void* V,
                                            const int32_t* idx, int64_t L, int Hq, int Hkv, int d,
-                                           int k, float scale, void* O, int32_t* err,
+                                           int k, float scale, void* O, void* workspace,
+                                           size_t workspace_bytes, int32_t* err,
                                            dsa_stream_t stream) {
     static const char fn[] = "dsa_sparse_attn_prefill_dedup";
     CHECK_PTR(Q);
@@ -363,29 +419,38 @@ dsa_status_t dsa_sparse_attn_prefill_dedup(const void* Q, const void* K, const v
     CHECK_PTR(O);
     CHECK_ERR_WORD(err);
     if (L < 1) return fail(DSA_ERR_INVALID_ARG, "%s: L = %lld", fn, (long long)L);
-    if (L > dsa::attn::kDedupMaxKeys)
-        return fail(DSA_ERR_UNSUPPORTED, "%s: L = %lld > %d", fn, (long long)L, dsa::attn::kDedupMaxKeys);
+    if (L > dsa::dedup::kMaxKeys)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: L = %lld > %d", fn, (long long)L, dsa::dedup::kMaxKeys);
     if (k < 1) return fail(DSA_ERR_INVALID_ARG, "%s: k = %d", fn, k);
-    if (k > dsa::attn::kDedupMaxK) return fail(DSA_ERR_UNSUPPORTED, "%s: k = %d > %d", fn, k, dsa::attn::kDedupMaxK);
     if (Hkv < 1 || Hq < 1 || Hq % Hkv) return fail(DSA_ERR_INVALID_ARG, "%s: Hq = %d, Hkv = %d", fn, Hq, Hkv);
     if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale", fn);
     const int G = Hq / Hkv;
-    dsa::attn::Params p{};
-    p.Q = static_cast<const __nv_bfloat16*>(Q);
-    p.K = static_cast<const __nv_bfloat16*>(K);
-    p.V = static_cast<const __nv_bfloat16*>(V);
-    p.idx = idx;
-    p.nkeys = L;
-    p.k = k;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.O = static_cast<__nv_bfloat16*>(O);
-    p.err = err;
+    if ((d != 64 && d != 128) || (G != 4 && G != 8))
+        return fail(DSA_ERR_UNSUPPORTED, "%s: (d, Hq/Hkv) = (%d, %d)", fn, d, G);
+    const int64_t cap = dsa::dedup::block_cap(L, 128 / G, k);
+    if (cap > dsa::dedup::kMaxCap)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: %d x k = %lld distinct keys per block > %d", fn,
+                    128 / G, (long long)cap, dsa::dedup::kMaxCap);
+    CHECK_PTR(workspace);
+    if (workspace_bytes < dedup_workspace_bytes(L, Hq, Hkv, d, k))
+        return fail(DSA_ERR_WORKSPACE, "%s: workspace_bytes = %zu < %zu", fn, workspace_bytes,
+                    dedup_workspace_bytes(L, Hq, Hkv, d, k));
+    dsa::dedup::TcParams tp{};
+    tp.Q = static_cast<const __nv_bfloat16*>(Q);
+    tp.K = static_cast<const __nv_bfloat16*>(K);
+    tp.V = static_cast<const __nv_bfloat16*>(V);
+    tp.O = static_cast<__nv_bfloat16*>(O);
+    tp.L = L;
+    tp.Hq = Hq;
+    tp.Hkv = Hkv;
+    tp.scale_log2 = scale * 1.4426950408889634f;
+    tp.err = err;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     dsa_status_t r;
-    if (d == 128 && Hkv == 4 && G == 8) r = launch_dedup<128, 4, 8>(fn, p, L, st);
-    else if (d == 64 && Hkv == 2 && G == 4) r = launch_dedup<64, 2, 4>(fn, p, L, st);
-    else
-        return fail(DSA_ERR_UNSUPPORTED, "%s: (d, Hkv, Hq/Hkv) = (%d, %d, %d)", fn, d, Hkv, G);
+    if (d == 128 && G == 8) r = launch_dedup<128, 8>(fn, tp, idx, k, workspace, st);
+    else if (d == 64 && G == 4) r = launch_dedup<64, 4>(fn, tp, idx, k, workspace, st);
+    else if (d == 128 && G == 4) r = launch_dedup<128, 4>(fn, tp, idx, k, workspace, st);
+    else r = launch_dedup<64, 8>(fn, tp, idx, k, workspace, st);
     return r == DSA_OK ? ok() : r;
 }
 

@@ -195,6 +195,53 @@ def test_indexer_kl_rejects_bad_arguments_and_small_workspaces(L):
     assert g(*bad, nb, None, None) == INVALID
 
 
+def test_dedup_workspace_size_and_argument_checks(L):
+    """The dedup attention's workspace: per slot (a block of 128 / G queries,
+    at most 4096 slots per wave) one int32 count (the counts 256-byte
+    aligned), `cap` int32 keys and cap / 64 x (128 / G) 64-bit masks, cap =
+    min((128 / G) k, L) rounded up to 64.  Shapes outside the kernel's
+    support get their own status before the workspace is looked at."""
+    size = L.dsa_sparse_attn_prefill_dedup_workspace_size
+
+    def expect(Lq, G, k):
+        qb = 128 // G
+        nslot = min(-(-Lq // qb), 4096)
+        cap = -(-min(qb * k, Lq) // 64) * 64
+        return -(-nslot * 4 // 256) * 256 + nslot * cap * 4 + nslot * (cap // 64) * qb * 8
+
+    assert size(3001, 32, 4, 128, 256) == expect(3001, 8, 256)
+    assert size(262144, 32, 4, 128, 2048) == expect(262144, 8, 2048)
+    assert size(1999, 8, 2, 64, 256) == expect(1999, 4, 256)
+    assert size(1000, 8, 4, 128, 64) == 0        # G = 2: no 128-row tile
+    assert size(1000, 32, 4, 96, 64) == 0        # d = 96
+    f = L.dsa_sparse_attn_prefill_dedup
+    sc = ctypes.c_float(0.088)
+    need = size(3001, 32, 4, 128, 256)
+    args = [FAKE] * 4 + [3001, 32, 4, 128, 256, sc, FAKE, FAKE]
+    assert f(*args, need - 1, None, None) == WORKSPACE
+    bad = list(args)
+    bad[11] = None                               # workspace
+    assert f(*bad, need, None, None) == INVALID
+    bad = list(args)
+    bad[5], bad[6] = 8, 4                        # G = 2
+    assert f(*bad, need, None, None) == UNSUPPORTED
+    bad = list(args)
+    bad[7] = 96                                  # d
+    assert f(*bad, need, None, None) == UNSUPPORTED
+    bad = list(args)
+    bad[4] = 262145                              # beyond the bitmap
+    assert f(*bad, need, None, None) == UNSUPPORTED
+    bad = list(args)
+    bad[4], bad[5], bad[6], bad[8] = 131072, 16, 4, 2048   # G = 4: 32 x 2048 keys per block
+    assert f(*bad, 1 << 40, None, None) == UNSUPPORTED
+    bad = list(args)
+    bad[9] = ctypes.c_float(0.0)                 # scale
+    assert f(*bad, need, None, None) == INVALID
+    bad = list(args)
+    bad[3] = None                                # idx
+    assert f(*bad, need, None, None) == INVALID
+
+
 def test_check_device_error_rejects_bad_arguments(L):
     code = ctypes.c_int(0)
     assert L.dsa_check_device_error(None, None, None) == INVALID
@@ -215,8 +262,8 @@ def test_every_launching_call_rejects_a_misaligned_error_word(L):
         "dsa_sparse_attn_prefill": [FAKE] * 4 + [64, 8, 2, 64, 16, sc, FAKE, None, bad_err, None],
         "dsa_sparse_attn_backward": [FAKE] * 7 + [64, 8, 2, 64, 16, sc, FAKE, FAKE, FAKE, bad_err,
                                                   None],
-        "dsa_sparse_attn_prefill_dedup": [FAKE] * 4 + [64, 8, 2, 64, 16, sc, FAKE, bad_err,
-                                                       None],
+        "dsa_sparse_attn_prefill_dedup": [FAKE] * 4 + [64, 8, 2, 64, 16, sc, FAKE, FAKE,
+                                                       1 << 30, bad_err, None],
         "dsa_prefill_from_host": [FAKE] * 15 + [64, 4, 64, 8, 2, 64, 16, sc, 128, bad_err, None,
                                                  None, None],
         "dsa_sparse_attn_decode": [FAKE] * 7 + [4, 40000, 64, 128, 32, 4, 128, 2048,

@@ -1,7 +1,14 @@
 """Adjacent-query dedup attention (dsa_sparse_attn_prefill_dedup) against the
 fp64 oracle: same bars as the per-query kernel (max-abs 2e-2, mean-abs
 2e-3), on index rows from the GPU indexer (bit-exact with the oracle's),
-with -1 holes, a ragged last block of queries and an out-of-range entry."""
+with -1 holes, a ragged last block of queries, an out-of-range entry, a
+repeated key, clustered (video) rows whose blocks share most keys, scores
+that grow along the key order (the running maximum moves many times, so the
+accumulator is rescaled in TMEM), and both block shapes (16 queries x 8
+heads, 32 queries x 4 heads).
+
+Kwai Keye-VL-2.0 technical-report summary, section 8, item 2 (the dedup) and
+section 1 (the attention it reproduces)."""
 import numpy as np
 import pytest
 import torch
@@ -73,3 +80,70 @@ def test_dedup_attention_holes_empty_rows_and_bad_index():
     check(O[torch.from_numpy(rows).cuda()], ref)
     assert float(O[5].float().abs().max()) == 0.0
     assert dsa.device_error() == dsa.DEVERR_NONE
+
+
+def test_dedup_attention_on_clustered_video_rows():
+    cfg = gen.custom(L=9000, H_I=64, d_I=128, k=2048, Hq=32, Hkv=4, d=128, video=True, seed=24)
+    inp = gen.prefill_inputs(cfg)
+    idx = dsa.index_topk(dev(inp["q_I"]), dev(inp["k_I"]), dev(inp["w"]), cfg.k)
+    Q, K, V = (dev(inp[n], torch.bfloat16) for n in ("Q", "K", "V"))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O = dsa.sparse_attn_prefill_dedup(Q, K, V, idx, cfg.scale, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == dsa.DEVERR_NONE
+    rows = np.unique(np.concatenate([np.arange(0, 20), np.arange(cfg.L - 20, cfg.L),
+                                     np.linspace(20, cfg.L - 21, 60).astype(np.int64)]))
+    ref = oracle.sparse_attn(inp["Q"], inp["K"], inp["V"], idx.cpu().numpy(), cfg.scale, rows=rows)
+    check(O[torch.from_numpy(rows).cuda()], ref)
+    O1 = dsa.sparse_attn_prefill(Q, K, V, idx, cfg.scale)
+    diff = (O.float() - O1.float()).abs()
+    assert diff.max().item() <= 2 * MAX_ABS and diff.mean().item() <= MEAN_ABS
+
+
+@pytest.mark.parametrize("Hq,Hkv,d", [(32, 4, 128), (8, 2, 64), (16, 4, 128), (16, 2, 64)])
+def test_dedup_attention_with_a_moving_maximum(Hq, Hkv, d):
+    """Key u's K row grows with u and every query has a positive bias along
+    it, so the scores of later (larger) keys are larger by up to ~40 in
+    log2 units: the running maximum moves past the rescale threshold many
+    times while a block walks its keys in ascending order."""
+    L, k = 2300, 512
+    rng = np.random.default_rng(31)
+    Qf = rng.standard_normal((L, Hq, d)) * 0.5 + 1.0
+    grow = 3.0 * np.arange(L, dtype=np.float64)[:, None, None] / L
+    Kf = (rng.standard_normal((L, Hkv, d)) * 0.5 + 1.0) * grow
+    Vf = rng.standard_normal((L, Hkv, d))
+    Qh, Kh, Vh = gen.encode_bf16(Qf), gen.encode_bf16(Kf), gen.encode_bf16(Vf)
+    idx = np.full((L, k), -1, dtype=np.int32)
+    for t in range(L):
+        n = min(k, t + 1)
+        idx[t, :n] = rng.permutation(rng.choice(t + 1, size=n, replace=False)).astype(np.int32)
+    scale = 1.0 / np.sqrt(d)
+    Q, K, V = (dev(a, torch.bfloat16) for a in (Qh, Kh, Vh))
+    O = dsa.sparse_attn_prefill_dedup(Q, K, V, dev(idx), scale)
+    assert dsa.device_error() == dsa.DEVERR_NONE
+    rows = np.unique(np.concatenate([np.arange(0, 40), np.arange(L - 40, L),
+                                     np.linspace(40, L - 41, 60).astype(np.int64)]))
+    ref = oracle.sparse_attn(Qh, Kh, Vh, idx, scale, rows=rows)
+    check(O[torch.from_numpy(rows).cuda()], ref)
+
+
+def test_dedup_attention_counts_a_repeated_key_once():
+    cfg = gen.custom(L=600, H_I=4, d_I=64, k=64, Hq=32, Hkv=4, d=128, seed=25)
+    inp = gen.prefill_inputs(cfg)
+    rng = np.random.default_rng(6)
+    idx = np.full((cfg.L, cfg.k), -1, dtype=np.int32)
+    for t in range(cfg.L):
+        n = min(cfg.k, t + 1)
+        idx[t, :n] = rng.choice(t + 1, size=n, replace=False).astype(np.int32)
+    idx_rep = idx.copy()
+    idx_rep[500, 10] = idx_rep[500, 3]       # key repeated in one row
+    idx_rep[501, :] = idx_rep[501, 0]        # one key, k times
+    Q, K, V = (dev(inp[n], torch.bfloat16) for n in ("Q", "K", "V"))
+    O = dsa.sparse_attn_prefill_dedup(Q, K, V, dev(idx_rep), cfg.scale)
+    assert dsa.device_error() == dsa.DEVERR_NONE
+    once = idx_rep.copy()
+    once[500, 10] = -1
+    once[501, 1:] = -1
+    rows = np.array([0, 1, 499, 500, 501, 502, 599])
+    ref = oracle.sparse_attn(inp["Q"], inp["K"], inp["V"], once, cfg.scale, rows=rows)
+    check(O[torch.from_numpy(rows).cuda()], ref)
