@@ -135,6 +135,17 @@ def test_prefill_full_size(cfg):
     err = np.abs(got_O - ref_O)
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
     assert torch.isfinite(O.float()).all()
+    if cfg.video:
+        # the adjacent-query dedup attention (the video workload's kernel) on
+        # the same rows, and close to the per-query kernel everywhere
+        O_dd = dsa.sparse_attn_prefill_dedup(dev(host["Q"], torch.bfloat16),
+                                             dev(host["K"], torch.bfloat16),
+                                             dev(host["V"], torch.bfloat16), idx, cfg.scale)
+        assert dsa.device_error() == dsa.DEVERR_NONE
+        err = np.abs(O_dd[torch.from_numpy(rows).cuda()].float().cpu().numpy() - ref_O)
+        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+        diff = (O_dd.float() - O.float()).abs()
+        assert diff.max().item() <= 2 * MAX_ABS and diff.mean().item() <= MEAN_ABS
 
 
 def test_decode_full_size():
