@@ -54,7 +54,14 @@ __host__ __device__ constexpr int slot_capacity(int k) { return (k + k / 2 + 127
 constexpr int kEpiWarps = 16;     // warps 0-15: four warpgroups, one per chunk quarter
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
-constexpr int kThreads = 18 * 32;
+constexpr int kThreads = 20 * 32;  // warps 18-19 idle: warpgroup 4 is whole for setmaxnreg
+// Register split (setmaxnreg): the launch gives every thread 96 registers (20
+// warps: five per scheduler, whose register file holds 5 x 32 x 96 of its
+// 16 K), warpgroup 4 (producer, MMA issuer, two idle warps) drops to 56 and
+// the four epilogue warpgroups rise to 104, without spills.
+constexpr int kEpiRegs = 104;
+constexpr int kCtlRegs = 56;
+static_assert(4 * 128 * kEpiRegs + 128 * kCtlRegs <= kThreads * 96, "register split");
 
 struct Params {
     const float* w;            // [B][HI]
@@ -207,6 +214,7 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem_base = misc->tmem_base;
     const int b_first = first_seq(p, r0);
+    if (warp >= kEpiWarps) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer
@@ -295,8 +303,9 @@ index_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__
             umma_commit(smem_u32(&misc->mma_done));
             mbar_wait_to(p.err, smem_u32(&misc->mma_done), 0);
         }
-    } else {
+    } else if (warp < kEpiWarps) {
         // ------------------------------------------------ epilogue (warps 0-15)
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
         const int w = warp >> 2;               // quarter of each segment
         const int q = warp & 3;                // TMEM lane quarter
         const int tid = threadIdx.x - w * 128;

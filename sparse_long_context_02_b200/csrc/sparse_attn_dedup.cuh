@@ -147,12 +147,12 @@ template <int QB>
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
     constexpr int NT = kPlanThreads;
     constexpr int NW = NT / 32;
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(16) uint8_t plan_smem[];
     const int nwords = (int)((p.L + 31) >> 5);
     const int64_t nmask = (p.cap / kChunk) * QB;
-    uint32_t* mk = reinterpret_cast<uint32_t*>(smem);  // [chunk][query] as two 32-bit halves
-    uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + nmask * 8);
-    uint16_t* prefix = reinterpret_cast<uint16_t*>(smem + nmask * 8 + (int64_t)nwords * 4);
+    uint32_t* mk = reinterpret_cast<uint32_t*>(plan_smem);  // [chunk][query] as 32-bit halves
+    uint32_t* bitmap = reinterpret_cast<uint32_t*>(plan_smem + nmask * 8);
+    uint16_t* prefix = reinterpret_cast<uint16_t*>(plan_smem + nmask * 8 + (int64_t)nwords * 4);
     __shared__ int s_warp[NW];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
