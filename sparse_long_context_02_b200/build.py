@@ -9,7 +9,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB_PATH = os.path.join(HERE, "libdsa_b200.so")
 SOURCES = [os.path.join(CSRC, "dsa_lib.cu")]
-# the benchmark's L2 bandwidth probe: a separate library, not part of the ABI
+# the benchmark's L2 bandwidth and FP8 tensor-rate probes: a separate library,
+# not part of the ABI
 PROBE_SOURCE = os.path.join(CSRC, "probe_l2.cu")
 PROBE_PATH = os.path.join(HERE, "libdsa_probe.so")
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
@@ -29,8 +30,9 @@ def nvcc() -> str:
 
 
 def build_probe(force: bool = False) -> str:
+    deps = (PROBE_SOURCE, os.path.join(CSRC, "ptx.cuh"))
     if (not force and os.path.exists(PROBE_PATH)
-            and os.path.getmtime(PROBE_PATH) >= os.path.getmtime(PROBE_SOURCE)):
+            and os.path.getmtime(PROBE_PATH) >= max(os.path.getmtime(d) for d in deps)):
         return PROBE_PATH
     tmp = PROBE_PATH + f".tmp{os.getpid()}"
     subprocess.check_call([nvcc(), *NVCC_FLAGS, "-o", tmp, PROBE_SOURCE])
