@@ -761,6 +761,13 @@ dsa_status_t launch_decode_select(const char* fn, const DecodePlan& pl, uint8_t*
     if (smem_idx > max_optin_smem())
         return fail(DSA_ERR_UNSUPPORTED, "%s: needs %d bytes of shared memory", fn, smem_idx);
 
+    // The scan re-splits its registers between warpgroups (setmaxnreg); the
+    // split adds up only if every thread starts with exactly 96.
+    cudaFuncAttributes fa;
+    CUDA_TRY(cudaFuncGetAttributes(&fa, dsa::dec::index_kernel));
+    if (fa.numRegs != 96)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: scan kernel built with %d registers per thread, not 96",
+                    fn, fa.numRegs);
     CUDA_TRY(cudaFuncSetAttribute(dsa::dec::index_kernel,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem_idx));
     CUDA_TRY(launch_chained(dsa::dec::index_kernel, dim3(pl.ctas), dim3(dsa::dec::kThreads),

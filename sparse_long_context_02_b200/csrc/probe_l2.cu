@@ -12,6 +12,11 @@
 // swizzle), with operands resident in shared memory and nothing else to do:
 // one CTA per SM, one thread issuing `iters` x 4 instructions (K = 128) into
 // two TMEM accumulators.  FLOP = 2 * 128 * 256 * 128 * iters per CTA.
+//
+// dsa_probe_wait_timeout: a test hook for the bounded waits every kernel
+// uses (ptx.cuh): one thread waits on an mbarrier that nothing arrives at;
+// after the limit (2 s) the wait gives up, records DSA_DEVERR_TIMEOUT in the
+// given error word and the kernel returns, leaving the context usable.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -102,7 +107,23 @@ __global__ void __launch_bounds__(128, 1) fp8_mma_kernel(int iters, uint32_t* si
     }
 }
 
+__global__ void wait_timeout_kernel(int* err) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        dsa::mbar_init(dsa::smem_u32(&bar), 1);
+        dsa::fence_mbar_init();
+        dsa::mbar_wait_to(err, dsa::smem_u32(&bar), 0);  // no arrival ever comes
+    }
+}
+
 }  // namespace
+
+extern "C" __attribute__((visibility("default"))) int dsa_probe_wait_timeout(void* err,
+                                                                             void* stream) {
+    if (err == nullptr || (reinterpret_cast<uintptr_t>(err) & 3u) != 0) return 1;
+    wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<int*>(err));
+    return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
 
 extern "C" __attribute__((visibility("default"))) int dsa_probe_l2_read(const void* buf,
                                                                         size_t bytes, int passes,
