@@ -147,3 +147,53 @@ def test_dedup_attention_counts_a_repeated_key_once():
     rows = np.array([0, 1, 499, 500, 501, 502, 599])
     ref = oracle.sparse_attn(inp["Q"], inp["K"], inp["V"], once, cfg.scale, rows=rows)
     check(O[torch.from_numpy(rows).cuda()], ref)
+
+
+def _random_rows(L, k, rng, hole_frac=0.0):
+    idx = np.full((L, k), -1, dtype=np.int32)
+    for t in range(L):
+        n = min(k, t + 1)
+        sel = rng.choice(t + 1, size=n, replace=False).astype(np.int32)
+        if hole_frac:
+            sel[rng.random(n) < hole_frac] = -1
+        idx[t, :n] = sel
+    return idx
+
+
+def test_dedup_attention_across_two_waves():
+    """4096 blocks of 16 rows form one wave: L = 66 536 needs two, so rows on
+    both sides of the wave boundary (65 535 / 65 536) and the ragged last
+    block are compared with the oracle."""
+    L, k = 4096 * 16 + 1000, 16
+    rng = np.random.default_rng(41)
+    cfg = gen.custom(L=L, H_I=4, d_I=64, k=k, Hq=32, Hkv=4, d=128, seed=42)
+    Qh, Kh, Vh = gen.prefill_Q(cfg), gen.prefill_K(cfg), gen.prefill_V(cfg)
+    idx = _random_rows(L, k, rng)
+    Q, K, V = (dev(a, torch.bfloat16) for a in (Qh, Kh, Vh))
+    O = dsa.sparse_attn_prefill_dedup(Q, K, V, dev(idx), cfg.scale)
+    assert dsa.device_error() == dsa.DEVERR_NONE
+    rows = np.unique(np.concatenate([np.arange(0, 20), np.arange(65520, 65552),
+                                     np.arange(L - 20, L),
+                                     np.linspace(20, L - 21, 60).astype(np.int64)]))
+    ref = oracle.sparse_attn(Qh, Kh, Vh, idx, cfg.scale, rows=rows)
+    check(O[torch.from_numpy(rows).cuda()], ref)
+
+
+@pytest.mark.parametrize("L,k", [(1, 1), (17, 4), (40, 64)])
+def test_dedup_attention_degenerate_shapes(L, k):
+    """One row; one full block plus one row; k above L; and a block whose
+    rows select nothing (rows 16..31 all holes: zeros)."""
+    rng = np.random.default_rng(43 + L)
+    cfg = gen.custom(L=L, H_I=4, d_I=64, k=k, Hq=32, Hkv=4, d=128, seed=44)
+    Qh, Kh, Vh = gen.prefill_Q(cfg), gen.prefill_K(cfg), gen.prefill_V(cfg)
+    idx = _random_rows(L, k, rng)
+    if L >= 32:
+        idx[16:32] = -1
+    Q, K, V = (dev(a, torch.bfloat16) for a in (Qh, Kh, Vh))
+    O = dsa.sparse_attn_prefill_dedup(Q, K, V, dev(idx), cfg.scale)
+    assert dsa.device_error() == dsa.DEVERR_NONE
+    rows = np.arange(L)
+    ref = oracle.sparse_attn(Qh, Kh, Vh, idx, cfg.scale, rows=rows)
+    check(O, ref)
+    if L >= 32:
+        assert float(O[16:32].float().abs().max()) == 0.0
