@@ -20,23 +20,28 @@
 // the query selected.  Entries < 0 are holes; entries >= L are skipped and
 // flagged (DSA_DEVERR_INDEX); a key repeated in one row counts once.
 //
-// tc_kernel, one CTA per (KV group g, block), 7 warps:
-//   warp 4 (K) and warp 5 (V) gather the chunk's K and V rows of group g
-//     with 16-byte cp.async into 128-byte-swizzled tiles, two stages each
-//     (warp 4 also loads the block's query rows with chunk 0);
+// tc_kernel, one CTA per (KV group g, block), 7 warps, two CTAs per SM:
+//   warp 4 gathers the chunk's K rows of group g (three stages; the block's
+//     query rows with chunk 0) and warp 5 its V rows (two stages), with
+//     16-byte cp.async into 128-byte-swizzled tiles; each loads the next
+//     chunk's key list while the current chunk's copies are issued;
 //   warp 6 allocates TMEM and one thread issues, per chunk c,
 //     S_c  = Q K_c^T   (kind::f16 bf16, M = 128, N = 64, K = d; K-major A
-//                       and B) into one of two TMEM score buffers, and
-//     O   += P_c V_c   (M = 128, N = d, K = 64; V is the MN-major B operand,
-//                       its rows as gathered) into the TMEM accumulator;
+//                       and B, both in shared memory) into one of two TMEM
+//                       score buffers, and
+//     O   += P_c V_c   (M = 128, N = d, K = 64; A = P_c read from TMEM, V the
+//                       MN-major B operand, its rows as gathered) into the
+//                       TMEM accumulator; S of chunk c + 2 reuses the buffer
+//                       of P_c, after P_c V_c in issue order;
 //   warps 0-3 (thread = row m, the TMEM lane) read S_c, put -inf on the keys
 //     their query did not select (the mask), and keep an online softmax in
 //     the exp2 domain.  The offset m_run is raised only when a chunk's
-//     maximum exceeds it by more than kRescaleLog2 (then the O row is read
-//     out of TMEM, scaled and written back), so probabilities stay below
-//     2^kRescaleLog2 and the accumulator is rarely touched.  P_c goes to a
-//     shared K-major tile in bf16.  At the end each thread divides its O row
-//     by the row's sum and stores it in bf16 (zeros for a row without keys).
+//     maximum exceeds it by more than kRescaleLog2 (then, once the previous
+//     product is done, the O row is read out of TMEM, scaled and written
+//     back), so probabilities stay below 2^kRescaleLog2 and the accumulator
+//     is rarely touched.  P_c goes to TMEM in bf16 over the first half of its
+//     score buffer.  At the end each thread divides its O row by the row's
+//     sum and stores it in bf16 (zeros for a row without keys).
 // Every wait is bounded (2 s); a wait that gives up records
 // DSA_DEVERR_TIMEOUT, the CTA stops issuing, waits (bounded) for its own
 // MMAs, frees TMEM and returns.
