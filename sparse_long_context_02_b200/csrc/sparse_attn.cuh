@@ -34,12 +34,14 @@ constexpr int kNK = 16;      // keys per stage
 // on an SM (136 registers x 160 threads x 3 also fits the register file).
 constexpr int kStages = 2;
 
-template <int D, int HKV>
+// NP producer warps split each stage's rows (two pay while the gathered rows
+// hit L2; one otherwise, see dsa_lib.cu).
+template <int D, int HKV, int NP = 1>
 struct Cfg {
     static constexpr int ROW = HKV * D * 2;       // bytes of one token's K (or V) row
     static constexpr int STRIDE = ROW + 16;       // padded shared-memory row
     static constexpr int STAGE = 2 * kNK * STRIDE;
-    static constexpr int THREADS = (HKV + 1) * 32;
+    static constexpr int THREADS = (HKV + NP) * 32;
     static constexpr int SMEM = kStages * STAGE + 128;
 };
 
@@ -98,12 +100,12 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
                  : "r"(addr));
 }
 
-template <int D, int HKV, int G, bool SPLIT>
-__global__ void __launch_bounds__(Cfg<D, HKV>::THREADS)
+template <int D, int HKV, int G, bool SPLIT, int NP = 1>
+__global__ void __launch_bounds__(Cfg<D, HKV, NP>::THREADS)
 attn_kernel(const Params p) {
     pdl_wait();  // decode: the index rows come from the merge kernel
     pdl_launch_dependents();
-    using C = Cfg<D, HKV>;
+    using C = Cfg<D, HKV, NP>;
     constexpr int HQ = HKV * G;
     static_assert(G <= 8, "at most 8 query heads per KV group");
     extern __shared__ __align__(128) uint8_t smem[];
@@ -146,15 +148,16 @@ attn_kernel(const Params p) {
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(smem_u32(&full[s]), 33);  // 32 copy-completion arrivals + lane 0
+            mbar_init(smem_u32(&full[s]), 32 * NP + 1);  // copy completions + one lane 0
             mbar_init(smem_u32(&empty[s]), HKV);
         }
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp == HKV) {
-        // ------------------------------------------------ gather producer (16-byte cp.async)
+    if (warp >= HKV) {
+        // ------------------------------------------------ gather producers (16-byte cp.async)
+        const int pw = warp - HKV;  // rows pw, pw + NP, ... of each stage
         constexpr int CPR = C::ROW / 16;  // 16-byte chunks per row
         int issued = 0;
         // Each chunk's index entries are loaded one chunk ahead, so their
@@ -187,7 +190,7 @@ attn_kernel(const Params p) {
             const uint32_t sbase = smem_u32(smem + s * C::STAGE);
             if (bal) {
 #pragma unroll 4
-                for (int r = 0; r < kNK; ++r) {
+                for (int r = pw; r < kNK; r += NP) {
                     // A masked entry still gets a real row (row 0): its P is 0,
                     // and 0 times stale shared memory could be NaN.  (The
                     // shuffle stays outside any branch: a conditional one
@@ -206,7 +209,7 @@ attn_kernel(const Params p) {
             }
             const uint32_t fb = smem_u32(&full[s]);
             cp_async_arrive(fb);  // this lane's copies of the stage
-            if (lane == 0) {
+            if (lane == 0 && pw == 0) {
                 mask[s] = bal;
                 mbar_arrive(fb);
             }

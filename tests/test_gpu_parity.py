@@ -149,6 +149,27 @@ def test_attention_shapes_with_padding_and_holes(d, Hkv, G):
     check_attn(O, ref)
 
 
+@pytest.mark.parametrize("d,Hkv,G,L", [(128, 4, 8, 50000), (64, 4, 8, 98400)])
+def test_attention_with_keys_beyond_l2(d, Hkv, G, L):
+    """K and V above 96 MB: the kernel runs with one producer warp per CTA
+    (the smaller cases above run with two); sampled rows against the oracle."""
+    k = 64
+    cfg = gen.custom(L=L, Hq=Hkv * G, Hkv=Hkv, d=d, seed=31 + d)
+    Q, K, V = gen.prefill_Q(cfg), gen.prefill_K(cfg), gen.prefill_V(cfg)
+    rng = np.random.default_rng(6)
+    idx = np.full((L, k), -1, np.int32)
+    for t in range(L):
+        m = min(k, t + 1)
+        idx[t, :m] = rng.choice(t + 1, m, replace=False).astype(np.int32)
+    rows = np.unique(np.concatenate([np.arange(0, 70), np.arange(L - 10, L),
+                                     np.linspace(70, L - 11, 50).astype(np.int64)]))
+    ref = oracle.sparse_attn(Q, K, V, idx, cfg.scale, rows=rows)
+    O = dsa.sparse_attn_prefill(dev(Q, torch.bfloat16), dev(K, torch.bfloat16),
+                                dev(V, torch.bfloat16), dev(idx), cfg.scale)
+    no_device_error()
+    check_attn(O[torch.from_numpy(rows).cuda()], ref)
+
+
 def test_attention_empty_rows_are_zero_and_out_of_range_is_flagged():
     cfg = gen.custom(L=64, Hq=32, Hkv=4, d=128, seed=31)
     Q, K, V = gen.prefill_Q(cfg), gen.prefill_K(cfg), gen.prefill_V(cfg)
