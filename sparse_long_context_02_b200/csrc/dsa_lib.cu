@@ -231,6 +231,13 @@ dsa_status_t launch_dedup(const char* fn, dsa::dedup::TcParams tp, const int32_t
                     plan_smem > C::SMEM_LAUNCH ? plan_smem : C::SMEM_LAUNCH);
     auto plan = dd::plan_kernel<QB>;
     auto tc = dd::tc_kernel<D, G>;
+    // the tensor-core kernel re-splits its registers (setmaxnreg); the split
+    // adds up only with exactly C::LAUNCH_REGS per thread at launch
+    cudaFuncAttributes fa;
+    CUDA_TRY(cudaFuncGetAttributes(&fa, tc));
+    if (fa.numRegs != C::LAUNCH_REGS)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: kernel built with %d registers per thread, not %d", fn,
+                    fa.numRegs, C::LAUNCH_REGS);
     CUDA_TRY(cudaFuncSetAttribute(plan, cudaFuncAttributeMaxDynamicSharedMemorySize, plan_smem));
     CUDA_TRY(cudaFuncSetAttribute(tc, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_LAUNCH));
     uint8_t* ws = static_cast<uint8_t*>(workspace);

@@ -20,12 +20,14 @@
 // the query selected.  Entries < 0 are holes; entries >= L are skipped and
 // flagged (DSA_DEVERR_INDEX); a key repeated in one row counts once.
 //
-// tc_kernel, one CTA per (KV group g, block), 7 warps, two CTAs per SM:
-//   warp 4 gathers the chunk's K rows of group g (three stages; the block's
-//     query rows with chunk 0) and warp 5 its V rows (two stages), with
-//     16-byte cp.async into 128-byte-swizzled tiles; each loads the next
-//     chunk's key list while the current chunk's copies are issued;
-//   warp 6 allocates TMEM and one thread issues, per chunk c,
+// tc_kernel, one CTA per (KV group g, block), 12 warps, two CTAs per SM:
+//   warps 4-5 gather the chunk's K rows of group g (three stages; the
+//     block's query rows with chunk 0) and warps 6-7 its V rows (two
+//     stages), with 16-byte cp.async into 128-byte-swizzled tiles; each
+//     loads the next chunk's key list while the current chunk's copies are
+//     issued (the rate of the gather follows the number of warps issuing
+//     copies; the register split keeps the softmax at 128 registers);
+//   warp 8 allocates TMEM and one thread issues, per chunk c,
 //     S_c  = Q K_c^T   (kind::f16 bf16, M = 128, N = 64, K = d; K-major A
 //                       and B, both in shared memory) into one of two TMEM
 //                       score buffers, and
@@ -260,11 +262,16 @@ struct TcCfg {
     static constexpr int SMEM = OFF_BAR + 256;
     // two CTAs per SM at most: each allocates half of TMEM
     static constexpr int SMEM_LAUNCH = SMEM > 100 * 1024 ? SMEM : 100 * 1024;
-    static constexpr int THREADS = 7 * 32;
+    // warps 0-3 softmax, 4-5 K and 6-7 V gather, 8 MMA issuer, 9-11 idle (whole
+    // warpgroups for setmaxnreg): 80 registers at launch, 128 for the
+    // softmax warpgroup, 56 for the other two (128 x 128 + 256 x 56 = 384 x 80)
+    static constexpr int THREADS = 12 * 32;
+    static constexpr int LAUNCH_REGS = 80, SOFTMAX_REGS = 128, OTHER_REGS = 56;
     static constexpr int TMEM_COLS = 256;          // O at 0; S (then P) buffers at 128, 192
     static_assert(G * QB == 128, "block rows");
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
+    static_assert(128 * SOFTMAX_REGS + 256 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
 struct TcBars {
@@ -413,11 +420,11 @@ __global__ void __launch_bounds__(TcCfg<D, G>::THREADS, 2) tc_kernel(const TcPar
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < 3; ++s) {
-            mbar_init(smem_u32(&bars->kfull[s]), 32);
+            mbar_init(smem_u32(&bars->kfull[s]), 64);
             mbar_init(smem_u32(&bars->kempty[s]), 1);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&bars->vfull[s]), 32);
+            mbar_init(smem_u32(&bars->vfull[s]), 64);
             mbar_init(smem_u32(&bars->vempty[s]), 1);
             mbar_init(smem_u32(&bars->sfull[s]), 1);
             mbar_init(smem_u32(&bars->pready[s]), 4);
@@ -427,7 +434,7 @@ __global__ void __launch_bounds__(TcCfg<D, G>::THREADS, 2) tc_kernel(const TcPar
         bars->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 6) {
+    if (warp == 8) {
         tmem_alloc(smem_u32(&bars->tmem_base), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -435,12 +442,15 @@ __global__ void __launch_bounds__(TcCfg<D, G>::THREADS, 2) tc_kernel(const TcPar
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
+    if (warp >= 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
 
-    if (warp == 4 || warp == 5) {
+    if (warp >= 4 && warp < 8) {
         // ------------------------------------------------ K / V gather
-        // Warp 4: K rows (3 stages; the query rows with chunk 0), warp 5: V
-        // rows (2 stages).  The chunk's key list is loaded one chunk ahead.
-        const bool isK = warp == 4;
+        // Warps 4-5: K rows (3 stages; the query rows with chunk 0), warps
+        // 6-7: V rows (2 stages); the two warps of a role take alternate row
+        // pairs.  The chunk's key list is loaded one chunk ahead.
+        const bool isK = warp < 6;
+        const int pw = (warp - 4) & 1;
         const int nst = isK ? C::KST : C::VST;
         const __nv_bfloat16* src = isK ? p.K : p.V;
         const uint32_t tile0 = sb + (isK ? C::OFF_K : C::OFF_V);
@@ -448,7 +458,7 @@ __global__ void __launch_bounds__(TcCfg<D, G>::THREADS, 2) tc_kernel(const TcPar
         uint64_t* empty = isK ? bars->kempty : bars->vempty;
         const int rr = lane / PR, pc = lane % PR;
         if (isK && nch > 0) {
-            for (int m0 = 0; m0 < 128; m0 += RPI) {
+            for (int m0 = pw * RPI; m0 < 128; m0 += 2 * RPI) {
                 const int m = m0 + rr, j = m / G, h = m % G;
                 const bool ok = t0 + j < p.L;
                 const __nv_bfloat16* s =
@@ -476,7 +486,7 @@ __global__ void __launch_bounds__(TcCfg<D, G>::THREADS, 2) tc_kernel(const TcPar
             }
             const uint32_t tile = tile0 + s * C::KV_BYTES;
 #pragma unroll 4
-            for (int r0 = 0; r0 < kChunk; r0 += RPI) {
+            for (int r0 = pw * RPI; r0 < kChunk; r0 += 2 * RPI) {
                 const int r = r0 + rr;
                 const int32_t a = __shfl_sync(0xffffffffu, c0, r & 31);
                 const int32_t b = __shfl_sync(0xffffffffu, c1, r & 31);
@@ -488,7 +498,7 @@ __global__ void __launch_bounds__(TcCfg<D, G>::THREADS, 2) tc_kernel(const TcPar
             cp_async_arrive(smem_u32(&full[s]));
         }
         cp_async_wait_all();
-    } else if (warp == 6) {
+    } else if (warp == 8) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && nch > 0) {
             constexpr uint32_t idS = idesc_bf16(kChunk, false);
@@ -543,8 +553,9 @@ __global__ void __launch_bounds__(TcCfg<D, G>::THREADS, 2) tc_kernel(const TcPar
             mbar_wait_to(p.err, smem_u32(&bars->done), 0);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 4) {
         // ------------------------------------------------ softmax, row m
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
         const int m = warp * 32 + lane;
         const int j = m / G, h = m % G;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -666,7 +677,7 @@ __global__ void __launch_bounds__(TcCfg<D, G>::THREADS, 2) tc_kernel(const TcPar
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 6) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
